@@ -1,0 +1,238 @@
+"""Plain fp64 restatement of the MuonAdamW optimizer step (oracle).
+
+TEST INFRASTRUCTURE ONLY: imported by tests, the smoke check and the
+benchmark's CPU-baseline leg, never by the product path.
+
+Sources (page title, section):
+  [MAC]  "Chapter 4: The MuonAdamW Optimizer" -- sections "The Muon Update
+         Rule", "Polar Express: Newton-Schulz Orthogonalization", "The Full
+         Muon Step", "The AdamW Step".
+  [OPT]  "3.9 Optimizers: SGD, Adam, Adafactor, Lion, Muon & Shampoo" --
+         sections "From Gradient Descent to Momentum", "Implementing AdamW
+         from scratch", "Muon: Orthogonalizing the Update", "Exercises".
+  [NC]   "Stuck at the optimizer after figuring out backward()" (nanochat
+         discussion 856), reply by mira687: cautious weight decay mask,
+         per-step Polar Express coefficient table.
+  [RACE] "Muon vs AdamW, Lion and Sophia: a fair race", section "Muon".
+  [TAB]  "A transformer trained with Muon", section "The optimizer, Muon".
+
+Readings taken where the pages are silent or disagree are listed in the
+module-level notes of each function.
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+# [MAC] "Polar Express: Newton-Schulz Orthogonalization" and [OPT] "Muon:
+# Orthogonalizing the Update" both print this triple, used for every step.
+NS_COEFFS_FIXED: Tuple[float, float, float] = (3.4445, -4.7750, 2.0315)
+# [TAB] "The optimizer, Muon": the classical quintic with 15/8, -10/8, 3/8
+# converges to exactly 1.
+NS_COEFFS_CLASSICAL: Tuple[float, float, float] = (15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0)
+# [OPT] newton_schulz5(..., eps=1e-7); [MAC] adds 1e-7 to the norm.
+NS_EPS = 1e-7
+
+
+def _coeff_list(coeffs, steps: int):
+    """Per-step (a, b, c) list.  A single triple is repeated for every step;
+    a table with one row per step ([NC]: per-iteration Polar Express triples)
+    is used row by row."""
+    arr = np.asarray(coeffs, dtype=np.float64)
+    if arr.ndim == 1:
+        return [tuple(arr)] * steps
+    if arr.shape[0] < steps:
+        raise ValueError("coefficient table shorter than ns_steps")
+    return [tuple(row) for row in arr[:steps]]
+
+
+# ----------------------------------------------------------------------------
+# momentum
+# ----------------------------------------------------------------------------
+def nesterov_momentum(m: np.ndarray, g: np.ndarray, beta: float, nesterov: bool = True):
+    """Momentum buffer update and the matrix that gets orthogonalised.
+
+    [MAC] "The Muon Update Rule": m_t = beta*m_{t-1} + G_t, then the Nesterov
+    lookahead m~_t = beta*m_t + G_t.  [OPT] "Muon: Orthogonalizing the Update"
+    shows the heavy-ball form, which orthogonalises the buffer m_t itself.
+
+    Returns (m_new, matrix_to_orthogonalise).
+    """
+    m_new = beta * m + g
+    if nesterov:
+        return m_new, beta * m_new + g
+    return m_new, m_new.copy()
+
+
+# ----------------------------------------------------------------------------
+# Newton-Schulz / Polar Express
+# ----------------------------------------------------------------------------
+def frobenius_normalize(x: np.ndarray, eps: float = NS_EPS) -> np.ndarray:
+    """X0 = M / (||M||_F + eps)  ([MAC] "Polar Express ..."; [OPT] newton_schulz5).
+
+    The norm is the square root of the sum of squared entries ([RACE] "Muon").
+    eps is added to the norm, not to its square.
+    """
+    return x / (np.sqrt(np.sum(x * x)) + eps)
+
+
+def ns_polynomial(sigma, a: float, b: float, c: float):
+    """p(s) = a s + b s^3 + c s^5: what one iteration does to each singular value
+    ([MAC] "Why 5 Steps?"; [RACE] "Muon": 'on each singular value ... a step is a
+    polynomial')."""
+    s = np.asarray(sigma, dtype=np.float64)
+    return a * s + b * s ** 3 + c * s ** 5
+
+
+def ns_singular_value_map(sigma, coeffs=NS_COEFFS_FIXED, steps: int = 5):
+    """Compose the per-step scalar polynomials: p_k o ... o p_1 (sigma)."""
+    s = np.asarray(sigma, dtype=np.float64)
+    for a, b, c in _coeff_list(coeffs, steps):
+        s = ns_polynomial(s, a, b, c)
+    return s
+
+
+def newton_schulz(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: int = 5,
+                  eps: float = NS_EPS) -> np.ndarray:
+    """Quintic Newton-Schulz orthogonalisation of one matrix, in fp64.
+
+    Steps, in the order [MAC] "Polar Express: Newton-Schulz Orthogonalization"
+    gives them:
+      1. X = G / (||G||_F + eps)
+      2. if rows > cols, iterate on X^T (the smaller Gram product)
+      3. for each step k:  A = X X^T;  B = b_k A + c_k A A;  X = a_k X + B X
+      4. transpose back if step 2 transposed.
+    [OPT] transposes before normalising; the Frobenius norm is transpose
+    invariant, so the two orders agree.
+    """
+    x = frobenius_normalize(np.asarray(g, dtype=np.float64), eps)
+    transposed = x.shape[0] > x.shape[1]
+    if transposed:
+        x = x.T
+    for a, b, c in _coeff_list(coeffs, steps):
+        A = x @ x.T
+        B = b * A + c * (A @ A)
+        x = a * x + B @ x
+    if transposed:
+        x = x.T
+    return np.ascontiguousarray(x)
+
+
+def ns_closed_form(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: int = 5,
+                   eps: float = NS_EPS) -> np.ndarray:
+    """What the iteration must equal, written through an SVD.
+
+    Each step keeps the singular vectors and maps each singular value through
+    p ([MAC] "Why 5 Steps?", [RACE] "Muon", [TAB] "The optimizer, Muon").  So
+    NS(G) = U diag(p_k o ... o p_1 (s_i / (||G||_F + eps))) V^T with G = U S V^T.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    u, s, vt = np.linalg.svd(g, full_matrices=False)
+    scale = 1.0 / (np.sqrt(np.sum(g * g)) + eps)
+    return (u * ns_singular_value_map(s * scale, coeffs, steps)[None, :]) @ vt
+
+
+# ----------------------------------------------------------------------------
+# cautious weight decay + update
+# ----------------------------------------------------------------------------
+def cautious_mask(update: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """[NC]: decay only where the update and the parameter agree in sign,
+    mask = (update * param) >= 0.  A zero product (either factor +-0) keeps the
+    mask on.  Decided from the signs, which is what the product's sign is for
+    finite values, so no underflow of a tiny product can flip it."""
+    su = np.signbit(update)
+    sw = np.signbit(w)
+    return (su == sw) | (update == 0) | (w == 0)
+
+
+def cautious_weight_decay_update(w: np.ndarray, update: np.ndarray, lr: float, wd: float,
+                                 cautious: bool = True) -> np.ndarray:
+    """W <- W - lr * (U + wd * mask * W).
+
+    [MAC] "The Full Muon Step": decoupled decay p *= (1 - lr*wd) then the
+    update.  [NC] gates that decay with the cautious mask.  Reading: the decay
+    uses the pre-update W and the same lr as the update; without the cautious
+    flag the mask is all ones (plain decoupled decay).
+    """
+    mask = cautious_mask(update, w) if cautious else np.ones(w.shape, dtype=bool)
+    return w - lr * (update + wd * mask * w)
+
+
+def muon_step(w: np.ndarray, g: np.ndarray, m: np.ndarray, lr: float, beta: float, wd: float,
+              ns_steps: int = 5, coeffs=NS_COEFFS_FIXED, nesterov: bool = True,
+              cautious: bool = True, lr_scale: float = 1.0, eps: float = NS_EPS):
+    """One Muon step on one matrix: momentum -> NS -> cautious decay + update.
+
+    Returns (w_new, m_new, update) in fp64.  lr_scale is the per-matrix shape
+    factor some recipes multiply the learning rate by; 1 gives W -= lr*update.
+    """
+    m_new, mt = nesterov_momentum(m, g, beta, nesterov)
+    u = newton_schulz(mt, coeffs, ns_steps, eps)
+    w_new = cautious_weight_decay_update(w, u, lr * lr_scale, wd, cautious)
+    return w_new, m_new, u
+
+
+# ----------------------------------------------------------------------------
+# AdamW
+# ----------------------------------------------------------------------------
+def adamw_step(p: np.ndarray, g: np.ndarray, m: np.ndarray, v: np.ndarray, t: int,
+               lr: float, beta1: float, beta2: float, eps: float, wd: float):
+    """One AdamW step with bias correction, t >= 1.
+
+    [OPT] "Implementing AdamW from scratch" (and [MAC] "The AdamW Step"):
+      p <- p (1 - lr wd)                    decoupled decay, on the weights
+      m <- b1 m + (1 - b1) g
+      v <- b2 v + (1 - b2) g^2
+      p <- p - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+    Returns (p_new, m_new, v_new).
+    """
+    if t < 1:
+        raise ValueError("AdamW step count starts at 1")
+    p = p * (1.0 - lr * wd)
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    bc1 = 1.0 - beta1 ** t
+    bc2 = 1.0 - beta2 ** t
+    denom = np.sqrt(v) / np.sqrt(bc2) + eps
+    p = p - (lr / bc1) * m / denom
+    return p, m, v
+
+
+# ----------------------------------------------------------------------------
+# bf16 storage emulation (diagnostic only, never a parity gate)
+# ----------------------------------------------------------------------------
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to bfloat16 (nearest, ties to even) via fp32, returned as float64."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: int = 5,
+                                eps: float = NS_EPS) -> np.ndarray:
+    """The iteration with bf16 rounding wherever a bf16 matrix is stored.
+
+    [MAC] casts to bf16 before iterating and keeps X, A, B in bf16.  Storage
+    points here: X0 = bf16(M) with the 1/(||M||+eps) factor carried as a
+    scalar into the first Gram product and the first X update, A, B and each
+    new X; products are exact (fp64) between roundings.  Used to tell bf16
+    precision apart from kernel bugs; the gate is always the fp64 oracle.
+    """
+    g = np.asarray(g, dtype=np.float64)
+    s = 1.0 / (np.sqrt(np.sum(g * g)) + eps)
+    x = round_bf16(g)
+    transposed = x.shape[0] > x.shape[1]
+    if transposed:
+        x = x.T
+    for k, (a, b, c) in enumerate(_coeff_list(coeffs, steps)):
+        sk = s if k == 0 else 1.0
+        A = round_bf16(sk * sk * (x @ x.T))
+        B = round_bf16(b * A + c * (A @ A))
+        x = round_bf16(sk * (a * x + B @ x))
+    if steps == 0:
+        x = round_bf16(s * x)
+    if transposed:
+        x = x.T
+    return np.ascontiguousarray(x)
