@@ -1,0 +1,183 @@
+/*
+ * muon_b200.h -- C ABI of the B200 (sm_100a) Muon + AdamW optimizer step.
+ *
+ * The step (sources, by page title and section):
+ *   - "Chapter 4: The MuonAdamW Optimizer": The Muon Update Rule (Nesterov
+ *     momentum m = beta*m + G, lookahead m~ = beta*m + G); Polar Express:
+ *     Newton-Schulz Orthogonalization (X0 = m~/(||m~||_F + 1e-7), tall
+ *     matrices iterated as their transpose, A = X X^T, B = b*A + c*A*A,
+ *     X = a*X + B*X, five steps, (a,b,c) = (3.4445, -4.7750, 2.0315));
+ *     The AdamW Step.
+ *   - "Stuck at the optimizer after figuring out backward()" (nanochat
+ *     discussion, mira687's reply): cautious weight decay, decay only where
+ *     update * param >= 0; per-step coefficient tables.
+ *   - "3.9 Optimizers: SGD, Adam, Adafactor, Lion, Muon & Shampoo":
+ *     Implementing AdamW from scratch (bias-corrected AdamW with decoupled
+ *     decay); Muon: Orthogonalizing the Update (heavy-ball variant).
+ *
+ * Conventions for every entry point:
+ *   Ownership  All tensors and the workspace belong to the caller.  Pointer
+ *              arrays and descriptors are host memory, read only during the
+ *              call.  The library allocates no device memory.
+ *   Layout     Matrices are dense row-major (row pitch = cols elements).
+ *              params, momentum, exp_avg, exp_avg_sq are fp32; grads are
+ *              fp32 or bf16 as the group says.
+ *   In place   params, momentum, exp_avg and exp_avg_sq are updated in place;
+ *              grads are read only.
+ *   Async      Work is enqueued on `stream` (NULL = the legacy default
+ *              stream).  No host synchronisation and no device-to-host copy
+ *              happen inside muon_step / muon_orthogonalize / adamw_step.
+ *   Errors     Arguments are validated on the host before any launch; a
+ *              failed check returns a status and touches no tensor.
+ *              muon_last_error() gives a one-line reason.  Launch failures
+ *              return MUON_ERR_CUDA.  Device-side bounded waits that run out
+ *              record MUON_ERR_TIMEOUT in the workspace status word, read by
+ *              muon_query_status().
+ *   Threads    Entry points are reentrant; calls on different streams with
+ *              different workspaces may run concurrently.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t.  Declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st* muon_stream_t;
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, bad scalar, misaligned pointer */
+  MUON_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run (no sm_100 device, ...) */
+  MUON_ERR_WORKSPACE = 3,    /* workspace null, misaligned or smaller than muon_workspace_min_size */
+  MUON_ERR_CUDA = 4,         /* a CUDA runtime/driver call or kernel launch failed */
+  MUON_ERR_TIMEOUT = 5       /* a device-side bounded wait ran out (status word) */
+} muon_status;
+
+typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype;
+
+/* muon_step / muon_orthogonalize flags */
+enum {
+  MUON_NESTEROV = 1u,       /* orthogonalise beta*m + G (else m itself, heavy-ball) */
+  MUON_CAUTIOUS_WD = 2u,    /* decay only where update*param >= 0 (else plain decoupled decay) */
+  MUON_FP32_DEBUG = 4u,     /* fp32 operands and fp32 FMA GEMMs (slow; tolerance 1e-4 mode) */
+  MUON_UNFUSED_UPDATE = 8u  /* apply the update in its own kernel instead of the last B*X epilogue */
+};
+
+/*
+ * One shape group: `count` matrices of rows x cols (parameter orientation),
+ * the pointers params[first .. first+count-1] (same for grads, momentum).
+ * A group with rows > cols is iterated as its transpose ("Polar Express"
+ * orientation); no physical transpose is made: the kernels read it
+ * MN-major.
+ */
+typedef struct {
+  int32_t rows;
+  int32_t cols;
+  int32_t count;
+  int32_t first;
+  int32_t grad_dtype;  /* muon_dtype */
+  float lr_scale;      /* per-group learning-rate multiplier (1 => W -= lr*update) */
+} muon_group;
+
+/*
+ * Workspace bytes to run every matrix of `groups` in a single wave (fastest).
+ * muon_workspace_min_size: the least workspace muon_step accepts; with less
+ * than muon_workspace_size the matrices are processed in several waves.
+ * Returns 0 on invalid groups.  Host only, no CUDA call.
+ */
+size_t muon_workspace_size(const muon_group* groups, int n_groups, uint32_t flags);
+size_t muon_workspace_min_size(const muon_group* groups, int n_groups, uint32_t flags);
+
+/*
+ * One Muon step over every matrix of every group.
+ *
+ *   for each matrix:  m <- beta*m + G;   m~ <- beta*m + G  (MUON_NESTEROV) or m
+ *                     X0 <- m~ / (||m~||_F + 1e-7)
+ *                     ns_steps x { A = X X^T; B = b_k A + c_k A A; X = a_k X + B X }
+ *                     (wide orientation: rows > cols iterates on X^T)
+ *                     U  <- X (values rounded to bf16, as the pages keep X in bf16)
+ *                     W  <- W - lr*lr_scale*(U + wd*mask*W),
+ *                           mask = (U*W >= 0) with MUON_CAUTIOUS_WD, else 1
+ *
+ * params[i], momentum[i]: fp32 device, rows x cols, 16-byte aligned.
+ * grads[i]: device, rows x cols, dtype per group, 16-byte aligned.
+ * coeffs: host, ns_steps rows of (a, b, c); may be NULL only if ns_steps == 0.
+ * ns_steps in [0, 16].  beta in [0, 1).  lr, wd finite.
+ * workspace: device, 256-byte aligned, >= muon_workspace_min_size bytes; its
+ * contents need no initialisation and are scratch between calls.
+ * Two calls that share a workspace must be ordered (same stream).
+ */
+muon_status muon_step(float* const* params, const void* const* grads, float* const* momentum,
+                      const muon_group* groups, int n_groups,
+                      float lr, float beta, float wd, int ns_steps, const float* coeffs,
+                      uint32_t flags, void* workspace, size_t workspace_bytes,
+                      muon_stream_t stream);
+
+/*
+ * The orthogonaliser alone: outputs[i] <- NS(inputs[i]) as fp32, rows x cols,
+ * with the same normalisation, orientation, iteration and bf16 rounding of
+ * the result as muon_step.  inputs[i] dtype per group.  Only MUON_FP32_DEBUG
+ * is honoured in `flags`.
+ */
+muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs,
+                               const muon_group* groups, int n_groups,
+                               int ns_steps, const float* coeffs, uint32_t flags,
+                               void* workspace, size_t workspace_bytes, muon_stream_t stream);
+
+/*
+ * AdamW group ("3.9 Optimizers", Implementing AdamW from scratch), for t >= 1:
+ *   p <- p*(1 - lr*wd);  m <- b1*m + (1-b1)*g;  v <- b2*v + (1-b2)*g^2
+ *   p <- p - (lr/(1-b1^t)) * m / (sqrt(v)/sqrt(1-b2^t) + eps)
+ * params/exp_avg/exp_avg_sq fp32 device, grads fp32 or bf16 device, each
+ * tensor numel[i] >= 0 contiguous elements, 16-byte aligned.
+ * Per-group betas and lr carry per-role settings (embeddings, head, gains).
+ */
+typedef struct {
+  float* const* params;
+  const void* const* grads;
+  float* const* exp_avg;
+  float* const* exp_avg_sq;
+  const int64_t* numel;
+  int32_t count;
+  int32_t grad_dtype; /* muon_dtype */
+  float lr, beta1, beta2, eps, wd;
+} adamw_group;
+
+/* One fused AdamW step over all tensors of all groups (multi-tensor launches). */
+muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step,
+                       muon_stream_t stream);
+
+/*
+ * Synchronises `stream`, reads the workspace status word written by the
+ * device during the last muon_step / muon_orthogonalize on it, and returns
+ * MUON_OK or the recorded error (MUON_ERR_TIMEOUT).
+ */
+muon_status muon_query_status(const void* workspace, muon_stream_t stream);
+
+const char* muon_status_string(muon_status s);
+
+/* One-line description of the last failure on the calling thread ("" if none). */
+const char* muon_last_error(void);
+
+/*
+ * Optional per-kernel timing.  When enabled, every launch is bracketed by
+ * CUDA events on its own stream.  muon_profiler_read synchronises on those
+ * events and writes, per kernel kind, the summed device milliseconds and the
+ * launch count since the last reset; it returns the number of kinds.
+ */
+int muon_profiler_enable(int on);
+void muon_profiler_reset(void);
+int muon_profiler_read(double* ms_out, int64_t* launches_out, int max_kinds);
+int muon_kernel_kind_count(void);
+const char* muon_kernel_kind_name(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

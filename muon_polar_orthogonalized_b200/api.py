@@ -1,0 +1,144 @@
+"""Python binding of the C ABI: same names, torch tensors in, pointers out.
+
+Argument marshalling only: every step of the optimizer runs in the CUDA
+library.  Tensors must already live on the current CUDA device; streams are
+torch streams (default: the current stream).
+"""
+from __future__ import annotations
+
+import ctypes
+from ctypes import c_double, c_float, c_int64, c_void_p
+from typing import List, Optional, Sequence, Tuple
+
+from . import _native as N
+from ._native import AdamWGroup, MuonGroup, check
+
+GroupSpec = Tuple[int, int, int, int, int, float]  # rows, cols, count, first, grad_dtype, lr_scale
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _ptrs(tensors) -> ctypes.Array:
+    arr = (c_void_p * max(len(tensors), 1))()
+    for i, t in enumerate(tensors):
+        arr[i] = t if isinstance(t, int) else t.data_ptr()
+    return arr
+
+
+def make_groups(specs: Sequence) -> ctypes.Array:
+    arr = (MuonGroup * max(len(specs), 1))()
+    for i, s in enumerate(specs):
+        if isinstance(s, MuonGroup):
+            arr[i] = s
+        else:
+            r, c, n, first, dt, ls = s
+            arr[i] = MuonGroup(int(r), int(c), int(n), int(first), int(dt), float(ls))
+    return arr
+
+
+def _coeff_array(coeffs, ns_steps: int):
+    if ns_steps == 0:
+        return None
+    flat: List[float] = []
+    if len(coeffs) == 3 and not hasattr(coeffs[0], "__len__"):
+        flat = [float(x) for x in coeffs] * ns_steps
+    else:
+        for row in list(coeffs)[:ns_steps]:
+            flat.extend(float(x) for x in row)
+    arr = (c_float * len(flat))(*flat)
+    return arr
+
+
+def muon_workspace_size(groups: Sequence, flags: int = 0) -> int:
+    g = make_groups(groups)
+    return int(N.lib().muon_workspace_size(g, len(groups), flags))
+
+
+def muon_workspace_min_size(groups: Sequence, flags: int = 0) -> int:
+    g = make_groups(groups)
+    return int(N.lib().muon_workspace_min_size(g, len(groups), flags))
+
+
+def muon_step(params, grads, momentum, groups: Sequence, lr: float, beta: float, wd: float,
+              ns_steps: int, coeffs, flags: int, workspace, workspace_bytes: Optional[int] = None,
+              stream=None) -> None:
+    """One Muon step; see include/muon_b200.h.  params/grads/momentum are lists
+    of tensors (or raw pointers) in pointer-array order."""
+    g = make_groups(groups)
+    ca = _coeff_array(coeffs, ns_steps)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
+    st = N.lib().muon_step(_ptrs(params), _ptrs(grads), _ptrs(momentum), g, len(groups),
+                           float(lr), float(beta), float(wd), int(ns_steps), ca, int(flags),
+                           c_void_p(ws), wsb, c_void_p(_stream_handle(stream)))
+    check(st, "muon_step")
+
+
+def muon_orthogonalize(inputs, outputs, groups: Sequence, ns_steps: int, coeffs, flags: int,
+                       workspace, workspace_bytes: Optional[int] = None, stream=None) -> None:
+    g = make_groups(groups)
+    ca = _coeff_array(coeffs, ns_steps)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
+    st = N.lib().muon_orthogonalize(_ptrs(inputs), _ptrs(outputs), g, len(groups), int(ns_steps), ca,
+                                    int(flags), c_void_p(ws), wsb, c_void_p(_stream_handle(stream)))
+    check(st, "muon_orthogonalize")
+
+
+class AdamWSpec:
+    """One AdamW group: lists of tensors plus hyperparameters."""
+
+    def __init__(self, params, grads, exp_avg, exp_avg_sq, lr, beta1, beta2, eps, wd,
+                 grad_dtype: Optional[int] = None):
+        self.params, self.grads, self.exp_avg, self.exp_avg_sq = params, grads, exp_avg, exp_avg_sq
+        self.lr, self.beta1, self.beta2, self.eps, self.wd = lr, beta1, beta2, eps, wd
+        if grad_dtype is None:
+            import torch
+            grad_dtype = N.MUON_BF16 if (grads and grads[0].dtype == torch.bfloat16) else N.MUON_F32
+        self.grad_dtype = grad_dtype
+
+
+def adamw_step(groups: Sequence[AdamWSpec], step: int, stream=None) -> None:
+    n = len(groups)
+    arr = (AdamWGroup * max(n, 1))()
+    keep = []
+    for i, g in enumerate(groups):
+        p, gr, m, v = _ptrs(g.params), _ptrs(g.grads), _ptrs(g.exp_avg), _ptrs(g.exp_avg_sq)
+        numel = (c_int64 * max(len(g.params), 1))(*[t.numel() for t in g.params])
+        keep.extend([p, gr, m, v, numel])
+        arr[i] = AdamWGroup(ctypes.cast(p, ctypes.POINTER(c_void_p)),
+                            ctypes.cast(gr, ctypes.POINTER(c_void_p)),
+                            ctypes.cast(m, ctypes.POINTER(c_void_p)),
+                            ctypes.cast(v, ctypes.POINTER(c_void_p)),
+                            numel, len(g.params), int(g.grad_dtype), float(g.lr), float(g.beta1),
+                            float(g.beta2), float(g.eps), float(g.wd))
+    st = N.lib().adamw_step(arr, n, int(step), c_void_p(_stream_handle(stream)))
+    check(st, "adamw_step")
+
+
+def muon_query_status(workspace, stream=None) -> int:
+    ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
+    return int(N.lib().muon_query_status(c_void_p(ws), c_void_p(_stream_handle(stream))))
+
+
+# --------------------------------------------------------------- profiler
+def muon_profiler_enable(on: bool) -> bool:
+    return bool(N.lib().muon_profiler_enable(1 if on else 0))
+
+
+def muon_profiler_reset() -> None:
+    N.lib().muon_profiler_reset()
+
+
+def muon_profiler_read() -> dict:
+    """{kernel kind: (device ms summed, launches)} since the last reset."""
+    L = N.lib()
+    k = L.muon_kernel_kind_count()
+    ms = (c_double * k)()
+    cnt = (c_int64 * k)()
+    L.muon_profiler_read(ms, cnt, k)
+    return {L.muon_kernel_kind_name(i).decode(): (ms[i], int(cnt[i])) for i in range(k)}

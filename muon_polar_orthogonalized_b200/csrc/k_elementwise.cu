@@ -1,0 +1,382 @@
+// k_elementwise.cu -- the HBM-bound kernels of the Muon + AdamW step.
+//
+//   momentum_norm  m <- beta*m + G;  m~ <- beta*m + G (Nesterov) or m;
+//                  X0 <- m~ stored in the workspace (bf16, or fp32 in debug
+//                  mode) and one partial sum of m~^2 per block.
+//                  ("Chapter 4: The MuonAdamW Optimizer", The Muon Update Rule)
+//   norm_finalize  s <- 1 / (sqrt(sum of partials) + 1e-7), one block per
+//                  matrix, fixed summation order (deterministic).
+//                  ("Chapter 4", Polar Express: X / (||X|| + 1e-7))
+//   update         W <- W - lr*(U + wd*mask*W), mask = (U*W >= 0) by sign bits
+//                  (nanochat discussion, mira687's reply: cautious weight decay)
+//   emit           out <- U as fp32 (orthogonaliser entry point)
+//   adamw          bias-corrected AdamW with decoupled decay
+//                  ("3.9 Optimizers", Implementing AdamW from scratch)
+//
+// All of them stream: 16-byte vector accesses where the matrix allows it,
+// several independent loads in flight per thread, one chunk per block.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace muon {
+
+constexpr int kEltThreads = 256;
+constexpr int kEltUnroll = 8;                                // vec4 units per thread
+constexpr int kEltChunk = kEltThreads * kEltUnroll * 4;      // elements per block
+
+__device__ __forceinline__ int find_mat(const MatRef* mats, int n, int blk) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (mats[mid].blk_begin <= blk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float round_bf16(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// Load 4 consecutive gradient values as fp32.
+template <bool BF16>
+__device__ __forceinline__ float4 load_g4(const void* g, long long e) {
+  if constexpr (BF16) {
+    uint2 raw = __ldcs(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(g) + e));
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  } else {
+    return __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(g) + e));
+  }
+}
+template <bool BF16>
+__device__ __forceinline__ float load_g1(const void* g, long long e) {
+  if constexpr (BF16) return bf16_to_f(static_cast<const __nv_bfloat16*>(g)[e]);
+  else return static_cast<const float*>(g)[e];
+}
+
+__device__ __forceinline__ void store_x4(void* x, long long idx, float4 v, bool f32) {
+  if (f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(x) + idx) = v;
+  } else {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<uint32_t*>(&a);
+    raw.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(x) + idx) = raw;
+  }
+}
+__device__ __forceinline__ void store_x1(void* x, long long idx, float v, bool f32) {
+  if (f32) static_cast<float*>(x)[idx] = v;
+  else static_cast<__nv_bfloat16*>(x)[idx] = __float2bfloat16_rn(v);
+}
+__device__ __forceinline__ float4 load_x4(const void* x, long long idx, bool f32) {
+  if (f32) return *reinterpret_cast<const float4*>(static_cast<const float*>(x) + idx);
+  uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(x) + idx);
+  float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.x));
+  float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&raw.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float load_x1(const void* x, long long idx, bool f32) {
+  if (f32) return static_cast<const float*>(x)[idx];
+  return bf16_to_f(static_cast<const __nv_bfloat16*>(x)[idx]);
+}
+
+// Deterministic block sum (fixed shuffle tree, then warp 0 in order).
+__device__ __forceinline__ float block_sum(float v) {
+  __shared__ float red[kEltThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  if (w == 0) {
+    s = (l < kEltThreads / 32) ? red[l] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  }
+  return s;  // valid in thread 0
+}
+
+// ------------------------------------------------------------ momentum_norm
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads)
+momentum_norm_kernel(const __grid_constant__ EltParams p) {
+  const int blk = blockIdx.x;
+  const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
+  const long long numel = static_cast<long long>(r.rows) * r.cols;
+  const long long e0 = static_cast<long long>(blk - r.blk_begin) * kEltChunk;
+  const float beta = p.beta;
+  const bool f32x = p.x_f32 != 0;
+  float acc = 0.f;
+  if (r.vec) {
+    const int cols4 = r.cols >> 2;
+    float4 gv[kEltUnroll], mv[kEltUnroll];
+#pragma unroll
+    for (int u = 0; u < kEltUnroll; ++u) {
+      const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
+      if (e < numel) {
+        gv[u] = load_g4<GBF16>(r.g, e);
+        mv[u] = r.m ? *reinterpret_cast<const float4*>(r.m + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kEltUnroll; ++u) {
+      const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
+      if (e < numel) {
+        float4 mt;
+        if (r.m) {
+          float4 mn;
+          mn.x = fmaf(beta, mv[u].x, gv[u].x);
+          mn.y = fmaf(beta, mv[u].y, gv[u].y);
+          mn.z = fmaf(beta, mv[u].z, gv[u].z);
+          mn.w = fmaf(beta, mv[u].w, gv[u].w);
+          *reinterpret_cast<float4*>(r.m + e) = mn;
+          if (p.nesterov) {
+            mt.x = fmaf(beta, mn.x, gv[u].x);
+            mt.y = fmaf(beta, mn.y, gv[u].y);
+            mt.z = fmaf(beta, mn.z, gv[u].z);
+            mt.w = fmaf(beta, mn.w, gv[u].w);
+          } else {
+            mt = mn;
+          }
+        } else {
+          mt = gv[u];
+        }
+        acc = fmaf(mt.x, mt.x, acc);
+        acc = fmaf(mt.y, mt.y, acc);
+        acc = fmaf(mt.z, mt.z, acc);
+        acc = fmaf(mt.w, mt.w, acc);
+        const long long q = e >> 2;
+        const long long row = q / cols4;
+        const long long col = (q - row * cols4) * 4;
+        store_x4(r.x, row * r.ldx + col, mt, f32x);
+      }
+    }
+  } else {
+    for (int u = 0; u < kEltUnroll * 4; ++u) {
+      const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
+      if (e < numel) {
+        const float g = load_g1<GBF16>(r.g, e);
+        float mt = g;
+        if (r.m) {
+          const float mn = fmaf(beta, r.m[e], g);
+          r.m[e] = mn;
+          mt = p.nesterov ? fmaf(beta, mn, g) : mn;
+        }
+        acc = fmaf(mt, mt, acc);
+        const long long row = e / r.cols;
+        const long long col = e - row * r.cols;
+        store_x1(r.x, row * r.ldx + col, mt, f32x);
+      }
+    }
+  }
+  const float s = block_sum(acc);
+  if (threadIdx.x == 0) p.partials[blk] = s;
+}
+
+// ------------------------------------------------------------ norm_finalize
+__global__ void __launch_bounds__(kEltThreads)
+norm_finalize_kernel(const __grid_constant__ EltParams p) {
+  const MatRef& r = p.mats[blockIdx.x];
+  const long long numel = static_cast<long long>(r.rows) * r.cols;
+  const int nblk = static_cast<int>((numel + kEltChunk - 1) / kEltChunk);
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nblk; i += kEltThreads) acc += p.partials[r.blk_begin + i];
+  __shared__ double red[kEltThreads];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = kEltThreads / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.scales[r.sidx] = static_cast<float>(1.0 / (sqrt(red[0]) + 1e-7));
+}
+
+// --------------------------------------------------------- update / emit
+// U = X (bf16 values, or fp32 in debug mode), times the matrix scale when no
+// Newton-Schulz step ran; the bf16 path rounds that product to bf16 as the
+// pages' bf16 X would be.
+__device__ __forceinline__ float cautious_apply(float w, float u, float lr, float wd,
+                                                bool cautious) {
+  // mask = (u*w >= 0) decided from sign bits: equal signs, or either is zero
+  bool mask = true;
+  if (cautious) {
+    const bool sdiff = (__float_as_uint(u) ^ __float_as_uint(w)) >> 31;
+    mask = !sdiff || u == 0.f || w == 0.f;
+  }
+  const float t = mask ? fmaf(wd, w, u) : u;
+  return fmaf(-lr, t, w);
+}
+
+template <bool EMIT>
+__global__ void __launch_bounds__(kEltThreads)
+update_kernel(const __grid_constant__ EltParams p) {
+  const int blk = blockIdx.x;
+  const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
+  const long long numel = static_cast<long long>(r.rows) * r.cols;
+  const long long e0 = static_cast<long long>(blk - r.blk_begin) * kEltChunk;
+  const bool f32x = p.x_f32 != 0;
+  const float sc = p.use_scale ? p.scales[r.sidx] : 1.f;
+  auto make_u = [&](float x) {
+    if (!p.use_scale) return x;
+    return f32x ? sc * x : round_bf16(sc * x);
+  };
+  if (r.vec) {
+    const int cols4 = r.cols >> 2;
+    float4 xv[kEltUnroll], wv[kEltUnroll];
+#pragma unroll
+    for (int u = 0; u < kEltUnroll; ++u) {
+      const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
+      if (e < numel) {
+        const long long q = e >> 2;
+        const long long row = q / cols4;
+        const long long col = (q - row * cols4) * 4;
+        xv[u] = load_x4(r.x, row * r.ldx + col, f32x);
+        if (!EMIT) wv[u] = *reinterpret_cast<const float4*>(r.w + e);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kEltUnroll; ++u) {
+      const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
+      if (e < numel) {
+        float4 uu = make_float4(make_u(xv[u].x), make_u(xv[u].y), make_u(xv[u].z), make_u(xv[u].w));
+        if (EMIT) {
+          __stcs(reinterpret_cast<float4*>(r.out + e), uu);
+        } else {
+          float4 w = wv[u];
+          w.x = cautious_apply(w.x, uu.x, r.lr, p.wd, p.cautious);
+          w.y = cautious_apply(w.y, uu.y, r.lr, p.wd, p.cautious);
+          w.z = cautious_apply(w.z, uu.z, r.lr, p.wd, p.cautious);
+          w.w = cautious_apply(w.w, uu.w, r.lr, p.wd, p.cautious);
+          *reinterpret_cast<float4*>(r.w + e) = w;
+        }
+      }
+    }
+  } else {
+    for (int u = 0; u < kEltUnroll * 4; ++u) {
+      const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
+      if (e < numel) {
+        const long long row = e / r.cols;
+        const long long col = e - row * r.cols;
+        const float uu = make_u(load_x1(r.x, row * r.ldx + col, f32x));
+        if (EMIT) r.out[e] = uu;
+        else r.w[e] = cautious_apply(r.w[e], uu, r.lr, p.wd, p.cautious);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ AdamW
+__device__ __forceinline__ int find_tensor(const AdamTensor* t, int n, int blk) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (t[mid].blk_begin <= blk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void adam_elem(const AdamTensor& T, float g, float& p, float& m,
+                                          float& v) {
+  p = p * T.decay;
+  m = fmaf(T.b1, m, T.omb1 * g);
+  v = fmaf(T.b2, v, T.omb2 * (g * g));
+  const float denom = sqrtf(v) / T.sqrt_bc2 + T.eps;
+  p = fmaf(-T.step_size, m / denom, p);
+}
+
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads)
+adamw_kernel(const __grid_constant__ AdamParams P) {
+  const int blk = blockIdx.x;
+  const AdamTensor& T = P.t[find_tensor(P.t, P.ntensors, blk)];
+  const long long e0 = static_cast<long long>(blk - T.blk_begin) * kEltChunk;
+  if (T.vec) {
+    constexpr int U = kEltUnroll / 2;  // 4 streams per element: keep registers in check
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      float4 gv[U], pv[U], mv[U], vv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const long long e =
+            e0 + (static_cast<long long>(half * U + u) * kEltThreads + threadIdx.x) * 4;
+        if (e < T.numel) {
+          gv[u] = load_g4<GBF16>(T.g, e);
+          pv[u] = *reinterpret_cast<const float4*>(T.p + e);
+          mv[u] = *reinterpret_cast<const float4*>(T.m + e);
+          vv[u] = *reinterpret_cast<const float4*>(T.v + e);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const long long e =
+            e0 + (static_cast<long long>(half * U + u) * kEltThreads + threadIdx.x) * 4;
+        if (e < T.numel) {
+          adam_elem(T, gv[u].x, pv[u].x, mv[u].x, vv[u].x);
+          adam_elem(T, gv[u].y, pv[u].y, mv[u].y, vv[u].y);
+          adam_elem(T, gv[u].z, pv[u].z, mv[u].z, vv[u].z);
+          adam_elem(T, gv[u].w, pv[u].w, mv[u].w, vv[u].w);
+          *reinterpret_cast<float4*>(T.p + e) = pv[u];
+          *reinterpret_cast<float4*>(T.m + e) = mv[u];
+          *reinterpret_cast<float4*>(T.v + e) = vv[u];
+        }
+      }
+    }
+  } else {
+    for (int u = 0; u < kEltUnroll * 4; ++u) {
+      const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
+      if (e < T.numel) {
+        float pp = T.p[e], mm = T.m[e], vv = T.v[e];
+        adam_elem(T, load_g1<GBF16>(T.g, e), pp, mm, vv);
+        T.p[e] = pp;
+        T.m[e] = mm;
+        T.v[e] = vv;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- launchers
+int elt_chunk() { return kEltChunk; }
+
+cudaError_t launch_momentum_norm(const EltParams& p, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  if (p.grad_bf16)
+    momentum_norm_kernel<true><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  else
+    momentum_norm_kernel<false><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s) {
+  if (p.nmats <= 0) return cudaSuccess;
+  norm_finalize_kernel<<<p.nmats, kEltThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_update(const EltParams& p, bool emit, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  if (emit)
+    update_kernel<true><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  else
+    update_kernel<false><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_adamw(const AdamParams& p, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  if (p.grad_bf16)
+    adamw_kernel<true><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  else
+    adamw_kernel<false><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

@@ -1,0 +1,420 @@
+// k_gemm_tc.cu -- the Newton-Schulz GEMMs on the 5th-generation tensor cores.
+//
+// One quintic iteration ("Chapter 4: The MuonAdamW Optimizer", Polar Express:
+// Newton-Schulz Orthogonalization; "3.9 Optimizers", Muon: Orthogonalizing
+// the Update) is three products:
+//   gram  A = s^2 X X^T          symmetric: only tiles touching the upper
+//                                triangle run; off-diagonal blocks are also
+//                                stored transposed (mirrored)
+//   poly  B = b A + c A A        symmetric likewise; A A = A A^T since A is
+//                                symmetric, so both operands are rows of A;
+//                                the epilogue reads the A tile for b*A
+//   axpy  X' = s (a X + B X)     wide matrices; tall ones (iterated as X^T)
+//                                compute X' = s (a X + X B) in parameter layout
+//   axpy_update                  last iteration: U = bf16(X') feeds the
+//                                cautious-decay update of W directly
+// s is the Frobenius scale 1/(||m~||+1e-7), applied on the first iteration
+// only (X0 is stored unscaled; bf16 rounding is scale-free up to exponent).
+//
+// Structure: persistent grouped kernel, one CTA per SM, 128x256 output tiles,
+// BK = 64, 4-stage TMA -> shared-memory ring, tcgen05.mma kind::f16 (bf16 in,
+// fp32 accumulate) issued by one thread into a double-buffered TMEM
+// accumulator (2 x 256 columns), and four epilogue warps that drain TMEM with
+// tcgen05.ld while the next tile's MMAs run.
+//   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
+//   warps 2-5: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31)
+// No multicast is used anywhere.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace muon {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 256;
+constexpr int TC_BK = 64;
+constexpr int TC_STAGES = 4;
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;   // 16 KB
+constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;   // 32 KB
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
+constexpr int TC_THREADS = 192;
+constexpr int TC_TMEM_COLS = 512;
+constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+constexpr int TC_RASTER_GN = 8;   // tile-column band width of the non-symmetric raster
+
+struct TileCoord {
+  int prob, mat, tm, tn;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
+  int pi = 0;
+  while (pi + 1 < p.nprob && t >= p.prob[pi + 1].tile_begin) ++pi;
+  const GemmProblem& q = p.prob[pi];
+  int lt = t - q.tile_begin;
+  const int mat = lt / q.tiles_per_mat;
+  int r = lt - mat * q.tiles_per_mat;
+  int tm, tn;
+  if (q.sym) {
+    int I = 0;
+    for (;;) {
+      const int cnt = q.tiles_n - (I >> 1);
+      if (r < cnt) break;
+      r -= cnt;
+      ++I;
+    }
+    tm = I;
+    tn = (I >> 1) + r;
+  } else {
+    const int band_tiles = q.tiles_m * TC_RASTER_GN;
+    const int band = r / band_tiles;
+    const int rem = r - band * band_tiles;
+    const int width = min(TC_RASTER_GN, q.tiles_n - band * TC_RASTER_GN);
+    tm = rem / width;
+    tn = band * TC_RASTER_GN + (rem - (rem / width) * width);
+  }
+  return {pi, mat, tm, tn};
+}
+
+__device__ __forceinline__ void record_timeout(unsigned int* status, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicOr(status, kDevTimeout);
+}
+
+// 32 consecutive bf16 -> fp32 (16-byte loads; address 16-byte aligned).
+__device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 raw = s4[q];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+      v[q * 8 + h * 2] = f.x;
+      v[q * 8 + h * 2 + 1] = f.y;
+    }
+  }
+}
+__device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(v[q * 8 + h * 2], v[q * 8 + h * 2 + 1]);
+      w[h] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+__device__ __forceinline__ float cautious_w(float w, float u, float lr, float wd, bool cautious) {
+  bool mask = true;
+  if (cautious) {
+    const bool sdiff = (__float_as_uint(u) ^ __float_as_uint(w)) >> 31;
+    mask = !sdiff || u == 0.f || w == 0.f;
+  }
+  const float t = mask ? fmaf(wd, w, u) : u;
+  return fmaf(-lr, t, w);
+}
+
+// Epilogue for one 32-column chunk held by this thread (row i, cols j0..j0+31).
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const TcGemmParams& p, const GemmProblem& q,
+                                               int mat, int i, int j0, bool mirror,
+                                               float (&v)[32]) {
+  if (i >= q.M) return;
+  const bool full = (j0 + 32 <= q.N);
+  float f = 1.f;
+  if (q.scale_mode) {
+    const float s = p.scales[q.scale_base + mat];
+    f = (q.scale_mode == 1) ? s * s : s;
+  }
+  if constexpr (EPI == EPI_GRAM) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] *= f;
+  } else if constexpr (EPI == EPI_POLY) {
+    const __nv_bfloat16* ein =
+        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0;
+    float a[32];
+    if (full) {
+      ld_bf16x32(ein, a);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) a[c] = (j0 + c < q.N) ? __bfloat162float(ein[c]) : 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]);
+  } else {  // AXPY, AXPY_UPDATE
+    const __nv_bfloat16* ein =
+        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0;
+    float x[32];
+    if (full) {
+      ld_bf16x32(ein, x);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = (j0 + c < q.N) ? __bfloat162float(ein[c]) : 0.f;
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = f * fmaf(q.ca, x[c], v[c]);
+  }
+
+  if constexpr (EPI == EPI_AXPY_UPDATE) {
+    const int wi = q.w_first + mat;
+    float* w = p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0;
+    const bool cautious = p.cautious != 0;
+    if (full && ((reinterpret_cast<uintptr_t>(w) & 15u) == 0)) {
+      float4* w4 = reinterpret_cast<float4*>(w);
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        float4 ww = w4[c4];
+        ww.x = cautious_w(ww.x, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 0])), q.lr, p.wd, cautious);
+        ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), q.lr, p.wd, cautious);
+        ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), q.lr, p.wd, cautious);
+        ww.w = cautious_w(ww.w, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 3])), q.lr, p.wd, cautious);
+        w4[c4] = ww;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (j0 + c < q.N)
+          w[c] = cautious_w(w[c], __bfloat162float(__float2bfloat16_rn(v[c])), q.lr, p.wd, cautious);
+    }
+  } else {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(q.out) + mat * q.out_bs;
+    __nv_bfloat16* row = out + static_cast<long long>(i) * q.out_ld + j0;
+    if (full) {
+      st_bf16x32(row, v);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (j0 + c < q.N) row[c] = __float2bfloat16_rn(v[c]);
+    }
+    if (mirror) {
+      // out[j][i] for this thread's 32 columns; lanes hold consecutive i, so
+      // each of these stores is one coalesced 64-byte run across the warp.
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (j0 + c < q.N) out[static_cast<long long>(j0 + c) * q.out_ld + i] = __float2bfloat16_rn(v[c]);
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + TC_STAGES * TC_STAGE_BYTES);
+  uint64_t* empty_bar = full_bar + TC_STAGES;
+  uint64_t* tfull_bar = empty_bar + TC_STAGES;   // [2]
+  uint64_t* tempty_bar = tfull_bar + 2;          // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      sm100::mbar_init(&full_bar[s], 1);
+      sm100::mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      sm100::mbar_init(&tfull_bar[b], 1);
+      sm100::mbar_init(&tempty_bar[b], 128);
+    }
+    *abort_flag = 0;
+    sm100::fence_mbar_init();
+    for (int i = 0; i < p.nprob; ++i) {
+      sm100::prefetch_tmap(&p.tmA[i]);
+      sm100::prefetch_tmap(&p.tmB[i]);
+    }
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(tmem_slot, TC_TMEM_COLS);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase_mask = 0;  // per stage: loads issued / their phase
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = decode_tile(p, t);
+        const GemmProblem& q = p.prob[tc.prob];
+        const int kblocks = (q.K + TC_BK - 1) / TC_BK;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!sm100::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
+            record_timeout(p.status, abort_flag);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * TC_STAGE_BYTES;
+          uint8_t* sb = sa + TC_A_BYTES;
+          sm100::mbar_arrive_expect_tx(&full_bar[stage], TC_STAGE_BYTES);
+          issued_mask |= 1u << stage;
+          issued_phase_mask = (issued_phase_mask & ~(1u << stage)) | (phase << stage);
+          const int k0 = kb * TC_BK;
+          if (!q.a_mn) {
+            sm100::tma_load_3d(sa, &p.tmA[tc.prob], &full_bar[stage], k0, tc.tm * TC_BM, tc.mat);
+          } else {
+#pragma unroll
+            for (int h = 0; h < TC_BM / 64; ++h)
+              sm100::tma_load_3d(sa + h * 8192, &p.tmA[tc.prob], &full_bar[stage], tc.tm * TC_BM + h * 64, k0, tc.mat);
+          }
+          if (!q.b_mn) {
+            sm100::tma_load_3d(sb, &p.tmB[tc.prob], &full_bar[stage], k0, tc.tn * TC_BN, tc.mat);
+          } else {
+#pragma unroll
+            for (int h = 0; h < TC_BN / 64; ++h)
+              sm100::tma_load_3d(sb + h * 8192, &p.tmB[tc.prob], &full_bar[stage], tc.tn * TC_BN + h * 64, k0, tc.mat);
+          }
+          if (++stage == TC_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: let every load this thread issued land before the CTA exits
+        for (int s = 0; s < TC_STAGES; ++s) {
+          if (!((issued_mask >> s) & 1u)) continue;
+          const uint64_t t0 = sm100::globaltimer();
+          while (!sm100::mbar_try_wait(&full_bar[s], (issued_phase_mask >> s) & 1u) &&
+                 sm100::globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = decode_tile(p, t);
+        const GemmProblem& q = p.prob[tc.prob];
+        const int kblocks = (q.K + TC_BK - 1) / TC_BK;
+        const uint32_t idesc = sm100::make_idesc_bf16(TC_BM, TC_BN, q.a_mn, q.b_mn);
+        if (!sm100::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) {
+          record_timeout(p.status, abort_flag);
+          break;
+        }
+        sm100::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TC_BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!sm100::mbar_wait(&full_bar[stage], phase, abort_flag)) {
+            record_timeout(p.status, abort_flag);
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t sa = sm100::smem_u32(smem + stage * TC_STAGE_BYTES);
+          const uint32_t sb = sa + TC_A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint64_t ad = q.a_mn ? sm100::make_sdesc(sa + kk * 2048, 8192, 1024)
+                                       : sm100::make_sdesc(sa + kk * 32, 16, 1024);
+            const uint64_t bd = q.b_mn ? sm100::make_sdesc(sb + kk * 2048, 8192, 1024)
+                                       : sm100::make_sdesc(sb + kk * 32, 16, 1024);
+            sm100::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+          }
+          sm100::umma_commit(&empty_bar[stage]);
+          if (++stage == TC_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        sm100::umma_commit(&tfull_bar[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+      const TileCoord tc = decode_tile(p, t);
+      const GemmProblem& q = p.prob[tc.prob];
+      if (!sm100::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
+        record_timeout(p.status, abort_flag);
+        break;
+      }
+      sm100::tc_fence_after();
+      const int i = tc.tm * TC_BM + row_in_tile;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(acc * TC_BN);
+#pragma unroll 1
+      for (int c = 0; c < TC_BN / 32; ++c) {
+        const int j0 = tc.tn * TC_BN + c * 32;
+        if (j0 >= q.N) break;  // warp-uniform
+        bool mirror = false;
+        if (q.sym) {
+          const int jb = j0 / TC_BM;        // 128-wide column block
+          if (jb < tc.tm) continue;         // strictly lower block: produced by its mirror
+          mirror = jb > tc.tm;
+        }
+        float v[32];
+        sm100::tmem_ld32(t_row + static_cast<uint32_t>(c * 32), v);
+        epilogue_chunk<EPI>(p, q, tc.mat, i, j0, mirror, v);
+      }
+      sm100::tc_fence_before();
+      sm100::mbar_arrive(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    sm100::tmem_dealloc(tmem_base, TC_TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- launcher
+int tc_tile_m() { return TC_BM; }
+int tc_tile_n() { return TC_BN; }
+
+template <int EPI>
+static cudaError_t launch_tc_epi(const TcGemmParams& p, int grid, cudaStream_t s) {
+  auto kern = tc_gemm_kernel<EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, TC_THREADS, TC_SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, int num_sms, cudaStream_t s) {
+  if (p.total_tiles <= 0) return cudaSuccess;
+  const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
+  switch (epi) {
+    case EPI_GRAM: return launch_tc_epi<EPI_GRAM>(p, grid, s);
+    case EPI_POLY: return launch_tc_epi<EPI_POLY>(p, grid, s);
+    case EPI_AXPY: return launch_tc_epi<EPI_AXPY>(p, grid, s);
+    case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE>(p, grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace muon

@@ -1,0 +1,102 @@
+"""MuonAdamW: the hybrid optimizer over two disjoint parameter sets.
+
+Hidden 2-D weight matrices go to Muon; embeddings, the LM head, norm gains
+and biases go to AdamW ("Chapter 4: The MuonAdamW Optimizer", Parameter
+Dispatch; "3.9 Optimizers", Wiring the hybrid recipe).  The caller decides
+the split.  This class only owns the state tensors (momentum, exp_avg,
+exp_avg_sq, the step count), groups matrices by shape, and calls the C ABI;
+all arithmetic runs in the CUDA library.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Optional, Sequence
+
+import torch
+
+from . import _native as N
+from . import api
+
+DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
+
+
+class MuonAdamW:
+    def __init__(self, muon_params: Sequence[torch.Tensor], adamw_groups: Sequence[Dict] = (),
+                 lr: float = 0.02, momentum: float = 0.95, weight_decay: float = 0.01,
+                 ns_steps: int = 5, coeffs=DEFAULT_COEFFS, nesterov: bool = True,
+                 cautious: bool = True, lr_scale_fn=None, fp32_debug: bool = False,
+                 fused_update: bool = True, workspace_bytes: Optional[int] = None):
+        """muon_params: fp32 2-D CUDA tensors.  adamw_groups: dicts with keys
+        params, lr, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.  lr_scale_fn:
+        optional (rows, cols) -> float learning-rate multiplier per shape."""
+        self.lr, self.beta, self.wd = lr, momentum, weight_decay
+        self.ns_steps, self.coeffs = ns_steps, coeffs
+        self.flags = ((N.MUON_NESTEROV if nesterov else 0) | (N.MUON_CAUTIOUS_WD if cautious else 0)
+                      | (N.MUON_FP32_DEBUG if fp32_debug else 0)
+                      | (0 if fused_update else N.MUON_UNFUSED_UPDATE))
+        # shape groups: matrices with equal (rows, cols) are contiguous in the pointer arrays
+        order: Dict[tuple, List[torch.Tensor]] = {}
+        for p in muon_params:
+            if p.dim() != 2 or p.dtype != torch.float32 or not p.is_cuda or not p.is_contiguous():
+                raise ValueError("Muon parameters must be contiguous fp32 2-D CUDA tensors")
+            order.setdefault(tuple(p.shape), []).append(p)
+        self.muon_params: List[torch.Tensor] = []
+        self._shapes = []
+        for (r, c), ps in order.items():
+            self._shapes.append((r, c, len(ps), len(self.muon_params),
+                                 float(lr_scale_fn(r, c)) if lr_scale_fn else 1.0))
+            self.muon_params.extend(ps)
+        self.momentum = [torch.zeros_like(p) for p in self.muon_params]
+        self.adamw_groups = []
+        for g in adamw_groups:
+            ps = list(g["params"])
+            self.adamw_groups.append(dict(
+                params=ps, lr=g.get("lr", 3e-4), betas=g.get("betas", (0.9, 0.95)),
+                eps=g.get("eps", 1e-8), weight_decay=g.get("weight_decay", 0.0),
+                exp_avg=[torch.zeros_like(p) for p in ps],
+                exp_avg_sq=[torch.zeros_like(p) for p in ps]))
+        self.step_count = 0
+        ws_need = api.muon_workspace_size(self._groups(torch.float32), self.flags) if self.muon_params else 0
+        nbytes = ws_need if workspace_bytes is None else max(int(workspace_bytes), 0)
+        dev = self.muon_params[0].device if self.muon_params else torch.device("cuda")
+        self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+
+    def _groups(self, grad_dtype):
+        dt = N.MUON_BF16 if grad_dtype == torch.bfloat16 else N.MUON_F32
+        return [(r, c, n, first, dt, ls) for (r, c, n, first, ls) in self._shapes]
+
+    @torch.no_grad()
+    def step(self, stream=None) -> None:
+        self.step_count += 1
+        if self.muon_params:
+            grads = [p.grad for p in self.muon_params]
+            if any(g is None for g in grads):
+                raise ValueError("every Muon parameter needs a .grad")
+            gd = grads[0].dtype
+            if any(g.dtype != gd for g in grads):
+                raise ValueError("Muon grads must share one dtype")
+            api.muon_step(self.muon_params, grads, self.momentum, self._groups(gd), self.lr,
+                          self.beta, self.wd, self.ns_steps, self.coeffs, self.flags,
+                          self.workspace, stream=stream)
+        specs = []
+        for g in self.adamw_groups:
+            grads = [p.grad for p in g["params"]]
+            specs.append(api.AdamWSpec(g["params"], grads, g["exp_avg"], g["exp_avg_sq"], g["lr"],
+                                       g["betas"][0], g["betas"][1], g["eps"], g["weight_decay"]))
+        if specs:
+            api.adamw_step(specs, self.step_count, stream=stream)
+
+    def state_dict(self) -> dict:
+        return {"step": self.step_count,
+                "momentum": [m.clone() for m in self.momentum],
+                "exp_avg": [[t.clone() for t in g["exp_avg"]] for g in self.adamw_groups],
+                "exp_avg_sq": [[t.clone() for t in g["exp_avg_sq"]] for g in self.adamw_groups]}
+
+    def load_state_dict(self, sd: dict) -> None:
+        self.step_count = int(sd["step"])
+        for dst, src in zip(self.momentum, sd["momentum"]):
+            dst.copy_(src)
+        for g, ea, es in zip(self.adamw_groups, sd["exp_avg"], sd["exp_avg_sq"]):
+            for dst, src in zip(g["exp_avg"], ea):
+                dst.copy_(src)
+            for dst, src in zip(g["exp_avg_sq"], es):
+                dst.copy_(src)

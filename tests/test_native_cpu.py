@@ -1,0 +1,130 @@
+"""Host-side checks of the native library; no GPU work is launched.
+
+  * the library loads and exports every function include/muon_b200.h declares;
+  * the ctypes structs have the C layout;
+  * argument validation rejects bad calls before any CUDA call;
+  * workspace sizing is consistent.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from muon_polar_orthogonalized_b200 import _native as N
+from muon_polar_orthogonalized_b200 import api
+from muon_polar_orthogonalized_b200.build import LIB_PATH, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return N.lib()
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+\**([a-z_][a-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_entry_points():
+    names = header_functions()
+    for must in ("muon_step", "adamw_step", "muon_orthogonalize", "muon_workspace_size",
+                 "muon_query_status", "muon_status_string"):
+        assert must in names
+    assert set(names) == set(N.SIGNATURES), set(names) ^ set(N.SIGNATURES)
+
+
+def test_library_exports_every_header_symbol(L):
+    out = os.popen(f"nm -D --defined-only {LIB_PATH}").read()
+    exported = set(re.findall(r" T (\w+)$", out, flags=re.M))
+    for name in header_functions():
+        assert name in exported, name
+        assert getattr(L, name) is not None
+
+
+def test_struct_layouts():
+    assert ctypes.sizeof(N.MuonGroup) == 24
+    assert N.AdamWGroup.count.offset == 40 and N.AdamWGroup.lr.offset == 48
+    assert ctypes.sizeof(N.AdamWGroup) == 72
+
+
+def test_status_strings(L):
+    for code, name in [(0, "MUON_OK"), (1, "MUON_ERR_INVALID_ARG"), (3, "MUON_ERR_WORKSPACE"),
+                       (5, "MUON_ERR_TIMEOUT")]:
+        assert N.status_string(code) == name
+
+
+def _call_step(L, groups, ptr_count, ns=5, coeffs=True, flags=3, ws=0x1000, wsb=1 << 40,
+               beta=0.95, lr=0.02, ptr=0x10000):
+    g = api.make_groups(groups)
+    arr = (ctypes.c_void_p * max(ptr_count, 1))(*([ptr] * ptr_count))
+    ca = (ctypes.c_float * 48)(*([1.0] * 48)) if coeffs else None
+    return L.muon_step(arr, arr, arr, g, len(groups), lr, beta, 0.01, ns, ca, flags,
+                       ctypes.c_void_p(ws), wsb, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(groups=[(0, 4, 1, 0, 0, 1.0)]), N.MUON_ERR_INVALID_ARG),          # rows 0
+    (dict(groups=[(4, 4, 1, 0, 7, 1.0)]), N.MUON_ERR_INVALID_ARG),          # dtype
+    (dict(groups=[(4, 4, 1, 0, 0, float("nan"))]), N.MUON_ERR_INVALID_ARG),  # lr_scale
+    (dict(groups=[(70000, 4, 1, 0, 0, 1.0)]), N.MUON_ERR_INVALID_ARG),      # too large
+    (dict(ns=17), N.MUON_ERR_INVALID_ARG),
+    (dict(ns=-1), N.MUON_ERR_INVALID_ARG),
+    (dict(coeffs=False), N.MUON_ERR_INVALID_ARG),
+    (dict(flags=64), N.MUON_ERR_INVALID_ARG),
+    (dict(ws=0), N.MUON_ERR_WORKSPACE),
+    (dict(ws=0x1010), N.MUON_ERR_WORKSPACE),                                 # misaligned
+    (dict(wsb=100), N.MUON_ERR_WORKSPACE),
+    (dict(beta=1.0), N.MUON_ERR_INVALID_ARG),
+    (dict(lr=float("inf")), N.MUON_ERR_INVALID_ARG),
+    (dict(ptr=0), N.MUON_ERR_INVALID_ARG),                                   # NULL tensor
+    (dict(ptr=0x10008), N.MUON_ERR_INVALID_ARG),                             # misaligned tensor
+])
+def test_muon_step_validation(L, case, expect):
+    groups = case.pop("groups", [(64, 128, 2, 0, 0, 1.0)])
+    st = _call_step(L, groups, 2, **case)
+    assert st == expect, N.last_error()
+    assert N.last_error() != ""
+
+
+def test_adamw_validation(L):
+    p = (ctypes.c_void_p * 1)(0x10000)
+    n = (ctypes.c_int64 * 1)(16)
+    g = N.AdamWGroup(p, p, p, p, n, 1, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0)
+    assert L.adamw_step(ctypes.byref(g), 1, 0, None) == N.MUON_ERR_INVALID_ARG  # step 0
+    bad = N.AdamWGroup(p, p, p, p, n, 1, 0, 1e-3, 1.5, 0.95, 1e-8, 0.0)
+    assert L.adamw_step(ctypes.byref(bad), 1, 1, None) == N.MUON_ERR_INVALID_ARG  # beta1
+    q = (ctypes.c_void_p * 1)(0x10004)
+    mis = N.AdamWGroup(q, p, p, p, n, 1, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0)
+    assert L.adamw_step(ctypes.byref(mis), 1, 1, None) == N.MUON_ERR_INVALID_ARG
+    neg = N.AdamWGroup(p, p, p, p, (ctypes.c_int64 * 1)(-1), 1, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0)
+    assert L.adamw_step(ctypes.byref(neg), 1, 1, None) == N.MUON_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(L):
+    g = [(768, 768, 48, 0, 1, 1.0), (3072, 768, 12, 48, 1, 1.0), (768, 3072, 12, 60, 1, 1.0)]
+    full = api.muon_workspace_size(g)
+    mn = api.muon_workspace_min_size(g)
+    assert 0 < mn < full
+    # X ping-pong (2 x bf16 params) + B (bf16 m x m) per matrix, plus small arrays
+    muon_elems = 48 * 768 * 768 + 24 * 768 * 3072
+    b_elems = 72 * 768 * 768
+    lower = 2 * 2 * muon_elems + 2 * b_elems
+    assert lower <= full <= lower * 1.01 + (1 << 20)
+    # fp32 debug mode doubles the matrix buffers
+    assert api.muon_workspace_size(g, N.MUON_FP32_DEBUG) > 1.9 * full
+    # invalid groups -> 0
+    assert api.muon_workspace_size([(0, 4, 1, 0, 0, 1.0)]) == 0
+
+
+def test_profiler_kinds(L):
+    names = [L.muon_kernel_kind_name(i).decode() for i in range(L.muon_kernel_kind_count())]
+    for k in ("momentum_norm", "ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update", "adamw"):
+        assert k in names
