@@ -1,0 +1,468 @@
+"""Benchmark: one Muon + AdamW optimizer step over a synthetic parameter set.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one muon_step (momentum + Frobenius norm, 5 quintic Newton-Schulz
+iterations as grouped tcgen05 GEMMs, cautious decay + update) over every
+hidden matrix plus one adamw_step over the embedding / LM head (/ gains),
+all through the C ABI.  Default workload: the 32-layer 8B-shaped set
+(Wq, Wo 4096^2; Wk, Wv 1024x4096; gate, up 14336x4096; down 4096x14336;
+AdamW on two 128256x4096 tables), fp32 params / momentum, bf16 grads.
+Inputs (~84 GB resident) are far larger than L2, so no flush is needed.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+cuda synchronize on both sides, CUDA events on the launching stream, max
+over ranks.  With N > 1 (torchrun), every rank runs its own replica of the
+workload on its GPU (matrices are independent problems; there is no data-path
+collective), so per-GPU work is fixed: weak scaling.
+
+Rank 0 prints one JSON line.  --impl reference times the CPU fp64 oracle on a
+bounded sample of the same workload instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon+AdamW step ms at 8B shapes; NS TFLOP/s as % of bf16 tensor peak"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- workload
+def algorithmic_work(wl):
+    """Per-step algorithmic FLOPs / bytes of each kernel kind (nominal FLOPs per
+    the spec: gram 2 m^2 n, A.A 2 m^3, B.X 2 m^2 n per iteration)."""
+    gram = poly = axpy = 0.0
+    mom_bytes = upd_bytes = 0.0
+    for s in wl.muon:
+        m, n = min(s.rows, s.cols), max(s.rows, s.cols)
+        gram += s.count * 2.0 * m * m * n
+        poly += s.count * 2.0 * m ** 3
+        axpy += s.count * 2.0 * m * m * n
+        gb = 2 if s.grad_dtype == "bf16" else 4
+        mom_bytes += s.count * s.rows * s.cols * (gb + 8 + 2)
+        upd_bytes += s.count * s.rows * s.cols * (2 + 8)
+    adam_bytes = 0.0
+    for t in wl.adamw:
+        gb = 2 if t.grad_dtype == "bf16" else 4
+        adam_bytes += t.count * math.prod(t.shape) * (gb + 24)
+    return dict(gram_flops=gram, poly_flops=poly, axpy_flops=axpy, momentum_bytes=mom_bytes,
+                update_bytes=upd_bytes, adamw_bytes=adam_bytes)
+
+
+class DeviceWorkload:
+    """All tensors of a workload resident on one GPU: params / momentum / grads
+    as views into one flat buffer per shape group (16-byte aligned views)."""
+
+    def __init__(self, wl, device, e2e_host: bool = False):
+        import torch
+        from muon_polar_orthogonalized_b200 import _native as N
+        from muon_polar_orthogonalized_b200 import workloads as W
+        self.wl = wl
+        self.device = device
+        self.groups, self.params, self.grads, self.mom = [], [], [], []
+        self.flat_grads = []
+        first = 0
+        for gi, s in enumerate(wl.muon):
+            numel = s.rows * s.cols
+            gdt = torch.bfloat16 if s.grad_dtype == "bf16" else torch.float32
+            P = torch.empty(s.count * numel, dtype=torch.float32, device=device)
+            Mm = torch.zeros(s.count * numel, dtype=torch.float32, device=device)
+            G = torch.empty(s.count * numel, dtype=gdt, device=device)
+            gen = W.device_generator(device, wl.name, "W", gi)
+            P.normal_(0.0, 0.02, generator=gen)
+            for j in range(s.count):
+                g = W.device_grad(wl, s.rows, s.cols, gdt, device, gi, j)
+                G[j * numel:(j + 1) * numel].copy_(g.reshape(-1))
+                del g
+            for j in range(s.count):
+                sl = slice(j * numel, (j + 1) * numel)
+                self.params.append(P[sl].view(s.rows, s.cols))
+                self.mom.append(Mm[sl].view(s.rows, s.cols))
+                self.grads.append(G[sl].view(s.rows, s.cols))
+            self.flat_grads.append(G)
+            self.groups.append((s.rows, s.cols, s.count, first,
+                                N.MUON_BF16 if s.grad_dtype == "bf16" else N.MUON_F32, 1.0))
+            first += s.count
+        self.adam = []
+        for ti, t in enumerate(wl.adamw):
+            gdt = torch.bfloat16 if t.grad_dtype == "bf16" else torch.float32
+            ps, gs, ms, vs = [], [], [], []
+            for j in range(t.count):
+                p = torch.empty(t.shape, dtype=torch.float32, device=device)
+                if t.init == "ones":
+                    p.fill_(1.0)
+                else:
+                    p.normal_(0.0, 0.02, generator=W.device_generator(device, wl.name, "aW", ti, j))
+                g = torch.randn(t.shape, generator=W.device_generator(device, wl.name, "aG", ti, j),
+                                device=device).mul_(wl.grad_std).to(gdt)
+                ps.append(p)
+                gs.append(g)
+                ms.append(torch.zeros_like(p))
+                vs.append(torch.zeros_like(p))
+                self.flat_grads.append(g.view(-1))
+            self.adam.append((ps, gs, ms, vs, t))
+        self.host_grads = None
+        if e2e_host:
+            self.host_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in self.flat_grads]
+            for h, g in zip(self.host_grads, self.flat_grads):
+                h.copy_(g)
+
+    def adam_specs(self):
+        from muon_polar_orthogonalized_b200 import api
+        from muon_polar_orthogonalized_b200 import workloads as W
+        return [api.AdamWSpec(ps, gs, ms, vs, W.ADAMW_LR, W.ADAMW_BETAS[0], W.ADAMW_BETAS[1],
+                              W.ADAMW_EPS, t.wd) for (ps, gs, ms, vs, t) in self.adam]
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from muon_polar_orthogonalized_b200 import _native as N
+    from muon_polar_orthogonalized_b200 import api
+    from muon_polar_orthogonalized_b200 import workloads as W
+    from muon_polar_orthogonalized_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if rank == 0:
+        build()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        dist.barrier()
+        if rank != 0:
+            build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = W.get(args.workload)
+    D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e)
+    flags = N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD
+    ws_bytes = api.muon_workspace_size(D.groups, flags)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    coeffs = W.NS_COEFFS_FIXED
+    specs = D.adam_specs()
+    stream = torch.cuda.current_stream()
+    step_no = [0]
+
+    def step():
+        step_no[0] += 1
+        api.muon_step(D.params, D.grads, D.mom, D.groups, W.MUON_LR, W.MUON_BETA, W.MUON_WD,
+                      wl.ns_steps, coeffs, flags, ws, stream=stream)
+        if specs:
+            api.adamw_step(specs, step_no[0], stream=stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if api.muon_query_status(ws) != N.MUON_OK:
+        raise RuntimeError("device status word reports an error after warm-up")
+
+    # ---------------------------------------------------- device-timed region
+    clocks = ClockSampler(local)
+    clocks.start()
+    api.muon_profiler_reset()
+    api.muon_profiler_enable(True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    api.muon_profiler_enable(False)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    prof = api.muon_profiler_read()
+    ms_step = ms_total / args.steps
+
+    # ------------------------------------------------------- end to end
+    e2e = None
+    if D.host_grads is not None:
+        h2d = sum(h.numel() * h.element_size() for h in D.host_grads)
+        status_host = torch.empty(1, dtype=torch.int32, pin_memory=True)
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            for g, h in zip(D.flat_grads, D.host_grads):
+                g.copy_(h, non_blocking=True)
+            step()
+            status_host.copy_(ws[:4].view(torch.int32), non_blocking=True)
+        a1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1)) / args.steps
+        e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": 4,
+               "path": "pinned host grads -> cudaMemcpyAsync -> muon_step + adamw_step -> status word read"}
+
+    if rank == 0:
+        work = algorithmic_work(wl)
+        peaks, peak_src = load_peaks()
+        ns_nom = wl.ns_flops_nominal()
+        ns_exe = wl.ns_flops_executed()
+        kinds = {k: v for k, v in prof.items() if v[1] > 0}
+        ns_ms = sum(kinds.get(k, (0, 0))[0] for k in ("ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update")) / args.steps
+        # dominant kernel and its roofline
+        dom = max(kinds.items(), key=lambda kv: kv[1][0])[0] if kinds else None
+        launches = sum(v[1] for v in kinds.values())
+        per_kernel = {}
+        for k, (ms, n) in kinds.items():
+            per_kernel[k] = {"ms_per_step": round(ms / args.steps, 4), "launches_per_step": n / args.steps,
+                             "avg_launch_ms": round(ms / n, 4)}
+        K = wl.ns_steps
+        alg = {
+            "ns_gram": ("tensor", work["gram_flops"]),
+            "ns_poly": ("tensor", work["poly_flops"]),
+            "ns_axpy": ("tensor", work["axpy_flops"]),
+            "ns_axpy_update": ("tensor", work["axpy_flops"]),
+            "momentum_norm": ("hbm", work["momentum_bytes"]),
+            "update": ("hbm", work["update_bytes"]),
+            "adamw": ("hbm", work["adamw_bytes"]),
+        }
+        # per-step algorithmic work of each kernel kind: GEMM kinds run once per
+        # NS iteration (the last B.X is the fused-update kind), elementwise once
+        per_step_work = {
+            "ns_gram": work["gram_flops"] * K, "ns_poly": work["poly_flops"] * K,
+            "ns_axpy": work["axpy_flops"] * (K - 1 if "ns_axpy_update" in kinds else K),
+            "ns_axpy_update": work["axpy_flops"],
+            "momentum_norm": work["momentum_bytes"], "update": work["update_bytes"],
+            "adamw": work["adamw_bytes"]}
+        roof = None
+        if dom in alg:
+            bound = alg[dom][0]
+            ms, n = kinds[dom]
+            launches_per_step = n / args.steps
+            per_launch = per_step_work[dom] / launches_per_step
+            avg_s = ms / n / 1e3
+            if bound == "tensor":
+                ach = per_launch / avg_s / 1e12
+                peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+                roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                        "peak_source": f"{peak_src} (sustained bf16 cuBLAS)",
+                        "work_per_launch": per_launch, "work_unit": "nominal FLOP"}
+            else:
+                ach = per_launch / avg_s / 1e9
+                peak = peaks["hbm_gbs"]
+                roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
+                        "unit": "GB/s", "frac": round(ach / peak, 4), "traffic": None,
+                        "peak_source": f"{peak_src} (HBM copy)",
+                        "work_per_launch": per_launch, "work_unit": "algorithmic bytes"}
+        ew = {}
+        for k in ("momentum_norm", "update", "adamw"):
+            if k in kinds:
+                ew[k] = round(per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e9, 1)
+        for k in ("ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update"):
+            if k in kinds:
+                per_kernel[k]["nominal_tflops"] = round(
+                    per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e12, 1)
+        res = {
+            "metric": METRIC,
+            "value": round(ms_step, 3),
+            "unit": "ms",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 3),
+            "higher_is_better": False,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "muon_params": wl.muon_params(), "adamw_params": wl.adamw_params(),
+                       "muon_groups": [[s.rows, s.cols, s.count] for s in wl.muon],
+                       "ns_steps": K, "grads": "bf16", "params_state": "fp32",
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+            "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
+            "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
+            "ns_ms_per_step": round(ns_ms, 3),
+            "ns_frac_of_peak_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4) if ns_ms else None,
+            "elementwise_gbs": ew,
+            "roofline": roof,
+            "per_kernel": per_kernel,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+        }
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl, reps=1)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------- CPU (oracle)
+def cpu_baseline(wl, reps: int = 1):
+    """The oracle, as it stands, on a bounded sample of the workload, scaled to
+    ms per full step: one Muon matrix of the cheapest shape group (timed
+    muon_step in fp64), extrapolated to every matrix by nominal NS FLOPs, plus
+    AdamW on a 4M-element slice extrapolated by element count."""
+    import numpy as np
+
+    import oracle
+    from muon_polar_orthogonalized_b200 import workloads as W
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    s = min(wl.muon, key=lambda s: min(s.rows, s.cols) ** 2 * max(s.rows, s.cols))
+    rng = np.random.default_rng(0)
+    Wm = rng.standard_normal((s.rows, s.cols)) * 0.02
+    G = rng.standard_normal((s.rows, s.cols)) * wl.grad_std
+    M = np.zeros_like(G)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.muon_step(Wm, G, M, W.MUON_LR, W.MUON_BETA, W.MUON_WD, wl.ns_steps, W.NS_COEFFS_FIXED)
+    t_mat = (time.perf_counter() - t0) / reps
+    m, n = min(s.rows, s.cols), max(s.rows, s.cols)
+    f_mat = 4.0 * m * m * n + 2.0 * m ** 3
+    muon_ms = t_mat * (wl.ns_flops_nominal() / wl.ns_steps / f_mat) * 1e3
+    adam_ms = 0.0
+    n_adam = wl.adamw_params()
+    if n_adam:
+        k = min(n_adam, 1 << 22)
+        p = rng.standard_normal(k) * 0.02
+        g = rng.standard_normal(k) * wl.grad_std
+        z = np.zeros(k)
+        t0 = time.perf_counter()
+        oracle.adamw_step(p, g, z, z, 1, W.ADAMW_LR, 0.9, 0.95, 1e-8, 0.0)
+        adam_ms = (time.perf_counter() - t0) * (n_adam / k) * 1e3
+    return {"value": round(muon_ms + adam_ms, 1), "unit": "ms", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 NumPy muon_step on one {s.rows}x{s.cols} matrix ({t_mat:.2f} s) scaled by "
+                      f"nominal NS FLOPs to all {sum(x.count for x in wl.muon)} matrices, plus AdamW on "
+                      f"{min(n_adam, 1 << 22)} elements scaled to {n_adam}",
+            "extrapolated": True}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from muon_polar_orthogonalized_b200 import workloads as W
+    wl = W.get(args.workload)
+    for _ in range(args.warmup):
+        cpu_baseline(wl)
+    vals = [cpu_baseline(wl)["value"] for _ in range(args.steps)]
+    cb = cpu_baseline(wl)
+    v = statistics.median(vals)
+    cb["value"] = v
+    res = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": wl.name, "parallelism": "cpu oracle"},
+           "cpu_baseline": cb,
+           "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama_8b_32l")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
