@@ -36,7 +36,8 @@ struct MatRef {
 struct EltParams {
   MatRef mats[kMaxMatsPerLaunch];
   int nmats;
-  int total_blocks;
+  int total_blocks;  // work chunks (one partial sum each); blocks loop over them
+  int grid;          // launched blocks (persistent, <= total_blocks)
   int grad_bf16;     // grads of every matrix in this launch are bf16
   int x_f32;         // workspace X is fp32 (debug mode)
   int nesterov;
@@ -118,7 +119,8 @@ struct AdamTensor {
 struct AdamParams {
   AdamTensor t[kMaxAdamTensors];
   int ntensors;
-  int total_blocks;
+  int total_blocks;  // work chunks
+  int grid;          // launched blocks (persistent)
   int grad_bf16;
 };
 

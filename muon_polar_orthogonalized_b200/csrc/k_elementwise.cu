@@ -23,7 +23,8 @@
 namespace muon {
 
 constexpr int kEltThreads = 256;
-constexpr int kEltUnroll = 8;                                // vec4 units per thread
+constexpr int kEltUnroll = 4;                                // vec4 units per thread
+constexpr int kEltMinBlocks = 4;                             // resident blocks per SM (occupancy)
 constexpr int kEltChunk = kEltThreads * kEltUnroll * 4;      // elements per block
 
 __device__ __forceinline__ int find_mat(const MatRef* mats, int n, int blk) {
@@ -105,25 +106,29 @@ __device__ __forceinline__ float block_sum(float v) {
 }
 
 // ------------------------------------------------------------ momentum_norm
+// X index of flat element e (multiple of 4 on the vector path): the X buffer
+// has pitch ldx >= cols; when they are equal it is e itself.
+__device__ __forceinline__ long long x_index(const MatRef& r, long long e) {
+  if (r.ldx == r.cols) return e;
+  const int ei = static_cast<int>(e);  // numel < 2^31 (checked on the host)
+  const int row = ei / r.cols;
+  return static_cast<long long>(row) * r.ldx + (ei - row * r.cols);
+}
+
 template <bool GBF16>
-__global__ void __launch_bounds__(kEltThreads)
-momentum_norm_kernel(const __grid_constant__ EltParams p) {
-  const int blk = blockIdx.x;
-  const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
+__device__ __forceinline__ float momentum_chunk(const EltParams& p, const MatRef& r, long long e0) {
   const long long numel = static_cast<long long>(r.rows) * r.cols;
-  const long long e0 = static_cast<long long>(blk - r.blk_begin) * kEltChunk;
   const float beta = p.beta;
   const bool f32x = p.x_f32 != 0;
   float acc = 0.f;
   if (r.vec) {
-    const int cols4 = r.cols >> 2;
     float4 gv[kEltUnroll], mv[kEltUnroll];
 #pragma unroll
     for (int u = 0; u < kEltUnroll; ++u) {
       const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
       if (e < numel) {
         gv[u] = load_g4<GBF16>(r.g, e);
-        mv[u] = r.m ? *reinterpret_cast<const float4*>(r.m + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        mv[u] = r.m ? __ldcs(reinterpret_cast<const float4*>(r.m + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
@@ -137,7 +142,7 @@ momentum_norm_kernel(const __grid_constant__ EltParams p) {
           mn.y = fmaf(beta, mv[u].y, gv[u].y);
           mn.z = fmaf(beta, mv[u].z, gv[u].z);
           mn.w = fmaf(beta, mv[u].w, gv[u].w);
-          *reinterpret_cast<float4*>(r.m + e) = mn;
+          __stcs(reinterpret_cast<float4*>(r.m + e), mn);
           if (p.nesterov) {
             mt.x = fmaf(beta, mn.x, gv[u].x);
             mt.y = fmaf(beta, mn.y, gv[u].y);
@@ -153,10 +158,7 @@ momentum_norm_kernel(const __grid_constant__ EltParams p) {
         acc = fmaf(mt.y, mt.y, acc);
         acc = fmaf(mt.z, mt.z, acc);
         acc = fmaf(mt.w, mt.w, acc);
-        const long long q = e >> 2;
-        const long long row = q / cols4;
-        const long long col = (q - row * cols4) * 4;
-        store_x4(r.x, row * r.ldx + col, mt, f32x);
+        store_x4(r.x, x_index(r, e), mt, f32x);
       }
     }
   } else {
@@ -171,14 +173,26 @@ momentum_norm_kernel(const __grid_constant__ EltParams p) {
           mt = p.nesterov ? fmaf(beta, mn, g) : mn;
         }
         acc = fmaf(mt, mt, acc);
-        const long long row = e / r.cols;
-        const long long col = e - row * r.cols;
-        store_x1(r.x, row * r.ldx + col, mt, f32x);
+        store_x1(r.x, x_index(r, e), mt, f32x);
       }
     }
   }
-  const float s = block_sum(acc);
-  if (threadIdx.x == 0) p.partials[blk] = s;
+  return acc;
+}
+
+// Persistent: block b handles chunks b, b + grid, ...; every chunk's partial
+// sum is reduced in a fixed order, so results do not depend on the grid.
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads, kEltMinBlocks)
+momentum_norm_kernel(const __grid_constant__ EltParams p) {
+  for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
+    const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
+    const long long e0 = static_cast<long long>(blk - r.blk_begin) * kEltChunk;
+    const float acc = momentum_chunk<GBF16>(p, r, e0);
+    const float s = block_sum(acc);
+    if (threadIdx.x == 0) p.partials[blk] = s;
+    __syncthreads();  // block_sum's shared scratch is reused by the next chunk
+  }
 }
 
 // ------------------------------------------------------------ norm_finalize
@@ -216,12 +230,8 @@ __device__ __forceinline__ float cautious_apply(float w, float u, float lr, floa
 }
 
 template <bool EMIT>
-__global__ void __launch_bounds__(kEltThreads)
-update_kernel(const __grid_constant__ EltParams p) {
-  const int blk = blockIdx.x;
-  const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
+__device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r, long long e0) {
   const long long numel = static_cast<long long>(r.rows) * r.cols;
-  const long long e0 = static_cast<long long>(blk - r.blk_begin) * kEltChunk;
   const bool f32x = p.x_f32 != 0;
   const float sc = p.use_scale ? p.scales[r.sidx] : 1.f;
   auto make_u = [&](float x) {
@@ -229,17 +239,13 @@ update_kernel(const __grid_constant__ EltParams p) {
     return f32x ? sc * x : round_bf16(sc * x);
   };
   if (r.vec) {
-    const int cols4 = r.cols >> 2;
     float4 xv[kEltUnroll], wv[kEltUnroll];
 #pragma unroll
     for (int u = 0; u < kEltUnroll; ++u) {
       const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
       if (e < numel) {
-        const long long q = e >> 2;
-        const long long row = q / cols4;
-        const long long col = (q - row * cols4) * 4;
-        xv[u] = load_x4(r.x, row * r.ldx + col, f32x);
-        if (!EMIT) wv[u] = *reinterpret_cast<const float4*>(r.w + e);
+        xv[u] = load_x4(r.x, x_index(r, e), f32x);
+        if (!EMIT) wv[u] = __ldcs(reinterpret_cast<const float4*>(r.w + e));
       }
     }
 #pragma unroll
@@ -255,7 +261,7 @@ update_kernel(const __grid_constant__ EltParams p) {
           w.y = cautious_apply(w.y, uu.y, r.lr, p.wd, p.cautious);
           w.z = cautious_apply(w.z, uu.z, r.lr, p.wd, p.cautious);
           w.w = cautious_apply(w.w, uu.w, r.lr, p.wd, p.cautious);
-          *reinterpret_cast<float4*>(r.w + e) = w;
+          __stcs(reinterpret_cast<float4*>(r.w + e), w);
         }
       }
     }
@@ -263,13 +269,20 @@ update_kernel(const __grid_constant__ EltParams p) {
     for (int u = 0; u < kEltUnroll * 4; ++u) {
       const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
       if (e < numel) {
-        const long long row = e / r.cols;
-        const long long col = e - row * r.cols;
-        const float uu = make_u(load_x1(r.x, row * r.ldx + col, f32x));
+        const float uu = make_u(load_x1(r.x, x_index(r, e), f32x));
         if (EMIT) r.out[e] = uu;
         else r.w[e] = cautious_apply(r.w[e], uu, r.lr, p.wd, p.cautious);
       }
     }
+  }
+}
+
+template <bool EMIT>
+__global__ void __launch_bounds__(kEltThreads, kEltMinBlocks)
+update_kernel(const __grid_constant__ EltParams p) {
+  for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
+    const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
+    update_chunk<EMIT>(p, r, static_cast<long long>(blk - r.blk_begin) * kEltChunk);
   }
 }
 
@@ -293,11 +306,7 @@ __device__ __forceinline__ void adam_elem(const AdamTensor& T, float g, float& p
 }
 
 template <bool GBF16>
-__global__ void __launch_bounds__(kEltThreads)
-adamw_kernel(const __grid_constant__ AdamParams P) {
-  const int blk = blockIdx.x;
-  const AdamTensor& T = P.t[find_tensor(P.t, P.ntensors, blk)];
-  const long long e0 = static_cast<long long>(blk - T.blk_begin) * kEltChunk;
+__device__ __forceinline__ void adamw_chunk(const AdamTensor& T, long long e0) {
   if (T.vec) {
     constexpr int U = kEltUnroll / 2;  // 4 streams per element: keep registers in check
 #pragma unroll 1
@@ -309,9 +318,9 @@ adamw_kernel(const __grid_constant__ AdamParams P) {
             e0 + (static_cast<long long>(half * U + u) * kEltThreads + threadIdx.x) * 4;
         if (e < T.numel) {
           gv[u] = load_g4<GBF16>(T.g, e);
-          pv[u] = *reinterpret_cast<const float4*>(T.p + e);
-          mv[u] = *reinterpret_cast<const float4*>(T.m + e);
-          vv[u] = *reinterpret_cast<const float4*>(T.v + e);
+          pv[u] = __ldcs(reinterpret_cast<const float4*>(T.p + e));
+          mv[u] = __ldcs(reinterpret_cast<const float4*>(T.m + e));
+          vv[u] = __ldcs(reinterpret_cast<const float4*>(T.v + e));
         }
       }
 #pragma unroll
@@ -323,9 +332,9 @@ adamw_kernel(const __grid_constant__ AdamParams P) {
           adam_elem(T, gv[u].y, pv[u].y, mv[u].y, vv[u].y);
           adam_elem(T, gv[u].z, pv[u].z, mv[u].z, vv[u].z);
           adam_elem(T, gv[u].w, pv[u].w, mv[u].w, vv[u].w);
-          *reinterpret_cast<float4*>(T.p + e) = pv[u];
-          *reinterpret_cast<float4*>(T.m + e) = mv[u];
-          *reinterpret_cast<float4*>(T.v + e) = vv[u];
+          __stcs(reinterpret_cast<float4*>(T.p + e), pv[u]);
+          __stcs(reinterpret_cast<float4*>(T.m + e), mv[u]);
+          __stcs(reinterpret_cast<float4*>(T.v + e), vv[u]);
         }
       }
     }
@@ -343,15 +352,44 @@ adamw_kernel(const __grid_constant__ AdamParams P) {
   }
 }
 
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads, kEltMinBlocks)
+adamw_kernel(const __grid_constant__ AdamParams P) {
+  for (int blk = blockIdx.x; blk < P.total_blocks; blk += gridDim.x) {
+    const AdamTensor& T = P.t[find_tensor(P.t, P.ntensors, blk)];
+    adamw_chunk<GBF16>(T, static_cast<long long>(blk - T.blk_begin) * kEltChunk);
+  }
+}
+
 // ------------------------------------------------------------- launchers
 int elt_chunk() { return kEltChunk; }
 
-cudaError_t launch_momentum_norm(const EltParams& p, cudaStream_t s) {
+// Persistent grid: every SM filled to its occupancy limit, never more blocks
+// than chunks.
+template <typename K>
+static int persistent_grid(K kernel, int chunks, int sms) {
+  static thread_local const void* last_kernel = nullptr;
+  static thread_local int last_occ = 0;
+  if (last_kernel != reinterpret_cast<const void*>(kernel)) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kEltThreads, 0) != cudaSuccess || occ < 1)
+      occ = 1;
+    last_kernel = reinterpret_cast<const void*>(kernel);
+    last_occ = occ;
+  }
+  const long long g = static_cast<long long>(sms) * last_occ;
+  return static_cast<int>(g < chunks ? g : chunks);
+}
+
+cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (p.grad_bf16)
-    momentum_norm_kernel<true><<<p.total_blocks, kEltThreads, 0, s>>>(p);
-  else
-    momentum_norm_kernel<false><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  if (p.grad_bf16) {
+    auto k = momentum_norm_kernel<true>;
+    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+  } else {
+    auto k = momentum_norm_kernel<false>;
+    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -361,21 +399,27 @@ cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_update(const EltParams& p, bool emit, cudaStream_t s) {
+cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (emit)
-    update_kernel<true><<<p.total_blocks, kEltThreads, 0, s>>>(p);
-  else
-    update_kernel<false><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  if (emit) {
+    auto k = update_kernel<true>;
+    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+  } else {
+    auto k = update_kernel<false>;
+    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
-cudaError_t launch_adamw(const AdamParams& p, cudaStream_t s) {
+cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (p.grad_bf16)
-    adamw_kernel<true><<<p.total_blocks, kEltThreads, 0, s>>>(p);
-  else
-    adamw_kernel<false><<<p.total_blocks, kEltThreads, 0, s>>>(p);
+  if (p.grad_bf16) {
+    auto k = adamw_kernel<true>;
+    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+  } else {
+    auto k = adamw_kernel<false>;
+    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -82,21 +82,6 @@ __device__ __forceinline__ void record_timeout(unsigned int* status, volatile in
   atomicOr(status, kDevTimeout);
 }
 
-// 32 consecutive bf16 -> fp32 (16-byte loads; address 16-byte aligned).
-__device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 raw = s4[q];
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
-      v[q * 8 + h * 2] = f.x;
-      v[q * 8 + h * 2 + 1] = f.y;
-    }
-  }
-}
 __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -121,13 +106,74 @@ __device__ __forceinline__ float cautious_w(float w, float u, float lr, float wd
   return fmaf(-lr, t, w);
 }
 
-// Epilogue for one 32-column chunk held by this thread (row i, cols j0..j0+31).
+// ------------------------------------------------------------- epilogue
+// Each epilogue thread owns one accumulator row i of the tile and walks it in
+// 32-column chunks.  Per chunk: (1) issue the global loads the epilogue needs
+// (the b*A / a*X operand, and W for the fused update) as independent loads,
+// (2) read the accumulator chunk from TMEM, (3) combine and store.  Before
+// waiting for a tile's accumulator, the thread prefetches its row segments of
+// those operands into L2, so the loads in (1) hit L2.
+
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 template <int EPI>
-__device__ __forceinline__ void epilogue_chunk(const TcGemmParams& p, const GemmProblem& q,
-                                               int mat, int i, int j0, bool mirror,
-                                               float (&v)[32]) {
+__device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const GemmProblem& q,
+                                                  int mat, int i, int jt) {
+  if (EPI == EPI_GRAM || i >= q.M) return;
+  const int ncols = min(TC_BN, q.N - jt);
+  const char* ein = reinterpret_cast<const char*>(
+      static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
+  for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
+  if (EPI == EPI_AXPY_UPDATE) {
+    const int wi = q.w_first + mat;
+    const char* w = reinterpret_cast<const char*>(p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + jt);
+    for (int b = 0; b < ncols * 4; b += 128) prefetch_l2(w + b);
+  }
+}
+
+struct EpiIn {
+  uint4 e[4];     // 32 bf16 of the epilogue operand (A or X)
+  float4 w[8];    // 32 fp32 parameters (fused update)
+};
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_load(const TcGemmParams& p, const GemmProblem& q, int mat,
+                                              int i, int j0, bool full, bool wvec, EpiIn& in) {
   if (i >= q.M) return;
-  const bool full = (j0 + 32 <= q.N);
+  if (EPI != EPI_GRAM && full) {
+    const uint4* e4 = reinterpret_cast<const uint4*>(
+        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) in.e[k] = e4[k];
+  }
+  if (EPI == EPI_AXPY_UPDATE && full && wvec) {
+    const int wi = q.w_first + mat;
+    const float4* w4 = reinterpret_cast<const float4*>(p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) in.w[k] = w4[k];
+  }
+}
+
+__device__ __forceinline__ void unpack_bf16x32(const uint4 (&e)[4], float (&a)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w[4] = {e[q].x, e[q].y, e[q].z, e[q].w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+      a[q * 8 + h * 2] = f.x;
+      a[q * 8 + h * 2 + 1] = f.y;
+    }
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const GemmProblem& q, int mat,
+                                               int i, int j0, bool full, bool wvec, bool mirror,
+                                               const EpiIn& in, float (&v)[32]) {
+  if (i >= q.M) return;
   float f = 1.f;
   if (q.scale_mode) {
     const float s = p.scales[q.scale_base + mat];
@@ -136,41 +182,34 @@ __device__ __forceinline__ void epilogue_chunk(const TcGemmParams& p, const Gemm
   if constexpr (EPI == EPI_GRAM) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] *= f;
-  } else if constexpr (EPI == EPI_POLY) {
-    const __nv_bfloat16* ein =
-        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0;
+  } else {
     float a[32];
     if (full) {
-      ld_bf16x32(ein, a);
+      unpack_bf16x32(in.e, a);
     } else {
+      const __nv_bfloat16* ein = static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs +
+                                 static_cast<long long>(i) * q.ein_ld + j0;
 #pragma unroll
       for (int c = 0; c < 32; ++c) a[c] = (j0 + c < q.N) ? __bfloat162float(ein[c]) : 0.f;
     }
+    if constexpr (EPI == EPI_POLY) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]);
-  } else {  // AXPY, AXPY_UPDATE
-    const __nv_bfloat16* ein =
-        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0;
-    float x[32];
-    if (full) {
-      ld_bf16x32(ein, x);
+      for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]);
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = (j0 + c < q.N) ? __bfloat162float(ein[c]) : 0.f;
+      for (int c = 0; c < 32; ++c) v[c] = f * fmaf(q.ca, a[c], v[c]);
     }
-#pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] = f * fmaf(q.ca, x[c], v[c]);
   }
 
   if constexpr (EPI == EPI_AXPY_UPDATE) {
     const int wi = q.w_first + mat;
     float* w = p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0;
     const bool cautious = p.cautious != 0;
-    if (full && ((reinterpret_cast<uintptr_t>(w) & 15u) == 0)) {
+    if (full && wvec) {
       float4* w4 = reinterpret_cast<float4*>(w);
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
-        float4 ww = w4[c4];
+        float4 ww = in.w[c4];
         ww.x = cautious_w(ww.x, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 0])), q.lr, p.wd, cautious);
         ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), q.lr, p.wd, cautious);
         ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), q.lr, p.wd, cautious);
@@ -354,12 +393,18 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
       const TileCoord tc = decode_tile(p, t);
       const GemmProblem& q = p.prob[tc.prob];
+      const int i = tc.tm * TC_BM + row_in_tile;
+      epilogue_prefetch<EPI>(p, q, tc.mat, i, tc.tn * TC_BN);
+      bool wvec = true;
+      if (EPI == EPI_AXPY_UPDATE && i < q.M) {
+        const int wi = q.w_first + tc.mat;
+        wvec = ((reinterpret_cast<uintptr_t>(p.wptr[wi]) | (static_cast<uintptr_t>(p.wcols[wi]) << 2)) & 15u) == 0;
+      }
       if (!sm100::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         record_timeout(p.status, abort_flag);
         break;
       }
       sm100::tc_fence_after();
-      const int i = tc.tm * TC_BM + row_in_tile;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * TC_BN);
 #pragma unroll 1
@@ -372,9 +417,12 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           if (jb < tc.tm) continue;         // strictly lower block: produced by its mirror
           mirror = jb > tc.tm;
         }
+        const bool full = (j0 + 32 <= q.N);
+        EpiIn in;
+        epilogue_load<EPI>(p, q, tc.mat, i, j0, full, wvec, in);
         float v[32];
         sm100::tmem_ld32(t_row + static_cast<uint32_t>(c * 32), v);
-        epilogue_chunk<EPI>(p, q, tc.mat, i, j0, mirror, v);
+        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, mirror, in, v);
       }
       sm100::tc_fence_before();
       sm100::mbar_arrive(&tempty_bar[acc]);

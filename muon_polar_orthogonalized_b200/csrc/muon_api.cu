@@ -25,10 +25,10 @@
 namespace muon {
 // kernels (k_elementwise.cu, k_gemm_tc.cu, k_gemm_simt.cu)
 int elt_chunk();
-cudaError_t launch_momentum_norm(const EltParams& p, cudaStream_t s);
+cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
-cudaError_t launch_update(const EltParams& p, bool emit, cudaStream_t s);
-cudaError_t launch_adamw(const AdamParams& p, cudaStream_t s);
+cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
+cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
 int tc_tile_m();
 int tc_tile_n();
 cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, int num_sms, cudaStream_t s);
@@ -383,13 +383,13 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
     if (kind == 0) {
       P.partials = partials + launch_blk0;
       P.grad_bf16 = pending_dtype == MUON_BF16;
-      e = timed_launch(K_MOMENTUM, a.stream, [&] { return launch_momentum_norm(P, a.stream); });
+      e = timed_launch(K_MOMENTUM, a.stream, [&] { return launch_momentum_norm(P, C.dev.sms, a.stream); });
     } else if (kind == 1) {
       P.partials = partials;
       e = timed_launch(K_NORM, a.stream, [&] { return launch_norm_finalize(P, a.stream); });
     } else {
       e = timed_launch(kind == 2 ? K_UPDATE : K_EMIT, a.stream,
-                       [&] { return launch_update(P, kind == 3, a.stream); });
+                       [&] { return launch_update(P, kind == 3, C.dev.sms, a.stream); });
     }
     if (e != cudaSuccess) return cuda_fail(e, "elementwise launch");
     launch_blk0 += P.total_blocks;
@@ -746,7 +746,7 @@ muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step, mu
     P.grad_bf16 = dt;
     auto flush = [&]() -> muon_status {
       if (P.ntensors == 0) return MUON_OK;
-      cudaError_t e = timed_launch(K_ADAMW, s, [&] { return launch_adamw(P, s); });
+      cudaError_t e = timed_launch(K_ADAMW, s, [&] { return launch_adamw(P, dev.sms, s); });
       if (e != cudaSuccess) return cuda_fail(e, "adamw launch");
       P.ntensors = 0;
       P.total_blocks = 0;

@@ -163,12 +163,26 @@ def llama_8b_32l() -> Workload:
         grad_kind="iid", grad_std=1e-3)
 
 
+def llama_8b_1layer() -> Workload:
+    """One layer of the 8B-shaped set plus a 16384x4096 AdamW slice (a few GB;
+    for profiler captures of the same kernels on the same shapes)."""
+    return Workload(
+        name="llama_8b_1layer",
+        muon=(MuonShape(4096, 4096, 2, "bf16", "wq+wo"),
+              MuonShape(1024, 4096, 2, "bf16", "wk+wv"),
+              MuonShape(14336, 4096, 2, "bf16", "gate+up"),
+              MuonShape(4096, 14336, 1, "bf16", "down")),
+        adamw=(AdamWTensor((16384, 4096), 1, "bf16", "wte slice"),),
+        grad_kind="iid", grad_std=1e-3)
+
+
 WORKLOADS = {
     "single_256x1024": single_256x1024,
     "illcond_256x1024": illcond_256x1024,
     "gpt_d768_12l": gpt_d768_12l,
     "gpt_d1664_26l": gpt_d1664_26l,
     "llama_8b_32l": llama_8b_32l,
+    "llama_8b_1layer": llama_8b_1layer,
 }
 
 
