@@ -65,7 +65,9 @@ enum {
   MUON_NESTEROV = 1u,       /* orthogonalise beta*m + G (else m itself, heavy-ball) */
   MUON_CAUTIOUS_WD = 2u,    /* decay only where update*param >= 0 (else plain decoupled decay) */
   MUON_FP32_DEBUG = 4u,     /* fp32 operands and fp32 FMA GEMMs (slow; tolerance 1e-4 mode) */
-  MUON_UNFUSED_UPDATE = 8u  /* apply the update in its own kernel instead of the last B*X epilogue */
+  MUON_UNFUSED_UPDATE = 8u, /* apply the update in its own kernel instead of the last B*X epilogue */
+  MUON_TC_SINGLE_CTA = 16u  /* run the Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of
+                               CTA-pair (cta_group::2) 256x256 tiles; same results, for comparison */
 };
 
 /*
@@ -122,7 +124,7 @@ muon_status muon_step(float* const* params, const void* const* grads, float* con
  * The orthogonaliser alone: outputs[i] <- NS(inputs[i]) as fp32, rows x cols,
  * with the same normalisation, orientation, iteration and bf16 rounding of
  * the result as muon_step.  inputs[i] dtype per group.  Only MUON_FP32_DEBUG
- * is honoured in `flags`.
+ * and MUON_TC_SINGLE_CTA are honoured in `flags`.
  */
 muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs,
                                const muon_group* groups, int n_groups,

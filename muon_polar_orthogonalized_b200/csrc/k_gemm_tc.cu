@@ -32,22 +32,37 @@
 
 namespace muon {
 
-constexpr int TC_BM = 128;
+// Tile geometry.  Single-CTA mode: 128x256 tiles, one SM per tile.  Pair mode
+// (cta_group::2): 256x256 tiles on a CTA pair; each CTA stages 128 rows of A
+// and 128 rows (N/2) of B, the leader issues one 256x256x16 MMA per K step
+// that reads both CTAs' shared memory, and each CTA's TMEM holds its 128
+// accumulator rows.
+template <bool PAIR>
+struct TcCfg {
+  static constexpr int BM = PAIR ? 256 : 128;        // tile rows
+  static constexpr int BN = 256;                     // tile columns
+  static constexpr int BK = 64;
+  static constexpr int A_ROWS = 128;                 // A rows staged per CTA
+  static constexpr int B_ROWS = PAIR ? 128 : 256;    // B rows staged per CTA
+  static constexpr int A_BYTES = A_ROWS * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+};
 constexpr int TC_BN = 256;
-constexpr int TC_BK = 64;
-constexpr int TC_STAGES = 4;
-constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;   // 16 KB
-constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;   // 32 KB
-constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_THREADS = 192;
 constexpr int TC_TMEM_COLS = 512;
-constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 constexpr int TC_RASTER_GN = 8;   // tile-column band width of the non-symmetric raster
 
 struct TileCoord {
   int prob, mat, tm, tn;
 };
 
+// Linear tile index -> (problem, matrix, tile row, tile column).  Symmetric
+// problems enumerate, per tile row I, only the tile columns that reach the
+// upper triangle: J >= I*BM/BN.
+template <int BM>
 __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
   int pi = 0;
   while (pi + 1 < p.nprob && t >= p.prob[pi + 1].tile_begin) ++pi;
@@ -59,13 +74,13 @@ __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
   if (q.sym) {
     int I = 0;
     for (;;) {
-      const int cnt = q.tiles_n - (I >> 1);
+      const int cnt = q.tiles_n - (I * BM) / TC_BN;
       if (r < cnt) break;
       r -= cnt;
       ++I;
     }
     tm = I;
-    tn = (I >> 1) + r;
+    tn = (I * BM) / TC_BN + r;
   } else {
     const int band_tiles = q.tiles_m * TC_RASTER_GN;
     const int band = r / band_tiles;
@@ -122,7 +137,7 @@ template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const GemmProblem& q,
                                                   int mat, int i, int jt) {
   if (EPI == EPI_GRAM || i >= q.M) return;
-  const int ncols = min(TC_BN, q.N - jt);
+  const int ncols = min(TC_BN, q.N - jt);  // jt < N
   const char* ein = reinterpret_cast<const char*>(
       static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
   for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
@@ -242,29 +257,33 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
   }
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
+  using C = TcCfg<PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + TC_STAGES * TC_STAGE_BYTES);
-  uint64_t* empty_bar = full_bar + TC_STAGES;
-  uint64_t* tfull_bar = empty_bar + TC_STAGES;   // [2]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty_bar = full_bar + C::STAGES;
+  uint64_t* tfull_bar = empty_bar + C::STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;          // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int rank = PAIR ? static_cast<int>(sm100::cluster_ctarank()) : 0;
+  const int unit = PAIR ? (blockIdx.x >> 1) : blockIdx.x;        // tile-processing unit
+  const int nunits = PAIR ? (gridDim.x >> 1) : gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       sm100::mbar_init(&full_bar[s], 1);
       sm100::mbar_init(&empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       sm100::mbar_init(&tfull_bar[b], 1);
-      sm100::mbar_init(&tempty_bar[b], 128);
+      sm100::mbar_init(&tempty_bar[b], PAIR ? 8 : 4);   // one arrival per epilogue warp
     }
     *abort_flag = 0;
     sm100::fence_mbar_init();
@@ -274,11 +293,17 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     }
   }
   if (warp == 1) {
-    sm100::tmem_alloc(tmem_slot, TC_TMEM_COLS);
-    sm100::tmem_relinquish();
+    if (PAIR) {
+      sm100::tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
+      sm100::tmem_relinquish_pair();
+    } else {
+      sm100::tmem_alloc(tmem_slot, TC_TMEM_COLS);
+      sm100::tmem_relinquish();
+    }
   }
   sm100::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR) sm100::cluster_sync(); else __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -289,45 +314,51 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase_mask = 0;  // per stage: loads issued / their phase
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
-        const TileCoord tc = decode_tile(p, t);
+      for (int t = unit; t < p.total_tiles && ok; t += nunits) {
+        const TileCoord tc = decode_tile<C::BM>(p, t);
         const GemmProblem& q = p.prob[tc.prob];
-        const int kblocks = (q.K + TC_BK - 1) / TC_BK;
+        const int kblocks = (q.K + C::BK - 1) / C::BK;
+        const int arow = tc.tm * C::BM + rank * C::A_ROWS;
+        const int brow = tc.tn * TC_BN + rank * C::B_ROWS;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!sm100::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
             record_timeout(p.status, abort_flag);
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * TC_STAGE_BYTES;
-          uint8_t* sb = sa + TC_A_BYTES;
-          sm100::mbar_arrive_expect_tx(&full_bar[stage], TC_STAGE_BYTES);
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          if (!PAIR || rank == 0)
+            sm100::mbar_arrive_expect_tx(&full_bar[stage], (PAIR ? 2 : 1) * C::STAGE_BYTES);
           issued_mask |= 1u << stage;
           issued_phase_mask = (issued_phase_mask & ~(1u << stage)) | (phase << stage);
-          const int k0 = kb * TC_BK;
+          const int k0 = kb * C::BK;
+          const uint32_t leader_full = PAIR ? sm100::mapa_shared(sm100::smem_u32(&full_bar[stage]), 0) : 0;
+          auto load = [&](uint8_t* dst, const CUtensorMap* m, int x, int y) {
+            if (PAIR) sm100::tma_load_3d_pair(dst, m, leader_full, x, y, tc.mat);
+            else sm100::tma_load_3d(dst, m, &full_bar[stage], x, y, tc.mat);
+          };
           if (!q.a_mn) {
-            sm100::tma_load_3d(sa, &p.tmA[tc.prob], &full_bar[stage], k0, tc.tm * TC_BM, tc.mat);
+            load(sa, &p.tmA[tc.prob], k0, arow);
           } else {
 #pragma unroll
-            for (int h = 0; h < TC_BM / 64; ++h)
-              sm100::tma_load_3d(sa + h * 8192, &p.tmA[tc.prob], &full_bar[stage], tc.tm * TC_BM + h * 64, k0, tc.mat);
+            for (int h = 0; h < C::A_ROWS / 64; ++h) load(sa + h * 8192, &p.tmA[tc.prob], arow + h * 64, k0);
           }
           if (!q.b_mn) {
-            sm100::tma_load_3d(sb, &p.tmB[tc.prob], &full_bar[stage], k0, tc.tn * TC_BN, tc.mat);
+            load(sb, &p.tmB[tc.prob], k0, brow);
           } else {
 #pragma unroll
-            for (int h = 0; h < TC_BN / 64; ++h)
-              sm100::tma_load_3d(sb + h * 8192, &p.tmB[tc.prob], &full_bar[stage], tc.tn * TC_BN + h * 64, k0, tc.mat);
+            for (int h = 0; h < C::B_ROWS / 64; ++h) load(sb + h * 8192, &p.tmB[tc.prob], brow + h * 64, k0);
           }
-          if (++stage == TC_STAGES) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (!ok) {
-        // drain: let every load this thread issued land before the CTA exits
-        for (int s = 0; s < TC_STAGES; ++s) {
+      if (!ok && (!PAIR || rank == 0)) {
+        // drain: let every load issued into this CTA's barriers land before exit
+        for (int s = 0; s < C::STAGES; ++s) {
           if (!((issued_mask >> s) & 1u)) continue;
           const uint64_t t0 = sm100::globaltimer();
           while (!sm100::mbar_try_wait(&full_bar[s], (issued_phase_mask >> s) & 1u) &&
@@ -338,17 +369,17 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && (!PAIR || rank == 0)) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
-        const TileCoord tc = decode_tile(p, t);
+      for (int t = unit; t < p.total_tiles && ok; t += nunits) {
+        const TileCoord tc = decode_tile<C::BM>(p, t);
         const GemmProblem& q = p.prob[tc.prob];
-        const int kblocks = (q.K + TC_BK - 1) / TC_BK;
-        const uint32_t idesc = sm100::make_idesc_bf16(TC_BM, TC_BN, q.a_mn, q.b_mn);
+        const int kblocks = (q.K + C::BK - 1) / C::BK;
+        const uint32_t idesc = sm100::make_idesc_bf16(C::BM, TC_BN, q.a_mn, q.b_mn);
         if (!sm100::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) {
           record_timeout(p.status, abort_flag);
           break;
@@ -362,24 +393,27 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
             break;
           }
           sm100::tc_fence_after();
-          const uint32_t sa = sm100::smem_u32(smem + stage * TC_STAGE_BYTES);
-          const uint32_t sb = sa + TC_A_BYTES;
+          const uint32_t sa = sm100::smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
             const uint64_t ad = q.a_mn ? sm100::make_sdesc(sa + kk * 2048, 8192, 1024)
                                        : sm100::make_sdesc(sa + kk * 32, 16, 1024);
             const uint64_t bd = q.b_mn ? sm100::make_sdesc(sb + kk * 2048, 8192, 1024)
                                        : sm100::make_sdesc(sb + kk * 32, 16, 1024);
-            sm100::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+            if (PAIR) sm100::umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+            else sm100::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
           }
-          sm100::umma_commit(&empty_bar[stage]);
-          if (++stage == TC_STAGES) {
+          if (PAIR) sm100::umma_commit_pair_both(&empty_bar[stage]);
+          else sm100::umma_commit(&empty_bar[stage]);
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        sm100::umma_commit(&tfull_bar[acc]);
+        if (PAIR) sm100::umma_commit_pair_both(&tfull_bar[acc]);
+        else sm100::umma_commit(&tfull_bar[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
@@ -387,13 +421,14 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   } else {
     // ----------------------------------------------------------- epilogue
     const int quad = warp & 3;
-    const int row_in_tile = quad * 32 + lane;
+    const int row_in_cta = quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-      const TileCoord tc = decode_tile(p, t);
+    for (int t = unit; t < p.total_tiles; t += nunits) {
+      const TileCoord tc = decode_tile<C::BM>(p, t);
       const GemmProblem& q = p.prob[tc.prob];
-      const int i = tc.tm * TC_BM + row_in_tile;
+      const int row0 = tc.tm * C::BM + rank * 128;   // first row this CTA holds
+      const int i = row0 + row_in_cta;
       epilogue_prefetch<EPI>(p, q, tc.mat, i, tc.tn * TC_BN);
       bool wvec = true;
       if (EPI == EPI_AXPY_UPDATE && i < q.M) {
@@ -413,9 +448,10 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         if (j0 >= q.N) break;  // warp-uniform
         bool mirror = false;
         if (q.sym) {
-          const int jb = j0 / TC_BM;        // 128-wide column block
-          if (jb < tc.tm) continue;         // strictly lower block: produced by its mirror
-          mirror = jb > tc.tm;
+          const int ib = row0 / 128;        // 128-row block of this CTA's rows
+          const int jb = j0 / 128;          // 128-wide column block
+          if (jb < ib) continue;            // strictly lower block: produced by its mirror
+          mirror = jb > ib;
         }
         const bool full = (j0 + 32 <= q.N);
         EpiIn in;
@@ -425,42 +461,84 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, mirror, in, v);
       }
       sm100::tc_fence_before();
-      sm100::mbar_arrive(&tempty_bar[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR) sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_u32(&tempty_bar[acc]), 0));
+        else sm100::mbar_arrive(&tempty_bar[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   sm100::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR) sm100::cluster_sync(); else __syncthreads();
   sm100::tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    sm100::tmem_dealloc(tmem_base, TC_TMEM_COLS);
+    if (PAIR) sm100::tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
+    else sm100::tmem_dealloc(tmem_base, TC_TMEM_COLS);
   }
 }
 
 // ---------------------------------------------------------------- launcher
-int tc_tile_m() { return TC_BM; }
+int tc_tile_m(bool pair) { return pair ? TcCfg<true>::BM : TcCfg<false>::BM; }
 int tc_tile_n() { return TC_BN; }
+int tc_b_box_rows(bool pair) { return pair ? TcCfg<true>::B_ROWS : TcCfg<false>::B_ROWS; }
 
-template <int EPI>
-static cudaError_t launch_tc_epi(const TcGemmParams& p, int grid, cudaStream_t s) {
-  auto kern = tc_gemm_kernel<EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
+template <int EPI, bool PAIR>
+static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_t s) {
+  using C = TcCfg<PAIR>;
+  auto kern = tc_gemm_kernel<EPI, PAIR>;
+  static thread_local int max_units = 0;   // co-resident tile units (CTAs or CTA pairs)
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, TC_THREADS, TC_SMEM_BYTES, s>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(TC_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_units == 0) {
+      cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+        clusters = num_sms / 2;
+      max_units = clusters;
+    }
+  } else {
+    max_units = num_sms;
+  }
+  const int units = p.total_tiles < max_units ? p.total_tiles : max_units;
+  cfg.gridDim = dim3((PAIR ? 2 : 1) * units, 1, 1);
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, int num_sms, cudaStream_t s) {
+cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
-  const int grid = p.total_tiles < num_sms ? p.total_tiles : num_sms;
-  switch (epi) {
-    case EPI_GRAM: return launch_tc_epi<EPI_GRAM>(p, grid, s);
-    case EPI_POLY: return launch_tc_epi<EPI_POLY>(p, grid, s);
-    case EPI_AXPY: return launch_tc_epi<EPI_AXPY>(p, grid, s);
-    case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE>(p, grid, s);
+  if (pair) {
+    switch (epi) {
+      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, true>(p, num_sms, s);
+      case EPI_POLY: return launch_tc_epi<EPI_POLY, true>(p, num_sms, s);
+      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, true>(p, num_sms, s);
+      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, true>(p, num_sms, s);
+    }
+  } else {
+    switch (epi) {
+      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, false>(p, num_sms, s);
+      case EPI_POLY: return launch_tc_epi<EPI_POLY, false>(p, num_sms, s);
+      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, false>(p, num_sms, s);
+      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, false>(p, num_sms, s);
+    }
   }
   return cudaErrorInvalidValue;
 }

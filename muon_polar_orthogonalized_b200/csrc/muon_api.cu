@@ -29,9 +29,10 @@ cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
-int tc_tile_m();
+int tc_tile_m(bool pair);
 int tc_tile_n();
-cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, int num_sms, cudaStream_t s);
+int tc_b_box_rows(bool pair);
+cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, int num_sms, cudaStream_t s);
 int simt_tile();
 cudaError_t launch_simt_gemm(const SimtGemmParams& p, int epi, int num_sms, cudaStream_t s);
 }  // namespace muon
@@ -452,8 +453,10 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
   const bool f32 = (a.flags & MUON_FP32_DEBUG) != 0;
   const float ca = a.coeffs[3 * k], cb = a.coeffs[3 * k + 1], cc = a.coeffs[3 * k + 2];
   const float* scales = reinterpret_cast<const float*>(a.ws + w.scales_off);
-  const int BM = f32 ? simt_tile() : tc_tile_m();
+  const bool pair = (a.flags & MUON_TC_SINGLE_CTA) == 0;
+  const int BM = f32 ? simt_tile() : tc_tile_m(pair);
   const int BN = f32 ? simt_tile() : tc_tile_n();
+  const int b_rows = tc_b_box_rows(pair);
 
   static thread_local TcGemmParams TP;
   static thread_local SimtGemmParams SP;
@@ -482,7 +485,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       TP.cautious = (a.flags & MUON_CAUTIOUS_WD) ? 1 : 0;
       const int kind = epi == EPI_GRAM ? K_GRAM : epi == EPI_POLY ? K_POLY
                      : epi == EPI_AXPY ? K_AXPY : K_AXPY_UPDATE;
-      e = timed_launch(kind, a.stream, [&] { return launch_tc_gemm(TP, epi, C.dev.sms, a.stream); });
+      e = timed_launch(kind, a.stream, [&] { return launch_tc_gemm(TP, epi, pair, C.dev.sms, a.stream); });
     }
     if (e != cudaSuccess) return cuda_fail(e, "NS GEMM launch");
     reset();
@@ -549,7 +552,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
     P.tiles_n = (P.N + BN - 1) / BN;
     if (P.sym) {
       int t = 0;
-      for (int I = 0; I < P.tiles_m; ++I) t += P.tiles_n - (I >> 1);
+      for (int I = 0; I < P.tiles_m; ++I) t += P.tiles_n - (I * BM) / BN;
       P.tiles_per_mat = t;
     } else {
       P.tiles_per_mat = P.tiles_m * P.tiles_n;
@@ -565,18 +568,19 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
                         bstride, 64, mn ? 64 : box_rows);
       };
       muon_status st;
+      // A boxes: 128 rows per CTA; B boxes: the rows of B this CTA stages
       if (epi == EPI_GRAM) {
         st = map_for(&TP.tmA[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, 256);
+        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, b_rows);
       } else if (epi == EPI_POLY) {
         st = map_for(&TP.tmA[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, 256);
+        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, b_rows);
       } else if (!q.tall) {
         st = map_for(&TP.tmA[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, 1, q.c, q.r, q.ldc, q.xstride, 256);
+        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, 1, q.c, q.r, q.ldc, q.xstride, b_rows);
       } else {
         st = map_for(&TP.tmA[nprob], xcur, 0, q.c, q.r, q.ldc, q.xstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, 256);
+        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, b_rows);
       }
       if (st != MUON_OK) return st;
       TP.prob[nprob] = P;
@@ -638,7 +642,8 @@ muon_status validate_common(const muon_group* groups, int n_groups, int ns_steps
                             uint32_t flags, void* workspace, size_t workspace_bytes) {
   muon_status st = validate_groups(groups, n_groups);
   if (st != MUON_OK) return st;
-  if (flags & ~(MUON_NESTEROV | MUON_CAUTIOUS_WD | MUON_FP32_DEBUG | MUON_UNFUSED_UPDATE))
+  if (flags & ~(MUON_NESTEROV | MUON_CAUTIOUS_WD | MUON_FP32_DEBUG | MUON_UNFUSED_UPDATE |
+                MUON_TC_SINGLE_CTA))
     return fail(MUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (ns_steps < 0 || ns_steps > kMaxNsSteps)
     return fail(MUON_ERR_INVALID_ARG, "ns_steps %d outside [0, %d]", ns_steps, kMaxNsSteps);
@@ -699,7 +704,7 @@ muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs,
                                int n_groups, int ns_steps, const float* coeffs, uint32_t flags,
                                void* workspace, size_t workspace_bytes, muon_stream_t stream) {
   g_err[0] = '\0';
-  flags &= MUON_FP32_DEBUG;
+  flags &= (MUON_FP32_DEBUG | MUON_TC_SINGLE_CTA);
   muon_status st = validate_common(groups, n_groups, ns_steps, coeffs, flags, workspace, workspace_bytes);
   if (st != MUON_OK) return st;
   if ((st = validate_ptrs("inputs", inputs, groups, n_groups)) != MUON_OK) return st;

@@ -149,6 +149,17 @@ def test_transpose_equivariance(dev):
     assert d == 0.0  # the tall path reads MN-major: the same products in the same order
 
 
+def test_pair_and_single_cta_kernels_agree(dev):
+    """CTA-pair (256x256) and single-CTA (128x256) tensor-core kernels compute
+    the same products in the same K order: identical bits, incl. ragged shapes."""
+    shapes = [(256, 1024), (1024, 256), (384, 640), (640, 384), (129, 257), (700, 700)]
+    a = orth_case(dev, shapes, "f32", seed=21)[1]
+    b = orth_case(dev, shapes, "f32", seed=21, flags=N.MUON_TC_SINGLE_CTA)[1]
+    for (r, c), x, y in zip(shapes, a, b):
+        print((r, c), "pair vs single max |diff|", np.abs(x - y).max())
+        assert np.array_equal(x, y), (r, c)
+
+
 def test_batch_invariance_and_determinism(dev):
     """A matrix alone and inside a batch give the same bits; so does a rerun."""
     x = wl.iid_normal((256, 512), 1.0, 77)
