@@ -121,6 +121,33 @@ muon_status muon_step(float* const* params, const void* const* grads, float* con
                       muon_stream_t stream);
 
 /*
+ * muon_step without a caller workspace, for callers that cannot allocate
+ * device memory (no counterpart on the optimizer pages: it is a deployment
+ * aid).  Programs whose device-memory budget is fixed at start-up by another
+ * runtime, or code running inside a framework callback that owns every
+ * allocation, cannot hand muon_step a workspace; this entry point takes its
+ * scratch from one built-in device array of MUON_NOALLOC_SCRATCH_BYTES instead
+ * and allocates nothing.
+ *
+ * Same arguments and semantics as muon_step, minus the workspace.  Limit: the
+ * largest single matrix must fit, i.e. muon_workspace_min_size(groups) <=
+ * MUON_NOALLOC_SCRATCH_BYTES (32 MiB: e.g. up to 2048 x 2048 or 1024 x 4096);
+ * larger sets are processed in waves; a matrix that does not fit returns
+ * MUON_ERR_WORKSPACE with the sizes in muon_last_error().  Every GPU that
+ * loads this library holds the array until the process exits.  The first
+ * call on a device looks up the array's device address (make it before any
+ * stream capture).  All calls on a device share the array: calls that overlap
+ * on the GPU race and must be ordered by the caller (e.g. one stream).
+ * muon_query_status(NULL, ...) cannot read its status word; a device-side
+ * timeout is not reported for this entry point.
+ */
+#define MUON_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+muon_status muon_step_noalloc(float* const* params, const void* const* grads,
+                              float* const* momentum, const muon_group* groups, int n_groups,
+                              float lr, float beta, float wd, int ns_steps, const float* coeffs,
+                              uint32_t flags, muon_stream_t stream);
+
+/*
  * The orthogonaliser alone: outputs[i] <- NS(inputs[i]) as fp32, rows x cols,
  * with the same normalisation, orientation, iteration and bf16 rounding of
  * the result as muon_step.  inputs[i] dtype per group.  Only MUON_FP32_DEBUG

@@ -53,6 +53,9 @@ static muon_status cuda_fail(cudaError_t e, const char* what) {
   return fail(MUON_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// Lets other translation units of this library set the muon_last_error() text.
+void muon_set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 // ============================================================== profiler
 namespace {
 enum Kind {
