@@ -211,7 +211,7 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     wl = W.get(args.workload)
     D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e)
-    flags = N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD
+    flags = N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
     ws_bytes = api.muon_workspace_size(D.groups, flags)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     coeffs = W.NS_COEFFS_FIXED
@@ -360,7 +360,8 @@ def run_gpu(args):
             "config": {"workload": wl.name, "muon_params": wl.muon_params(), "adamw_params": wl.adamw_params(),
                        "muon_groups": [[s.rows, s.cols, s.count] for s in wl.muon],
                        "ns_steps": K, "grads": "bf16", "params_state": "fp32",
-                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"},
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
+                       "gemm_tiles": "128x256 single-CTA" if args.single_cta else "256x256 CTA pair"},
             "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_ms_per_step": round(ns_ms, 3),
@@ -455,6 +456,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single-cta", action="store_true",
+                    help="Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of CTA pairs")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -22,10 +22,50 @@
 
 namespace muon {
 
+// Launch shapes, chosen by measurement on B200 (isolated, 1G elements):
+// the momentum / update kernels stream 2-3 arrays and run best at full
+// occupancy (8 x 256 threads per SM) with 2 vec4 units per thread; AdamW
+// streams 4 arrays and runs best with 4 units per thread at 4 blocks per SM.
+#ifndef MUON_ELT_UNROLL
+#define MUON_ELT_UNROLL 2
+#endif
+#ifndef MUON_ELT_MIN_BLOCKS
+#define MUON_ELT_MIN_BLOCKS 8
+#endif
+#ifndef MUON_ADAM_UNROLL
+#define MUON_ADAM_UNROLL 4
+#endif
+#ifndef MUON_ADAM_MIN_BLOCKS
+#define MUON_ADAM_MIN_BLOCKS 4
+#endif
 constexpr int kEltThreads = 256;
-constexpr int kEltUnroll = 4;                                // vec4 units per thread
-constexpr int kEltMinBlocks = 4;                             // resident blocks per SM (occupancy)
-constexpr int kEltChunk = kEltThreads * kEltUnroll * 4;      // elements per block
+constexpr int kEltUnroll = MUON_ELT_UNROLL;                  // vec4 units per thread
+constexpr int kEltMinBlocks = MUON_ELT_MIN_BLOCKS;           // resident blocks per SM (occupancy)
+constexpr int kEltChunk = kEltThreads * kEltUnroll * 4;      // elements per work chunk
+constexpr int kAdamUnroll = MUON_ADAM_UNROLL;
+constexpr int kAdamMinBlocks = MUON_ADAM_MIN_BLOCKS;
+constexpr int kAdamChunk = kEltThreads * kAdamUnroll * 4;
+
+// Streaming accesses (each element read and written once per step).
+#ifndef MUON_ELT_STREAM_HINTS
+#define MUON_ELT_STREAM_HINTS 0
+#endif
+template <typename T>
+__device__ __forceinline__ T ld_stream(const T* p) {
+#if MUON_ELT_STREAM_HINTS
+  return __ldcs(p);
+#else
+  return *p;
+#endif
+}
+template <typename T>
+__device__ __forceinline__ void st_stream(T* p, T v) {
+#if MUON_ELT_STREAM_HINTS
+  __stcs(p, v);
+#else
+  *p = v;
+#endif
+}
 
 __device__ __forceinline__ int find_mat(const MatRef* mats, int n, int blk) {
   int lo = 0, hi = n - 1;
@@ -45,13 +85,13 @@ __device__ __forceinline__ float round_bf16(float v) {
 template <bool BF16>
 __device__ __forceinline__ float4 load_g4(const void* g, long long e) {
   if constexpr (BF16) {
-    uint2 raw = __ldcs(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(g) + e));
+    uint2 raw = ld_stream(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(g) + e));
     __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
     __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
     float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
     return make_float4(fa.x, fa.y, fb.x, fb.y);
   } else {
-    return __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(g) + e));
+    return ld_stream(reinterpret_cast<const float4*>(static_cast<const float*>(g) + e));
   }
 }
 template <bool BF16>
@@ -128,7 +168,7 @@ __device__ __forceinline__ float momentum_chunk(const EltParams& p, const MatRef
       const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
       if (e < numel) {
         gv[u] = load_g4<GBF16>(r.g, e);
-        mv[u] = r.m ? __ldcs(reinterpret_cast<const float4*>(r.m + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        mv[u] = r.m ? ld_stream(reinterpret_cast<const float4*>(r.m + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
@@ -142,7 +182,7 @@ __device__ __forceinline__ float momentum_chunk(const EltParams& p, const MatRef
           mn.y = fmaf(beta, mv[u].y, gv[u].y);
           mn.z = fmaf(beta, mv[u].z, gv[u].z);
           mn.w = fmaf(beta, mv[u].w, gv[u].w);
-          __stcs(reinterpret_cast<float4*>(r.m + e), mn);
+          st_stream(reinterpret_cast<float4*>(r.m + e), mn);
           if (p.nesterov) {
             mt.x = fmaf(beta, mn.x, gv[u].x);
             mt.y = fmaf(beta, mn.y, gv[u].y);
@@ -245,7 +285,7 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
       const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
       if (e < numel) {
         xv[u] = load_x4(r.x, x_index(r, e), f32x);
-        if (!EMIT) wv[u] = __ldcs(reinterpret_cast<const float4*>(r.w + e));
+        if (!EMIT) wv[u] = ld_stream(reinterpret_cast<const float4*>(r.w + e));
       }
     }
 #pragma unroll
@@ -254,14 +294,14 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
       if (e < numel) {
         float4 uu = make_float4(make_u(xv[u].x), make_u(xv[u].y), make_u(xv[u].z), make_u(xv[u].w));
         if (EMIT) {
-          __stcs(reinterpret_cast<float4*>(r.out + e), uu);
+          st_stream(reinterpret_cast<float4*>(r.out + e), uu);
         } else {
           float4 w = wv[u];
           w.x = cautious_apply(w.x, uu.x, r.lr, p.wd, p.cautious);
           w.y = cautious_apply(w.y, uu.y, r.lr, p.wd, p.cautious);
           w.z = cautious_apply(w.z, uu.z, r.lr, p.wd, p.cautious);
           w.w = cautious_apply(w.w, uu.w, r.lr, p.wd, p.cautious);
-          __stcs(reinterpret_cast<float4*>(r.w + e), w);
+          st_stream(reinterpret_cast<float4*>(r.w + e), w);
         }
       }
     }
@@ -308,7 +348,7 @@ __device__ __forceinline__ void adam_elem(const AdamTensor& T, float g, float& p
 template <bool GBF16>
 __device__ __forceinline__ void adamw_chunk(const AdamTensor& T, long long e0) {
   if (T.vec) {
-    constexpr int U = kEltUnroll / 2;  // 4 streams per element: keep registers in check
+    constexpr int U = kAdamUnroll / 2;  // 4 streams per element: two halves keep registers in check
 #pragma unroll 1
     for (int half = 0; half < 2; ++half) {
       float4 gv[U], pv[U], mv[U], vv[U];
@@ -318,9 +358,9 @@ __device__ __forceinline__ void adamw_chunk(const AdamTensor& T, long long e0) {
             e0 + (static_cast<long long>(half * U + u) * kEltThreads + threadIdx.x) * 4;
         if (e < T.numel) {
           gv[u] = load_g4<GBF16>(T.g, e);
-          pv[u] = __ldcs(reinterpret_cast<const float4*>(T.p + e));
-          mv[u] = __ldcs(reinterpret_cast<const float4*>(T.m + e));
-          vv[u] = __ldcs(reinterpret_cast<const float4*>(T.v + e));
+          pv[u] = ld_stream(reinterpret_cast<const float4*>(T.p + e));
+          mv[u] = ld_stream(reinterpret_cast<const float4*>(T.m + e));
+          vv[u] = ld_stream(reinterpret_cast<const float4*>(T.v + e));
         }
       }
 #pragma unroll
@@ -332,14 +372,14 @@ __device__ __forceinline__ void adamw_chunk(const AdamTensor& T, long long e0) {
           adam_elem(T, gv[u].y, pv[u].y, mv[u].y, vv[u].y);
           adam_elem(T, gv[u].z, pv[u].z, mv[u].z, vv[u].z);
           adam_elem(T, gv[u].w, pv[u].w, mv[u].w, vv[u].w);
-          __stcs(reinterpret_cast<float4*>(T.p + e), pv[u]);
-          __stcs(reinterpret_cast<float4*>(T.m + e), mv[u]);
-          __stcs(reinterpret_cast<float4*>(T.v + e), vv[u]);
+          st_stream(reinterpret_cast<float4*>(T.p + e), pv[u]);
+          st_stream(reinterpret_cast<float4*>(T.m + e), mv[u]);
+          st_stream(reinterpret_cast<float4*>(T.v + e), vv[u]);
         }
       }
     }
   } else {
-    for (int u = 0; u < kEltUnroll * 4; ++u) {
+    for (int u = 0; u < kAdamUnroll * 4; ++u) {
       const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
       if (e < T.numel) {
         float pp = T.p[e], mm = T.m[e], vv = T.v[e];
@@ -353,16 +393,17 @@ __device__ __forceinline__ void adamw_chunk(const AdamTensor& T, long long e0) {
 }
 
 template <bool GBF16>
-__global__ void __launch_bounds__(kEltThreads, kEltMinBlocks)
+__global__ void __launch_bounds__(kEltThreads, kAdamMinBlocks)
 adamw_kernel(const __grid_constant__ AdamParams P) {
   for (int blk = blockIdx.x; blk < P.total_blocks; blk += gridDim.x) {
     const AdamTensor& T = P.t[find_tensor(P.t, P.ntensors, blk)];
-    adamw_chunk<GBF16>(T, static_cast<long long>(blk - T.blk_begin) * kEltChunk);
+    adamw_chunk<GBF16>(T, static_cast<long long>(blk - T.blk_begin) * kAdamChunk);
   }
 }
 
 // ------------------------------------------------------------- launchers
 int elt_chunk() { return kEltChunk; }
+int adam_chunk() { return kAdamChunk; }
 
 // Persistent grid: every SM filled to its occupancy limit, never more blocks
 // than chunks.

@@ -37,6 +37,13 @@ namespace muon {
 // and 128 rows (N/2) of B, the leader issues one 256x256x16 MMA per K step
 // that reads both CTAs' shared memory, and each CTA's TMEM holds its 128
 // accumulator rows.
+#ifndef MUON_TC_PAIR_STAGES
+#define MUON_TC_PAIR_STAGES 6
+#endif
+#ifndef MUON_TC_RASTER_GN
+#define MUON_TC_RASTER_GN 8
+#endif
+
 template <bool PAIR>
 struct TcCfg {
   static constexpr int BM = PAIR ? 256 : 128;        // tile rows
@@ -47,13 +54,13 @@ struct TcCfg {
   static constexpr int A_BYTES = A_ROWS * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int STAGES = PAIR ? MUON_TC_PAIR_STAGES : 4;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 };
 constexpr int TC_BN = 256;
 constexpr int TC_THREADS = 192;
 constexpr int TC_TMEM_COLS = 512;
-constexpr int TC_RASTER_GN = 8;   // tile-column band width of the non-symmetric raster
+constexpr int TC_RASTER_GN = MUON_TC_RASTER_GN;   // tile-column band width of the non-symmetric raster
 
 struct TileCoord {
   int prob, mat, tm, tn;

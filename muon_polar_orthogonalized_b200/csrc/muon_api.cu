@@ -25,6 +25,7 @@
 namespace muon {
 // kernels (k_elementwise.cu, k_gemm_tc.cu, k_gemm_simt.cu)
 int elt_chunk();
+int adam_chunk();
 cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
@@ -748,7 +749,7 @@ muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step, mu
   if (st != MUON_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   static thread_local AdamParams P;
-  const int chunk = elt_chunk();
+  const int chunk = adam_chunk();
   for (int dt = 0; dt < 2; ++dt) {
     std::memset(&P, 0, sizeof(P));
     P.grad_bf16 = dt;
