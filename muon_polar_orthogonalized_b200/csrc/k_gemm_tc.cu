@@ -58,7 +58,15 @@ struct TcCfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 };
 constexpr int TC_BN = 256;
-constexpr int TC_THREADS = 192;
+#ifndef MUON_TC_EPI_WARPS
+#define MUON_TC_EPI_WARPS 8
+#endif
+// Epilogue warps: a multiple of 4, since warp w may only read TMEM lanes
+// 32*(w%4) .. +31; with 8, two warps share each lane quadrant and split the
+// tile's 256 columns between them.
+constexpr int TC_EPI_WARPS = MUON_TC_EPI_WARPS;
+constexpr int TC_EPI_SPLIT = TC_EPI_WARPS / 4;          // column slices per lane quadrant
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;       // producer + MMA + epilogue warps
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_RASTER_GN = MUON_TC_RASTER_GN;   // tile-column band width of the non-symmetric raster
 
@@ -142,9 +150,9 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const GemmProblem& q,
-                                                  int mat, int i, int jt) {
+                                                  int mat, int i, int jt, int width) {
   if (EPI == EPI_GRAM || i >= q.M) return;
-  const int ncols = min(TC_BN, q.N - jt);  // jt < N
+  const int ncols = min(width, q.N - jt);  // jt < N
   const char* ein = reinterpret_cast<const char*>(
       static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
   for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
@@ -290,7 +298,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     }
     for (int b = 0; b < 2; ++b) {
       sm100::mbar_init(&tfull_bar[b], 1);
-      sm100::mbar_init(&tempty_bar[b], PAIR ? 8 : 4);   // one arrival per epilogue warp
+      sm100::mbar_init(&tempty_bar[b], (PAIR ? 2 : 1) * TC_EPI_WARPS);   // one arrival per epilogue warp
     }
     *abort_flag = 0;
     sm100::fence_mbar_init();
@@ -427,7 +435,9 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    const int quad = warp & 3;
+    const int quad = warp & 3;                          // TMEM lane quadrant this warp may read
+    const int slice = (warp - 2) / 4;                   // which column slice of the tile
+    constexpr int kChunks = TC_BN / 32 / TC_EPI_SPLIT;  // 32-column chunks per warp
     const int row_in_cta = quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -436,7 +446,8 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       const GemmProblem& q = p.prob[tc.prob];
       const int row0 = tc.tm * C::BM + rank * 128;   // first row this CTA holds
       const int i = row0 + row_in_cta;
-      epilogue_prefetch<EPI>(p, q, tc.mat, i, tc.tn * TC_BN);
+      const int jslice = tc.tn * TC_BN + slice * kChunks * 32;
+      if (jslice < q.N) epilogue_prefetch<EPI>(p, q, tc.mat, i, jslice, kChunks * 32);
       bool wvec = true;
       if (EPI == EPI_AXPY_UPDATE && i < q.M) {
         const int wi = q.w_first + tc.mat;
@@ -450,7 +461,8 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * TC_BN);
 #pragma unroll 1
-      for (int c = 0; c < TC_BN / 32; ++c) {
+      for (int cc = 0; cc < kChunks; ++cc) {
+        const int c = slice * kChunks + cc;
         const int j0 = tc.tn * TC_BN + c * 32;
         if (j0 >= q.N) break;  // warp-uniform
         bool mirror = false;
