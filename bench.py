@@ -126,7 +126,7 @@ class DeviceWorkload:
     """All tensors of a workload resident on one GPU: params / momentum / grads
     as views into one flat buffer per shape group (16-byte aligned views)."""
 
-    def __init__(self, wl, device, e2e_host: bool = False):
+    def __init__(self, wl, device, e2e_host: bool = False, pinned: bool = True):
         import torch
         from muon_polar_orthogonalized_b200 import _native as N
         from muon_polar_orthogonalized_b200 import workloads as W
@@ -175,8 +175,10 @@ class DeviceWorkload:
                 self.flat_grads.append(g.view(-1))
             self.adam.append((ps, gs, ms, vs, t))
         self.host_grads = None
+        self.host_pinned = False
         if e2e_host:
-            self.host_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in self.flat_grads]
+            self.host_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=pinned) for g in self.flat_grads]
+            self.host_pinned = pinned
             for h, g in zip(self.host_grads, self.flat_grads):
                 h.copy_(g)
 
@@ -187,30 +189,79 @@ class DeviceWorkload:
                               W.ADAMW_EPS, t.wd) for (ps, gs, ms, vs, t) in self.adam]
 
 
+class RankContext:
+    """Ranks of one benchmark job (torchrun env: RANK / LOCAL_RANK / WORLD_SIZE /
+    MASTER_*).  With one rank nothing is initialised.  The backend is "nccl"
+    on GPUs; the CPU tests drive the same logic with "gloo"."""
+
+    def __init__(self, backend: str = "nccl", timeout_s: int = 600):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.dist = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            self.dist = dist
+
+    @property
+    def is_root(self) -> bool:
+        return self.rank == 0
+
+    def barrier(self) -> None:
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        """Max of x over all ranks (every rank gets it)."""
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self) -> None:
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def pinned_fits(nbytes: int, ranks_on_host: int) -> bool:
+    """Pin host buffers for the end-to-end copies only if all ranks' buffers
+    leave a quarter of the host RAM free."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        return True
+    return nbytes * ranks_on_host < 0.75 * avail
+
+
 def run_gpu(args):
     import torch
-    import torch.distributed as dist
-
     from muon_polar_orthogonalized_b200 import _native as N
     from muon_polar_orthogonalized_b200 import api
     from muon_polar_orthogonalized_b200 import workloads as W
     from muon_polar_orthogonalized_b200.build import build
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    R = RankContext("nccl")
+    world, rank, local = R.world, R.rank, R.local
     if rank == 0:
         build()
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
-        dist.barrier()
-        if rank != 0:
-            build()
+    R.barrier()
+    if rank != 0:
+        build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = W.get(args.workload)
-    D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e)
+    grad_bytes = sum(s.rows * s.cols * s.count * (2 if s.grad_dtype == "bf16" else 4) for s in wl.muon) + \
+        sum(math.prod(t.shape) * t.count * (2 if t.grad_dtype == "bf16" else 4) for t in wl.adamw)
+    e2e_pinned = pinned_fits(grad_bytes, min(world, torch.cuda.device_count()))
+    D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e, pinned=e2e_pinned)
     flags = N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
     ws_bytes = api.muon_workspace_size(D.groups, flags)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -228,16 +279,11 @@ def run_gpu(args):
 
     def barrier():
         torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
+        R.barrier()
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return R.max(x, device=dev)
 
     for _ in range(args.warmup):
         step()
@@ -281,7 +327,8 @@ def run_gpu(args):
         e2e_ms = max_over_ranks(a0.elapsed_time(a1)) / args.steps
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": 4,
-               "path": "pinned host grads -> cudaMemcpyAsync -> muon_step + adamw_step -> status word read"}
+               "path": ("pinned" if D.host_pinned else "pageable") +
+                       " host grads -> cudaMemcpyAsync -> muon_step + adamw_step -> status word read"}
 
     if rank == 0:
         work = algorithmic_work(wl)
@@ -376,9 +423,7 @@ def run_gpu(args):
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(wl, reps=1)
         print(json.dumps(res), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    R.close()
 
 
 # --------------------------------------------------------- CPU (oracle)
@@ -427,9 +472,8 @@ def cpu_baseline(wl, reps: int = 1):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return
+    if int(os.environ.get("RANK", "0")) != 0:
+        return  # the oracle arm runs on rank 0 only; other ranks exit without work
     from muon_polar_orthogonalized_b200 import workloads as W
     wl = W.get(args.workload)
     for _ in range(args.warmup):
