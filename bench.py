@@ -119,7 +119,7 @@ def algorithmic_work(wl):
         gb = 2 if t.grad_dtype == "bf16" else 4
         adam_bytes += t.count * math.prod(t.shape) * (gb + 24)
     return dict(gram_flops=gram, poly_flops=poly, axpy_flops=axpy, momentum_bytes=mom_bytes,
-                update_bytes=upd_bytes, adamw_bytes=adam_bytes)
+                update_bytes=upd_bytes, adamw_bytes=adam_bytes, rowscale_bytes=upd_bytes / 5.0)
 
 
 class DeviceWorkload:
@@ -262,7 +262,8 @@ def run_gpu(args):
         sum(math.prod(t.shape) * t.count * (2 if t.grad_dtype == "bf16" else 4) for t in wl.adamw)
     e2e_pinned = pinned_fits(grad_bytes, min(world, torch.cuda.device_count()))
     D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e, pinned=e2e_pinned)
-    flags = N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
+    flags = (N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
+             | (N.MUON_NORMUON if args.normuon else 0))
     ws_bytes = api.muon_workspace_size(D.groups, flags)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     coeffs = W.NS_COEFFS_FIXED
@@ -352,6 +353,7 @@ def run_gpu(args):
             "ns_axpy_update": ("tensor", work["axpy_flops"]),
             "momentum_norm": ("hbm", work["momentum_bytes"]),
             "update": ("hbm", work["update_bytes"]),
+            "row_scale": ("hbm", work["rowscale_bytes"]),
             "adamw": ("hbm", work["adamw_bytes"]),
         }
         # per-step algorithmic work of each kernel kind: GEMM kinds run once per
@@ -361,6 +363,7 @@ def run_gpu(args):
             "ns_axpy": work["axpy_flops"] * (K - 1 if "ns_axpy_update" in kinds else K),
             "ns_axpy_update": work["axpy_flops"],
             "momentum_norm": work["momentum_bytes"], "update": work["update_bytes"],
+            "row_scale": work["rowscale_bytes"],
             "adamw": work["adamw_bytes"]}
         roof = None
         if dom in alg:
@@ -384,7 +387,7 @@ def run_gpu(args):
                         "peak_source": f"{peak_src} (HBM copy)",
                         "work_per_launch": per_launch, "work_unit": "algorithmic bytes"}
         ew = {}
-        for k in ("momentum_norm", "update", "adamw"):
+        for k in ("momentum_norm", "update", "row_scale", "adamw"):
             if k in kinds:
                 ew[k] = round(per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e9, 1)
         for k in ("ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update"):
@@ -408,7 +411,8 @@ def run_gpu(args):
                        "muon_groups": [[s.rows, s.cols, s.count] for s in wl.muon],
                        "ns_steps": K, "grads": "bf16", "params_state": "fp32",
                        "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
-                       "gemm_tiles": "128x256 single-CTA" if args.single_cta else "256x256 CTA pair"},
+                       "gemm_tiles": "128x256 single-CTA" if args.single_cta else "256x256 CTA pair",
+                       "normuon": bool(args.normuon)},
             "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_ms_per_step": round(ns_ms, 3),
@@ -500,6 +504,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--normuon", action="store_true",
+                    help="row-normalise the orthogonalised update (NorMuon)")
     ap.add_argument("--single-cta", action="store_true",
                     help="Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of CTA pairs")
     args = ap.parse_args()

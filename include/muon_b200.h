@@ -66,8 +66,11 @@ enum {
   MUON_CAUTIOUS_WD = 2u,    /* decay only where update*param >= 0 (else plain decoupled decay) */
   MUON_FP32_DEBUG = 4u,     /* fp32 operands and fp32 FMA GEMMs (slow; tolerance 1e-4 mode) */
   MUON_UNFUSED_UPDATE = 8u, /* apply the update in its own kernel instead of the last B*X epilogue */
-  MUON_TC_SINGLE_CTA = 16u  /* run the Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of
+  MUON_TC_SINGLE_CTA = 16u, /* run the Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of
                                CTA-pair (cta_group::2) 256x256 tiles; same results, for comparison */
+  MUON_NORMUON = 32u        /* NorMuon ("Chapter 4: The MuonAdamW Optimizer", NorMuon): divide every
+                               row of U (parameter orientation) by (||row||/sqrt(cols) + 1e-8) before
+                               the decay and update, so each row's RMS is 1 and the step's is lr */
 };
 
 /*
@@ -103,6 +106,7 @@ size_t muon_workspace_min_size(const muon_group* groups, int n_groups, uint32_t 
  *                     ns_steps x { A = X X^T; B = b_k A + c_k A A; X = a_k X + B X }
  *                     (wide orientation: rows > cols iterates on X^T)
  *                     U  <- X (values rounded to bf16, as the pages keep X in bf16)
+ *                     (MUON_NORMUON: U_row <- U_row / (||U_row||/sqrt(cols) + 1e-8))
  *                     W  <- W - lr*lr_scale*(U + wd*mask*W),
  *                           mask = (U*W >= 0) with MUON_CAUTIOUS_WD, else 1
  *

@@ -5,8 +5,8 @@ sm_100a); this package only marshals arguments to it.  Importing the package
 does not load the library; the first call does, and raises if it is missing.
 """
 from ._native import (MUON_BF16, MUON_CAUTIOUS_WD, MUON_F32, MUON_FP32_DEBUG,  # noqa: F401
-                      MUON_NESTEROV, MUON_TC_SINGLE_CTA, MUON_UNFUSED_UPDATE, MuonError,
-                      MuonGroup)
+                      MUON_NESTEROV, MUON_NORMUON, MUON_TC_SINGLE_CTA, MUON_UNFUSED_UPDATE,
+                      MuonError, MuonGroup)
 from .api import (AdamWSpec, adamw_step, muon_orthogonalize, muon_profiler_enable,  # noqa: F401
                   muon_profiler_read, muon_profiler_reset, muon_query_status, muon_step,
                   muon_workspace_min_size, muon_workspace_size)

@@ -30,6 +30,7 @@ MUON_CAUTIOUS_WD = 2
 MUON_FP32_DEBUG = 4
 MUON_UNFUSED_UPDATE = 8
 MUON_TC_SINGLE_CTA = 16
+MUON_NORMUON = 32
 
 
 class MuonGroup(ctypes.Structure):

@@ -10,6 +10,8 @@
 //   update         W <- W - lr*(U + wd*mask*W), mask = (U*W >= 0) by sign bits
 //                  (nanochat discussion, mira687's reply: cautious weight decay)
 //   emit           out <- U as fp32 (orthogonaliser entry point)
+//   row_scale      NorMuon: s_row = 1/(||U_row||/sqrt(cols) + 1e-8), one warp
+//                  per row, fixed-order reduction ("Chapter 4", NorMuon)
 //   adamw          bias-corrected AdamW with decoupled decay
 //                  ("3.9 Optimizers", Implementing AdamW from scratch)
 //
@@ -278,6 +280,7 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
     if (!p.use_scale) return x;
     return f32x ? sc * x : round_bf16(sc * x);
   };
+  const float* rs = p.rowscale ? p.rowscale + r.rbase : nullptr;
   if (r.vec) {
     float4 xv[kEltUnroll], wv[kEltUnroll];
 #pragma unroll
@@ -293,6 +296,10 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
       const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
       if (e < numel) {
         float4 uu = make_float4(make_u(xv[u].x), make_u(xv[u].y), make_u(xv[u].z), make_u(xv[u].w));
+        if (rs) {
+          const float f = rs[static_cast<int>(e) / r.cols];  // a vec4 unit never crosses a row
+          uu.x *= f; uu.y *= f; uu.z *= f; uu.w *= f;
+        }
         if (EMIT) {
           st_stream(reinterpret_cast<float4*>(r.out + e), uu);
         } else {
@@ -309,7 +316,8 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
     for (int u = 0; u < kEltUnroll * 4; ++u) {
       const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
       if (e < numel) {
-        const float uu = make_u(load_x1(r.x, x_index(r, e), f32x));
+        float uu = make_u(load_x1(r.x, x_index(r, e), f32x));
+        if (rs) uu *= rs[static_cast<int>(e) / r.cols];
         if (EMIT) r.out[e] = uu;
         else r.w[e] = cautious_apply(r.w[e], uu, r.lr, p.wd, p.cautious);
       }
@@ -323,6 +331,36 @@ update_kernel(const __grid_constant__ EltParams p) {
   for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
     const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
     update_chunk<EMIT>(p, r, static_cast<long long>(blk - r.blk_begin) * kEltChunk);
+  }
+}
+
+// -------------------------------------------------------------- row_scale
+// One warp per row: rows of all matrices of the launch are numbered
+// consecutively (MatRef.blk_begin = first row of the matrix).  U is the value
+// the update kernel will use (the bf16 X, or bf16(s*X0) when no iteration
+// ran), squared and summed in fp32 per lane in column order, then reduced with
+// a fixed shuffle tree.
+__global__ void __launch_bounds__(kEltThreads)
+row_scale_kernel(const __grid_constant__ EltParams p) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = kEltThreads / 32;
+  const bool f32x = p.x_f32 != 0;
+  for (int row_g = blockIdx.x * wpb + (threadIdx.x >> 5); row_g < p.total_blocks;
+       row_g += gridDim.x * wpb) {
+    const MatRef& r = p.mats[find_mat(p.mats, p.nmats, row_g)];
+    const int row = row_g - r.blk_begin;
+    const float sc = p.use_scale ? p.scales[r.sidx] : 1.f;
+    const long long base = static_cast<long long>(row) * r.ldx;
+    float acc = 0.f;
+    for (int c = lane; c < r.cols; c += 32) {
+      float u = load_x1(r.x, base + c, f32x);
+      if (p.use_scale) u = f32x ? sc * u : round_bf16(sc * u);
+      acc = fmaf(u, u, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0)
+      p.rowscale[r.rbase + row] = 1.f / (sqrtf(acc / static_cast<float>(r.cols)) + 1e-8f);
   }
 }
 
@@ -431,6 +469,15 @@ cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s) {
     auto k = momentum_norm_kernel<false>;
     k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_scale(const EltParams& p, int sms, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  const int wpb = kEltThreads / 32;
+  const long long need = (static_cast<long long>(p.total_blocks) + wpb - 1) / wpb;
+  const long long cap = static_cast<long long>(sms) * 8;
+  row_scale_kernel<<<static_cast<int>(need < cap ? need : cap), kEltThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -25,6 +25,8 @@ from .muon_ref import (  # noqa: F401
     cautious_mask,
     cautious_weight_decay_update,
     muon_step,
+    normuon_rows,
+    NORMUON_EPS,
     adamw_step,
     round_bf16,
     newton_schulz_bf16_emulated,

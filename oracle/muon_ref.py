@@ -159,16 +159,34 @@ def cautious_weight_decay_update(w: np.ndarray, update: np.ndarray, lr: float, w
     return w - lr * (update + wd * mask * w)
 
 
+NORMUON_EPS = 1e-8
+
+
+def normuon_rows(update: np.ndarray, eps: float = NORMUON_EPS) -> np.ndarray:
+    """NorMuon ([MAC] "NorMuon: Normalized Muon"): every row of the update is
+    divided by (its norm / sqrt(number of columns) + 1e-8), so each row's RMS
+    becomes 1 (the learning rate then sets the step's RMS).  Rows are in the
+    parameter orientation (the last dimension of the returned update)."""
+    u = np.asarray(update, dtype=np.float64)
+    rms = np.sqrt(np.sum(u * u, axis=-1, keepdims=True)) / np.sqrt(u.shape[-1])
+    return u / (rms + eps)
+
+
 def muon_step(w: np.ndarray, g: np.ndarray, m: np.ndarray, lr: float, beta: float, wd: float,
               ns_steps: int = 5, coeffs=NS_COEFFS_FIXED, nesterov: bool = True,
-              cautious: bool = True, lr_scale: float = 1.0, eps: float = NS_EPS):
-    """One Muon step on one matrix: momentum -> NS -> cautious decay + update.
+              cautious: bool = True, lr_scale: float = 1.0, eps: float = NS_EPS,
+              normuon: bool = False):
+    """One Muon step on one matrix: momentum -> NS -> (NorMuon) -> cautious decay + update.
 
     Returns (w_new, m_new, update) in fp64.  lr_scale is the per-matrix shape
     factor some recipes multiply the learning rate by; 1 gives W -= lr*update.
+    With normuon the orthogonalised update is row-normalised first ([MAC]
+    "The Full Muon Step": normalize_muon_update, then decay, then the step).
     """
     m_new, mt = nesterov_momentum(m, g, beta, nesterov)
     u = newton_schulz(mt, coeffs, ns_steps, eps)
+    if normuon:
+        u = normuon_rows(u)
     w_new = cautious_weight_decay_update(w, u, lr * lr_scale, wd, cautious)
     return w_new, m_new, u
 

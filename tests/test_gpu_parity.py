@@ -348,6 +348,30 @@ def test_multi_wave_matches_single_wave(dev):
         assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("fp32", [False, True])
+@pytest.mark.parametrize("ns", [5, 0])
+def test_normuon_parity(dev, fp32, ns):
+    """NorMuon ("Chapter 4", NorMuon): rows of U normalised to RMS 1 before the
+    cautious decay and update, wide and tall matrices and a ragged shape."""
+    shapes = [(256, 1024), (1024, 256), (130, 200)]
+    groups, W, G, M, hW, hG = make_state(dev, shapes, "f32", 13)
+    flags = STEP_FLAGS | N.MUON_NORMUON | (N.MUON_FP32_DEBUG if fp32 else 0)
+    ws = workspace(api.muon_workspace_size(groups, flags), dev)
+    lr = 0.02
+    api.muon_step(W, G, M, groups, lr, 0.95, 0.01, ns, FIXED, flags, ws)
+    torch.cuda.synchronize()
+    for i, (r, c) in enumerate(shapes):
+        rw, rm, ru = oracle.muon_step(hW[i], hG[i], np.zeros_like(hW[i]), lr, 0.95, 0.01,
+                                      ns_steps=ns, normuon=True)
+        e = check_step(hW[i], host64(W[i]), host64(M[i]), rw, rm, tol=(TOL_F32 if fp32 else TOL_BF16))
+        # the applied step's rows: RMS = lr up to the decay term and eps
+        step = (hW[i] - host64(W[i])) / lr
+        decay_free = step - 0.01 * oracle.cautious_mask(ru, hW[i]) * hW[i]
+        rms = np.sqrt(np.mean(decay_free ** 2, axis=1))
+        assert np.allclose(rms, 1.0, rtol=2e-3 if fp32 else 2e-2), (r, c)
+        print((r, c), "ns", ns, "fp32" if fp32 else "bf16", "normuon step rel err", e)
+
+
 # ---------------------------------------------------------------- AdamW
 @pytest.mark.parametrize("gdt", ["f32", "bf16"])
 def test_adamw_parity(dev, gdt):

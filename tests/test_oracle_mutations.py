@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 from tests.test_oracle_pins import (adamw_pin_failures, momentum_pin_failures,
-                                    ns_pin_failures, update_pin_failures)
+                                    normuon_pin_failures, ns_pin_failures, update_pin_failures)
 
 
 def _coeffs(coeffs, steps):
@@ -161,3 +161,27 @@ def _adamw_variant(kind):
                                   "v_uses_abs", "decay_after"])
 def test_adamw_mutant_caught(kind):
     assert adamw_pin_failures(_adamw_variant(kind)) != []
+
+
+def _normuon_variant(kind):
+    def norm(u, eps=oracle.NORMUON_EPS):
+        u = np.asarray(u, dtype=np.float64)
+        if kind == "wrong_axis":
+            rms = np.sqrt(np.sum(u * u, axis=0, keepdims=True)) / np.sqrt(u.shape[0])
+        elif kind == "no_sqrt_cols":
+            rms = np.sqrt(np.sum(u * u, axis=-1, keepdims=True))
+        elif kind == "whole_matrix":
+            rms = np.sqrt(np.mean(u * u))
+        else:
+            rms = np.sqrt(np.sum(u * u, axis=-1, keepdims=True)) / np.sqrt(u.shape[-1])
+        return u / (rms + eps)
+    return norm
+
+
+@pytest.mark.parametrize("kind", ["wrong_axis", "no_sqrt_cols", "whole_matrix"])
+def test_normuon_mutant_caught(kind):
+    assert normuon_pin_failures(_normuon_variant(kind)) != []
+
+
+def test_normuon_unmutated_copy_passes():
+    assert normuon_pin_failures(_normuon_variant("none")) == []

@@ -339,6 +339,65 @@ def test_full_step_matches_closed_form():
 
 
 # ============================================================================
+# NorMuon pins
+# ============================================================================
+def normuon_pin_failures(norm):
+    """[MAC] "NorMuon: Normalized Muon": the update is scaled so its RMS equals
+    lr, row by row (norm over the last dimension, divided by sqrt(cols))."""
+    fails = []
+    rng = np.random.default_rng(8)
+    for shape in [(7, 13), (13, 7), (1, 9), (9, 1), (16, 16)]:
+        u = rng.standard_normal(shape) * rng.uniform(0.01, 3.0, size=(shape[0], 1))
+        out = norm(u)
+        if out.shape != u.shape:
+            fails.append(f"shape{shape}")
+            continue
+        rms = np.sqrt(np.mean(u * u, axis=1))
+        got = np.sqrt(np.mean(out * out, axis=1))
+        if not np.allclose(got, rms / (rms + oracle.NORMUON_EPS), rtol=1e-12, atol=0):
+            fails.append(f"row_rms{shape}")
+        # direction of every row unchanged
+        if not np.allclose(out * np.linalg.norm(u, axis=1, keepdims=True),
+                           u * np.linalg.norm(out, axis=1, keepdims=True), rtol=1e-10, atol=1e-14):
+            fails.append(f"row_direction{shape}")
+    # orthonormal rows (a wide orthogonal update): every row has norm 1 and RMS
+    # 1/sqrt(cols), so the scale is sqrt(cols).  (The page's comment gives the
+    # whole matrix's RMS as 1/sqrt(min(m,n)); it is sqrt(min/(m n)) =
+    # 1/sqrt(max(m,n)), checked here on the input.)
+    q = np.linalg.qr(rng.standard_normal((24, 6)))[0].T  # 6 x 24, orthonormal rows
+    want = q * (1.0 / (1.0 / np.sqrt(24) + oracle.NORMUON_EPS))
+    if np.abs(norm(q) - want).max() > 1e-12:
+        fails.append("orthonormal_rows_scale")
+    if abs(np.sqrt(np.mean(q * q)) - 1 / np.sqrt(24)) > 1e-12:
+        fails.append("orthogonal_rms")
+    # a zero row stays zero
+    z = np.zeros((3, 5))
+    z[1] = 1.0
+    out = norm(z)
+    if not (np.all(out[0] == 0) and np.all(out[2] == 0)):
+        fails.append("zero_row")
+    return fails
+
+
+def test_normuon_pins():
+    assert normuon_pin_failures(oracle.normuon_rows) == []
+
+
+def test_muon_step_with_normuon_matches_page_sequence():
+    """[MAC] "The Full Muon Step": update = normalize_muon_update(NS(m~), lr);
+    p *= (1 - lr wd); p -= update  (plain decay, as the page sequences it)."""
+    rng = np.random.default_rng(12)
+    w, g = rng.standard_normal((20, 36)), rng.standard_normal((20, 36))
+    lr, wd = 0.02, 0.1
+    got, _, _ = oracle.muon_step(w, g, np.zeros_like(w), lr, 0.95, wd, normuon=True, cautious=False)
+    u = oracle.newton_schulz(0.95 * g + g)  # one step from zero momentum
+    scale = lr / (np.linalg.norm(u, axis=-1, keepdims=True) / u.shape[-1] ** 0.5 + 1e-8)
+    seq = w * (1 - lr * wd)
+    seq = seq - u * scale
+    assert _rel(got, seq) < 1e-14
+
+
+# ============================================================================
 # AdamW pins
 # ============================================================================
 def adamw_pin_failures(adamw):
