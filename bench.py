@@ -119,7 +119,7 @@ def algorithmic_work(wl):
         gb = 2 if t.grad_dtype == "bf16" else 4
         adam_bytes += t.count * math.prod(t.shape) * (gb + 24)
     return dict(gram_flops=gram, poly_flops=poly, axpy_flops=axpy, momentum_bytes=mom_bytes,
-                update_bytes=upd_bytes, adamw_bytes=adam_bytes, rowscale_bytes=upd_bytes / 5.0)
+                update_bytes=upd_bytes, adamw_bytes=adam_bytes)
 
 
 class DeviceWorkload:
@@ -353,7 +353,7 @@ def run_gpu(args):
             "ns_axpy_update": ("tensor", work["axpy_flops"]),
             "momentum_norm": ("hbm", work["momentum_bytes"]),
             "update": ("hbm", work["update_bytes"]),
-            "row_scale": ("hbm", work["rowscale_bytes"]),
+            "normuon_update": ("hbm", work["update_bytes"]),
             "adamw": ("hbm", work["adamw_bytes"]),
         }
         # per-step algorithmic work of each kernel kind: GEMM kinds run once per
@@ -363,7 +363,7 @@ def run_gpu(args):
             "ns_axpy": work["axpy_flops"] * (K - 1 if "ns_axpy_update" in kinds else K),
             "ns_axpy_update": work["axpy_flops"],
             "momentum_norm": work["momentum_bytes"], "update": work["update_bytes"],
-            "row_scale": work["rowscale_bytes"],
+            "normuon_update": work["update_bytes"],
             "adamw": work["adamw_bytes"]}
         roof = None
         if dom in alg:
@@ -387,7 +387,7 @@ def run_gpu(args):
                         "peak_source": f"{peak_src} (HBM copy)",
                         "work_per_launch": per_launch, "work_unit": "algorithmic bytes"}
         ew = {}
-        for k in ("momentum_norm", "update", "row_scale", "adamw"):
+        for k in ("momentum_norm", "update", "normuon_update", "adamw"):
             if k in kinds:
                 ew[k] = round(per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e9, 1)
         for k in ("ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update"):

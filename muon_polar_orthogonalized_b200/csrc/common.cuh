@@ -30,7 +30,6 @@ struct MatRef {
   int vec;           // 1: 4-wide vector path is legal for this matrix
   int blk_begin;     // first block of this matrix in the launch
   int sidx;          // index of this matrix's scale in the wave's scale array
-  int rbase;         // index of this matrix's row 0 in the wave's row-scale array (NorMuon)
   float lr;          // lr * lr_scale (update kernel)
 };
 
@@ -48,7 +47,6 @@ struct EltParams {
   int use_scale;     // update/emit: multiply X by the matrix scale (ns_steps == 0)
   float* partials;   // momentum kernel: one partial sum of squares per block
   float* scales;     // per-matrix 1/(||m~||+eps)
-  float* rowscale;   // NorMuon: per-row 1/(rms(U_row)+1e-8), or nullptr
 };
 
 // ------------------------------------------------------------ GEMM problems

@@ -10,8 +10,8 @@
 //   update         W <- W - lr*(U + wd*mask*W), mask = (U*W >= 0) by sign bits
 //                  (nanochat discussion, mira687's reply: cautious weight decay)
 //   emit           out <- U as fp32 (orthogonaliser entry point)
-//   row_scale      NorMuon: s_row = 1/(||U_row||/sqrt(cols) + 1e-8), one warp
-//                  per row, fixed-order reduction ("Chapter 4", NorMuon)
+//   normuon_update NorMuon + cautious update, one warp per row: U_row is divided
+//                  by (||U_row||/sqrt(cols) + 1e-8) first ("Chapter 4", NorMuon)
 //   adamw          bias-corrected AdamW with decoupled decay
 //                  ("3.9 Optimizers", Implementing AdamW from scratch)
 //
@@ -280,7 +280,6 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
     if (!p.use_scale) return x;
     return f32x ? sc * x : round_bf16(sc * x);
   };
-  const float* rs = p.rowscale ? p.rowscale + r.rbase : nullptr;
   if (r.vec) {
     float4 xv[kEltUnroll], wv[kEltUnroll];
 #pragma unroll
@@ -296,10 +295,6 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
       const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
       if (e < numel) {
         float4 uu = make_float4(make_u(xv[u].x), make_u(xv[u].y), make_u(xv[u].z), make_u(xv[u].w));
-        if (rs) {
-          const float f = rs[static_cast<int>(e) / r.cols];  // a vec4 unit never crosses a row
-          uu.x *= f; uu.y *= f; uu.z *= f; uu.w *= f;
-        }
         if (EMIT) {
           st_stream(reinterpret_cast<float4*>(r.out + e), uu);
         } else {
@@ -316,8 +311,7 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
     for (int u = 0; u < kEltUnroll * 4; ++u) {
       const long long e = e0 + static_cast<long long>(u) * kEltThreads + threadIdx.x;
       if (e < numel) {
-        float uu = make_u(load_x1(r.x, x_index(r, e), f32x));
-        if (rs) uu *= rs[static_cast<int>(e) / r.cols];
+        const float uu = make_u(load_x1(r.x, x_index(r, e), f32x));
         if (EMIT) r.out[e] = uu;
         else r.w[e] = cautious_apply(r.w[e], uu, r.lr, p.wd, p.cautious);
       }
@@ -334,14 +328,32 @@ update_kernel(const __grid_constant__ EltParams p) {
   }
 }
 
-// -------------------------------------------------------------- row_scale
-// One warp per row: rows of all matrices of the launch are numbered
-// consecutively (MatRef.blk_begin = first row of the matrix).  U is the value
-// the update kernel will use (the bf16 X, or bf16(s*X0) when no iteration
-// ran), squared and summed in fp32 per lane in column order, then reduced with
-// a fixed shuffle tree.
+// -------------------------------------------------------- normuon_update
+// NorMuon + cautious update, one warp per parameter row (rows of all matrices
+// of the launch are numbered consecutively: MatRef.blk_begin = first row).
+// Pass 1 sums U^2 over the row (U = the bf16 X, or bf16(s*X0) when no
+// iteration ran) in fp32 per lane in column order, reduced by a fixed shuffle
+// tree; f = 1/(sqrt(sum/cols) + 1e-8).  Pass 2 re-reads the row (now in
+// cache) and applies W <- W - lr*(f*U + wd*mask*W).
+__device__ __forceinline__ void ld_x8(const void* x, long long idx, bool f32, float (&v)[8]) {
+  if (f32) {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + idx + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 raw = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + idx);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+      v[2 * h] = f.x;
+      v[2 * h + 1] = f.y;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kEltThreads)
-row_scale_kernel(const __grid_constant__ EltParams p) {
+normuon_update_kernel(const __grid_constant__ EltParams p) {
   const int lane = threadIdx.x & 31;
   const int wpb = kEltThreads / 32;
   const bool f32x = p.x_f32 != 0;
@@ -350,17 +362,54 @@ row_scale_kernel(const __grid_constant__ EltParams p) {
     const MatRef& r = p.mats[find_mat(p.mats, p.nmats, row_g)];
     const int row = row_g - r.blk_begin;
     const float sc = p.use_scale ? p.scales[r.sidx] : 1.f;
-    const long long base = static_cast<long long>(row) * r.ldx;
+    auto make_u = [&](float x) {
+      if (!p.use_scale) return x;
+      return f32x ? sc * x : round_bf16(sc * x);
+    };
+    const long long xb = static_cast<long long>(row) * r.ldx;
+    float* wrow = r.w + static_cast<long long>(row) * r.cols;
+    // r.vec: cols % 8 == 0 and W 16-byte aligned (X rows always are)
     float acc = 0.f;
-    for (int c = lane; c < r.cols; c += 32) {
-      float u = load_x1(r.x, base + c, f32x);
-      if (p.use_scale) u = f32x ? sc * u : round_bf16(sc * u);
-      acc = fmaf(u, u, acc);
+    if (r.vec) {
+      for (int c = lane * 8; c < r.cols; c += 256) {
+        float v[8];
+        ld_x8(r.x, xb + c, f32x, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float u = make_u(v[k]);
+          acc = fmaf(u, u, acc);
+        }
+      }
+    } else {
+      for (int c = lane; c < r.cols; c += 32) {
+        const float u = make_u(load_x1(r.x, xb + c, f32x));
+        acc = fmaf(u, u, acc);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0)
-      p.rowscale[r.rbase + row] = 1.f / (sqrtf(acc / static_cast<float>(r.cols)) + 1e-8f);
+    const float f = 1.f / (sqrtf(acc / static_cast<float>(r.cols)) + 1e-8f);
+    if (r.vec) {
+      for (int c = lane * 8; c < r.cols; c += 256) {
+        float v[8];
+        ld_x8(r.x, xb + c, f32x, v);
+        float4* w4 = reinterpret_cast<float4*>(wrow + c);
+        float4 w0 = w4[0], w1 = w4[1];
+        w0.x = cautious_apply(w0.x, f * make_u(v[0]), r.lr, p.wd, p.cautious);
+        w0.y = cautious_apply(w0.y, f * make_u(v[1]), r.lr, p.wd, p.cautious);
+        w0.z = cautious_apply(w0.z, f * make_u(v[2]), r.lr, p.wd, p.cautious);
+        w0.w = cautious_apply(w0.w, f * make_u(v[3]), r.lr, p.wd, p.cautious);
+        w1.x = cautious_apply(w1.x, f * make_u(v[4]), r.lr, p.wd, p.cautious);
+        w1.y = cautious_apply(w1.y, f * make_u(v[5]), r.lr, p.wd, p.cautious);
+        w1.z = cautious_apply(w1.z, f * make_u(v[6]), r.lr, p.wd, p.cautious);
+        w1.w = cautious_apply(w1.w, f * make_u(v[7]), r.lr, p.wd, p.cautious);
+        w4[0] = w0;
+        w4[1] = w1;
+      }
+    } else {
+      for (int c = lane; c < r.cols; c += 32)
+        wrow[c] = cautious_apply(wrow[c], f * make_u(load_x1(r.x, xb + c, f32x)), r.lr, p.wd, p.cautious);
+    }
   }
 }
 
@@ -472,12 +521,12 @@ cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_row_scale(const EltParams& p, int sms, cudaStream_t s) {
+cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
   const int wpb = kEltThreads / 32;
   const long long need = (static_cast<long long>(p.total_blocks) + wpb - 1) / wpb;
   const long long cap = static_cast<long long>(sms) * 8;
-  row_scale_kernel<<<static_cast<int>(need < cap ? need : cap), kEltThreads, 0, s>>>(p);
+  normuon_update_kernel<<<static_cast<int>(need < cap ? need : cap), kEltThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

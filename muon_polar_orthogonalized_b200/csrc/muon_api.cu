@@ -28,7 +28,7 @@ int elt_chunk();
 int adam_chunk();
 cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
-cudaError_t launch_row_scale(const EltParams& p, int sms, cudaStream_t s);
+cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
 int tc_tile_m(bool pair);
@@ -62,12 +62,12 @@ void muon_set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s",
 namespace {
 enum Kind {
   K_MOMENTUM = 0, K_NORM, K_GRAM, K_POLY, K_AXPY, K_AXPY_UPDATE, K_UPDATE, K_EMIT, K_ADAMW,
-  K_GRAM_F32, K_POLY_F32, K_AXPY_F32, K_AXPY_UPDATE_F32, K_ROW_SCALE, K_COUNT
+  K_GRAM_F32, K_POLY_F32, K_AXPY_F32, K_AXPY_UPDATE_F32, K_NORMUON_UPDATE, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
     "momentum_norm", "norm_finalize", "ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update",
     "update", "emit", "adamw", "ns_gram_f32", "ns_poly_f32", "ns_axpy_f32", "ns_axpy_update_f32",
-    "row_scale"};
+    "normuon_update"};
 
 struct ProfRec {
   int kind;
@@ -199,37 +199,30 @@ struct WaveItem {
   size_t x0, x1, b;     // byte offsets in the workspace
   int sbase;            // index of the item's first matrix in the wave's scale array
   long long pbase;      // first momentum block of the item's first matrix (wave-relative)
-  long long rbase;      // first row of the item's first matrix in the row-scale array
 };
 
 struct Wave {
   std::vector<WaveItem> items;
-  size_t scales_off = 0, partials_off = 0, rows_off = 0, total = 0;
+  size_t scales_off = 0, partials_off = 0, total = 0;
   int nmats = 0;
   long long nblocks = 0;
-  long long nrows = 0;  // row-scale entries (NorMuon only)
 };
 
 // Lay out a wave and return its byte size.
-size_t layout_wave(Wave& w, const std::vector<GroupGeom>& geo, bool rowscale) {
+size_t layout_wave(Wave& w, const std::vector<GroupGeom>& geo) {
   w.nmats = 0;
   w.nblocks = 0;
-  w.nrows = 0;
   for (auto& it : w.items) {
     it.sbase = w.nmats;
     it.pbase = w.nblocks;
-    it.rbase = w.nrows;
     w.nmats += it.count;
     w.nblocks += geo[it.g].nblk * it.count;
-    if (rowscale) w.nrows += static_cast<long long>(geo[it.g].r) * it.count;
   }
   size_t off = kWsHeaderBytes;
   w.scales_off = off;
   off = align_up(off + 4ull * w.nmats, 256);
   w.partials_off = off;
-  off = align_up(off + 4ull * w.nblocks, 256);
-  w.rows_off = off;
-  off = align_up(off + 4ull * w.nrows, 1024);
+  off = align_up(off + 4ull * w.nblocks, 1024);
   for (auto& it : w.items) {
     const GroupGeom& q = geo[it.g];
     it.x0 = off;
@@ -261,8 +254,8 @@ muon_status validate_groups(const muon_group* groups, int n_groups) {
 }
 
 // Greedy waves: whole groups in order, split only where the workspace runs out.
-muon_status plan_waves(const muon_group* groups, int n_groups, bool f32, bool rowscale,
-                       size_t ws_bytes, std::vector<GroupGeom>& geo, std::vector<Wave>& waves) {
+muon_status plan_waves(const muon_group* groups, int n_groups, bool f32, size_t ws_bytes,
+                       std::vector<GroupGeom>& geo, std::vector<Wave>& waves) {
   geo.clear();
   for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32));
   waves.clear();
@@ -274,31 +267,31 @@ muon_status plan_waves(const muon_group* groups, int n_groups, bool f32, bool ro
           trial.items.back().count < kMaxUpdMats)
         trial.items.back().count += 1;
       else
-        trial.items.push_back({gi, j, 1, 0, 0, 0, 0, 0, 0});
-      if (layout_wave(trial, geo, rowscale) <= ws_bytes) {
+        trial.items.push_back({gi, j, 1, 0, 0, 0, 0, 0});
+      if (layout_wave(trial, geo) <= ws_bytes) {
         cur = trial;
         continue;
       }
       if (cur.items.empty())
         return fail(MUON_ERR_WORKSPACE, "workspace of %zu bytes cannot hold one %d x %d matrix", ws_bytes,
                     groups[gi].rows, groups[gi].cols);
-      layout_wave(cur, geo, rowscale);
+      layout_wave(cur, geo);
       waves.push_back(cur);
       cur = Wave();
-      cur.items.push_back({gi, j, 1, 0, 0, 0, 0, 0, 0});
-      if (layout_wave(cur, geo, rowscale) > ws_bytes)
+      cur.items.push_back({gi, j, 1, 0, 0, 0, 0, 0});
+      if (layout_wave(cur, geo) > ws_bytes)
         return fail(MUON_ERR_WORKSPACE, "workspace of %zu bytes cannot hold one %d x %d matrix", ws_bytes,
                     groups[gi].rows, groups[gi].cols);
     }
   }
   if (!cur.items.empty()) {
-    layout_wave(cur, geo, rowscale);
+    layout_wave(cur, geo);
     waves.push_back(cur);
   }
   return MUON_OK;
 }
 
-size_t full_wave_size(const muon_group* groups, int n_groups, bool f32, bool rowscale) {
+size_t full_wave_size(const muon_group* groups, int n_groups, bool f32) {
   std::vector<GroupGeom> geo;
   for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32));
   Wave w;
@@ -306,23 +299,23 @@ size_t full_wave_size(const muon_group* groups, int n_groups, bool f32, bool row
     int left = groups[gi].count, first = 0;
     while (left > 0) {
       const int c = std::min(left, kMaxUpdMats);
-      w.items.push_back({gi, first, c, 0, 0, 0, 0, 0, 0});
+      w.items.push_back({gi, first, c, 0, 0, 0, 0, 0});
       first += c;
       left -= c;
     }
   }
-  return layout_wave(w, geo, rowscale);
+  return layout_wave(w, geo);
 }
 
-size_t min_wave_size(const muon_group* groups, int n_groups, bool f32, bool rowscale) {
+size_t min_wave_size(const muon_group* groups, int n_groups, bool f32) {
   size_t mx = kWsHeaderBytes;
   std::vector<GroupGeom> geo;
   for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32));
   for (int gi = 0; gi < n_groups; ++gi) {
     if (groups[gi].count == 0) continue;
     Wave w;
-    w.items.push_back({gi, 0, 1, 0, 0, 0, 0, 0, 0});
-    mx = std::max(mx, layout_wave(w, geo, rowscale));
+    w.items.push_back({gi, 0, 1, 0, 0, 0, 0, 0});
+    mx = std::max(mx, layout_wave(w, geo));
   }
   return mx;
 }
@@ -373,13 +366,11 @@ struct Ctx {
 };
 
 muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
-  // kind: 0 momentum_norm, 1 finalize, 2 update, 3 emit, 4 row_scale (NorMuon)
+  // kind: 0 momentum_norm, 1 finalize, 2 update, 3 emit, 4 NorMuon update (row-wise)
   const StepArgs& a = C.a;
   const bool f32 = (a.flags & MUON_FP32_DEBUG) != 0;
   float* scales = reinterpret_cast<float*>(a.ws + w.scales_off);
   float* partials = reinterpret_cast<float*>(a.ws + w.partials_off);
-  const bool normuon = (a.flags & MUON_NORMUON) != 0 && !a.orth;
-  float* rowscale = normuon ? reinterpret_cast<float*>(a.ws + w.rows_off) : nullptr;
   // matrices of the wave in order, batched <= kMaxMatsPerLaunch per launch and,
   // for the momentum kernel, one grad dtype per launch
   EltParams P;
@@ -395,7 +386,6 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
     P.x_f32 = f32 ? 1 : 0;
     P.use_scale = (a.ns_steps == 0) ? 1 : 0;
     P.scales = scales;
-    P.rowscale = (kind == 2 || kind == 4) ? rowscale : nullptr;
     cudaError_t e = cudaSuccess;
     if (kind == 0) {
       P.partials = partials + launch_blk0;
@@ -405,7 +395,8 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
       P.partials = partials;
       e = timed_launch(K_NORM, a.stream, [&] { return launch_norm_finalize(P, a.stream); });
     } else if (kind == 4) {
-      e = timed_launch(K_ROW_SCALE, a.stream, [&] { return launch_row_scale(P, C.dev.sms, a.stream); });
+      e = timed_launch(K_NORMUON_UPDATE, a.stream,
+                       [&] { return launch_normuon_update(P, C.dev.sms, a.stream); });
     } else {
       e = timed_launch(kind == 2 ? K_UPDATE : K_EMIT, a.stream,
                        [&] { return launch_update(P, kind == 3, C.dev.sms, a.stream); });
@@ -432,7 +423,6 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
       r.cols = q.c;
       r.ldx = q.ldc;
       r.sidx = it.sbase + j;
-      r.rbase = static_cast<int>(it.rbase + static_cast<long long>(q.r) * j);
       r.lr = a.lr * g.lr_scale;
       // X buffer holding this matrix's current iterate
       const int cur = (a.ns_steps % 2 == 0) ? 0 : 1;
@@ -455,6 +445,7 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
         r.blk_begin = P.total_blocks;
         P.total_blocks += static_cast<int>(q.nblk);
       } else if (kind == 4) {
+        r.vec = (q.c % 8) == 0 && aligned(r.w, 16);
         r.blk_begin = P.total_blocks;  // rows, numbered across the launch
         P.total_blocks += q.r;
       } else {
@@ -633,7 +624,7 @@ muon_status run_step(const StepArgs& a, size_t ws_bytes) {
   std::vector<GroupGeom> geo;
   std::vector<Wave> waves;
   const bool normuon = (a.flags & MUON_NORMUON) != 0 && !a.orth;
-  muon_status st = plan_waves(a.groups, a.n_groups, f32, normuon, ws_bytes, geo, waves);
+  muon_status st = plan_waves(a.groups, a.n_groups, f32, ws_bytes, geo, waves);
   if (st != MUON_OK) return st;
   DevInfo dev;
   if ((st = device_info(&dev)) != MUON_OK) return st;
@@ -655,8 +646,7 @@ muon_status run_step(const StepArgs& a, size_t ws_bytes) {
     if (a.orth) {
       if ((st = run_elementwise(C, w, 3)) != MUON_OK) return st;
     } else if (!fused) {
-      if (normuon && (st = run_elementwise(C, w, 4)) != MUON_OK) return st;
-      if ((st = run_elementwise(C, w, 2)) != MUON_OK) return st;
+      if ((st = run_elementwise(C, w, normuon ? 4 : 2)) != MUON_OK) return st;
     }
   }
   return MUON_OK;
@@ -676,8 +666,7 @@ muon_status validate_common(const muon_group* groups, int n_groups, int ns_steps
     if (!std::isfinite(coeffs[i])) return fail(MUON_ERR_INVALID_ARG, "coeffs[%d] not finite", i);
   if (!workspace) return fail(MUON_ERR_WORKSPACE, "workspace is NULL");
   if (!aligned(workspace, 256)) return fail(MUON_ERR_WORKSPACE, "workspace not 256-byte aligned");
-  const size_t need = min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0,
-                                    (flags & MUON_NORMUON) != 0);
+  const size_t need = min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
   if (workspace_bytes < need)
     return fail(MUON_ERR_WORKSPACE, "workspace of %zu bytes < minimum %zu", workspace_bytes, need);
   return MUON_OK;
@@ -700,12 +689,12 @@ extern "C" {
 
 size_t muon_workspace_size(const muon_group* groups, int n_groups, uint32_t flags) {
   if (validate_groups(groups, n_groups) != MUON_OK) return 0;
-  return full_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0, (flags & MUON_NORMUON) != 0);
+  return full_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
 }
 
 size_t muon_workspace_min_size(const muon_group* groups, int n_groups, uint32_t flags) {
   if (validate_groups(groups, n_groups) != MUON_OK) return 0;
-  return min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0, (flags & MUON_NORMUON) != 0);
+  return min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
 }
 
 muon_status muon_step(float* const* params, const void* const* grads, float* const* momentum,
