@@ -192,6 +192,18 @@ muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step,
  */
 muon_status muon_query_status(const void* workspace, muon_stream_t stream);
 
+/*
+ * Self-test of the device failure channel (no counterpart on the optimizer
+ * pages).  Launches one thread that waits, with the same bounded wait the
+ * tensor-core kernels use but a limit of `limit_ns` nanoseconds, on an
+ * mbarrier that nothing ever arrives on; when the limit runs out it records
+ * MUON_ERR_TIMEOUT in the workspace status word (word 0) and returns.  A
+ * following muon_query_status(workspace, stream) must report
+ * MUON_ERR_TIMEOUT; the CUDA context stays usable.  limit_ns in
+ * [1000, 10^9].  The status word is not cleared first.
+ */
+muon_status muon_selftest_wait_timeout(void* workspace, uint64_t limit_ns, muon_stream_t stream);
+
 const char* muon_status_string(muon_status s);
 
 /* One-line description of the last failure on the calling thread ("" if none). */

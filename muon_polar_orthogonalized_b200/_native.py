@@ -60,6 +60,7 @@ SIGNATURES = {
                                    c_int, POINTER(c_float), c_uint32, c_void_p, c_size_t, c_void_p]),
     "adamw_step": (c_int, [POINTER(AdamWGroup), c_int, c_int64, c_void_p]),
     "muon_query_status": (c_int, [c_void_p, c_void_p]),
+    "muon_selftest_wait_timeout": (c_int, [c_void_p, ctypes.c_uint64, c_void_p]),
     "muon_status_string": (c_char_p, [c_int]),
     "muon_last_error": (c_char_p, []),
     "muon_profiler_enable": (c_int, [c_int]),

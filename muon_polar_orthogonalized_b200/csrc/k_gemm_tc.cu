@@ -501,6 +501,24 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   }
 }
 
+// ----------------------------------------------------------- self-test
+// One thread waits on an mbarrier that nothing arrives on, with the bounded
+// wait above and a short limit, and records the timeout in the status word.
+__global__ void selftest_wait_kernel(unsigned int* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  sm100::mbar_init(&bar, 1);
+  sm100::fence_mbar_init();
+  if (!sm100::mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicOr(status, kDevTimeout);
+}
+
+cudaError_t launch_selftest_wait(unsigned int* status, unsigned long long limit_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- launcher
 int tc_tile_m(bool pair) { return pair ? TcCfg<true>::BM : TcCfg<false>::BM; }
 int tc_tile_n() { return TC_BN; }

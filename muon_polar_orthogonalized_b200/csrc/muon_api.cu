@@ -35,6 +35,7 @@ int tc_tile_m(bool pair);
 int tc_tile_n();
 int tc_b_box_rows(bool pair);
 cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, int num_sms, cudaStream_t s);
+cudaError_t launch_selftest_wait(unsigned int* status, unsigned long long limit_ns, cudaStream_t s);
 int simt_tile();
 cudaError_t launch_simt_gemm(const SimtGemmParams& p, int epi, int num_sms, cudaStream_t s);
 }  // namespace muon
@@ -817,6 +818,21 @@ muon_status muon_query_status(const void* workspace, muon_stream_t stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (word & kDevTimeout) return fail(MUON_ERR_TIMEOUT, "a device-side wait ran out of time");
+  return MUON_OK;
+}
+
+muon_status muon_selftest_wait_timeout(void* workspace, uint64_t limit_ns, muon_stream_t stream) {
+  g_err[0] = '\0';
+  if (!workspace) return fail(MUON_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(MUON_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (limit_ns < 1000 || limit_ns > 1000000000ull)
+    return fail(MUON_ERR_INVALID_ARG, "limit_ns %llu outside [1e3, 1e9]", static_cast<unsigned long long>(limit_ns));
+  DevInfo dev;
+  muon_status st = device_info(&dev);
+  if (st != MUON_OK) return st;
+  cudaError_t e = launch_selftest_wait(static_cast<unsigned int*>(workspace), limit_ns,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
   return MUON_OK;
 }
 

@@ -9,6 +9,8 @@ Tolerances (stated by the optimizer's spec, derived where noted):
   cautious mask                                    bit-exact, checked with the GPU's own U
 Inputs are seeded and synthetic; both sides read identical stored values.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -483,6 +485,61 @@ def test_checkpoint_resume_bitwise(dev):
         opt.step()
     for a, b in zip(ref, mats + [emb]):
         assert torch.equal(a, b)
+
+
+def test_device_timeout_reaches_status_word(dev):
+    """A bounded device wait that runs out (an mbarrier nothing arrives on, 50 ms
+    limit) is reported through the status word, and the context stays usable:
+    the next step on the same workspace runs and reports MUON_OK."""
+    groups, W, G, M, hW, hG = make_state(dev, [(128, 256)], "f32", 10)
+    ws = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+    ws.zero_()
+    L = N.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert L.muon_selftest_wait_timeout(ctypes.c_void_p(ws.data_ptr()), 50_000_000, stream) == N.MUON_OK
+    assert api.muon_query_status(ws) == N.MUON_ERR_TIMEOUT
+    assert "device-side wait" in N.last_error()
+    api.muon_step(W, G, M, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws)
+    assert api.muon_query_status(ws) == N.MUON_OK
+    rw, rm, _ = oracle.muon_step(hW[0], hG[0], np.zeros_like(hW[0]), 0.02, 0.95, 0.01)
+    check_step(hW[0], host64(W[0]), host64(M[0]), rw, rm)
+
+
+def test_cuda_graph_replay_matches_eager(dev):
+    """muon_step launches only stream-ordered work with by-value descriptors, so
+    a captured step replays bit-identically to eager calls (fresh gradients
+    copied into the captured gradient tensors before each replay)."""
+    shapes = [(256, 512), (512, 256), (100, 300)]
+    groups, We, G, Me, _, _ = make_state(dev, shapes, "bf16", 14)
+    Wg = [w.clone() for w in We]
+    Mg = [m.clone() for m in Me]
+    Gg = [g.clone() for g in G]
+    ws_e = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+    ws_g = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up outside capture (one-time set-up calls)
+        Wt = [w.clone() for w in Wg]
+        Mt = [m.clone() for m in Mg]
+        api.muon_step(Wt, Gg, Mt, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws_g)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        api.muon_step(Wg, Gg, Mg, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws_g)
+    for step in range(3):
+        fresh = [dev_tensor(wl.round_through_dtype(wl.iid_normal(tuple(g.shape), 1.0,
+                                                                  wl.seed_of("graphG", step, k)), "bf16"),
+                            "bf16", dev) for k, g in enumerate(G)]
+        for dst, src in zip(Gg, fresh):
+            dst.copy_(src)
+        graph.replay()
+        api.muon_step(We, fresh, Me, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws_e)
+        torch.cuda.synchronize()
+        for a, b in zip(We + Me, Wg + Mg):
+            assert torch.equal(a, b), step
+    assert api.muon_query_status(ws_g) == N.MUON_OK
+    del graph
 
 
 def test_status_word_ok_after_step(dev):

@@ -128,3 +128,10 @@ def test_profiler_kinds(L):
     names = [L.muon_kernel_kind_name(i).decode() for i in range(L.muon_kernel_kind_count())]
     for k in ("momentum_norm", "ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update", "adamw"):
         assert k in names
+
+
+def test_selftest_validation(L):
+    assert L.muon_selftest_wait_timeout(None, 10**6, None) == N.MUON_ERR_WORKSPACE
+    assert L.muon_selftest_wait_timeout(ctypes.c_void_p(0x1010), 10**6, None) == N.MUON_ERR_WORKSPACE
+    assert L.muon_selftest_wait_timeout(ctypes.c_void_p(0x1000), 10, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_selftest_wait_timeout(ctypes.c_void_p(0x1000), 10**10, None) == N.MUON_ERR_INVALID_ARG
