@@ -39,6 +39,31 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM traffic per launch of a kernel, from one ncu capture of the named
+# kernel sources (sha256 prefix of the files listed).  When the sources differ
+# from the captured ones the figure no longer describes the kernel and the
+# roofline reports traffic = null.  Captured on the one-layer slice of the 8B
+# shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
+# set: same seven shapes, 1 layer instead of 32); see profiles/.
+TRAFFIC_CAPTURES = {
+    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "be4e8ded0b89d069",
+                "bytes_per_launch": {"llama_8b_32l": 32 * 1536711936, "llama_8b_1layer": 1536711936},
+                "profile": "profiles/tc_gemm_pair_llama_8b_1layer.md"},
+}
+
+
+def captured_traffic(kernel: str, workload: str):
+    import hashlib
+    cap = TRAFFIC_CAPTURES.get(kernel)
+    if not cap or workload not in cap["bytes_per_launch"]:
+        return None
+    csrc = os.path.join(ROOT, "muon_polar_orthogonalized_b200", "csrc")
+    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in cap["sources"]))
+    if h.hexdigest()[:16] != cap["sha"]:
+        return None
+    return cap["bytes_per_launch"][workload]
+
+
 def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -376,14 +401,16 @@ def run_gpu(args):
                 ach = per_launch / avg_s / 1e12
                 peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
                 roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
-                        "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                        "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                        "traffic": captured_traffic(dom, wl.name), "traffic_unit": "bytes per launch",
                         "peak_source": f"{peak_src} (sustained bf16 cuBLAS)",
                         "work_per_launch": per_launch, "work_unit": "nominal FLOP"}
             else:
                 ach = per_launch / avg_s / 1e9
                 peak = peaks["hbm_gbs"]
                 roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
-                        "unit": "GB/s", "frac": round(ach / peak, 4), "traffic": None,
+                        "unit": "GB/s", "frac": round(ach / peak, 4),
+                        "traffic": captured_traffic(dom, wl.name), "traffic_unit": "bytes per launch",
                         "peak_source": f"{peak_src} (HBM copy)",
                         "work_per_launch": per_launch, "work_unit": "algorithmic bytes"}
         ew = {}
