@@ -186,6 +186,44 @@ muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step,
                        muon_stream_t stream);
 
 /*
+ * Device-resident schedule state, for steps replayed from a captured CUDA
+ * graph: the learning rate and AdamW's step count change between replays
+ * without re-recording.  Device memory, 8-byte aligned, owned by the caller;
+ * start it at {lr_mult = 1 (or any), step = 0}.
+ *   lr_mult  multiplies lr in muon_step_scheduled and every group's lr in
+ *            adamw_step_scheduled
+ *   step     AdamW's t (>= 1 when adamw_step_scheduled runs)
+ */
+typedef struct {
+  float lr_mult;
+  float reserved;
+  int64_t step;
+} muon_schedule_state;
+
+/*
+ * On the device: step <- step + 1, then lr_mult <- the trapezoidal schedule
+ * ("Chapter 4: The MuonAdamW Optimizer", Learning Rate Schedule) at the
+ * 0-based step (step - 1): linear warmup from 0 over int(total_steps *
+ * warmup_frac) steps, 1 on the flat part, linear warmdown to final_frac over
+ * int(total_steps * warmdown_frac) steps, final_frac at and after total_steps.
+ * One single-thread kernel on `stream`.
+ */
+muon_status muon_schedule_advance(muon_schedule_state* state, int64_t total_steps,
+                                  float warmup_frac, float warmdown_frac, float final_frac,
+                                  muon_stream_t stream);
+
+/* muon_step with the learning rate lr * state->lr_mult read on the device. */
+muon_status muon_step_scheduled(float* const* params, const void* const* grads,
+                                float* const* momentum, const muon_group* groups, int n_groups,
+                                float lr, float beta, float wd, int ns_steps, const float* coeffs,
+                                uint32_t flags, void* workspace, size_t workspace_bytes,
+                                const muon_schedule_state* state, muon_stream_t stream);
+
+/* adamw_step with each group's lr * state->lr_mult and t = state->step read on the device. */
+muon_status adamw_step_scheduled(const adamw_group* groups, int n_groups,
+                                 const muon_schedule_state* state, muon_stream_t stream);
+
+/*
  * Synchronises `stream`, reads the workspace status word written by the
  * device during the last muon_step / muon_orthogonalize on it, and returns
  * MUON_OK or the recorded error (MUON_ERR_TIMEOUT).

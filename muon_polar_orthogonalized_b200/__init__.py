@@ -7,9 +7,11 @@ does not load the library; the first call does, and raises if it is missing.
 from ._native import (MUON_BF16, MUON_CAUTIOUS_WD, MUON_F32, MUON_FP32_DEBUG,  # noqa: F401
                       MUON_NESTEROV, MUON_NORMUON, MUON_TC_SINGLE_CTA, MUON_UNFUSED_UPDATE,
                       MuonError, MuonGroup)
-from .api import (AdamWSpec, adamw_step, muon_orthogonalize, muon_profiler_enable,  # noqa: F401
-                  muon_profiler_read, muon_profiler_reset, muon_query_status, muon_step,
-                  muon_workspace_min_size, muon_workspace_size)
+from .api import (AdamWSpec, adamw_step, adamw_step_scheduled, muon_orthogonalize,  # noqa: F401
+                  muon_profiler_enable, muon_profiler_read, muon_profiler_reset,
+                  muon_query_status, muon_schedule_advance, muon_step, muon_step_scheduled,
+                  muon_workspace_min_size, muon_workspace_size, new_schedule_state,
+                  read_schedule_state)
 
 __all__ = [
     "muon_step", "muon_orthogonalize", "adamw_step", "muon_workspace_size",

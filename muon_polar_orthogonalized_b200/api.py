@@ -78,6 +78,45 @@ def muon_step(params, grads, momentum, groups: Sequence, lr: float, beta: float,
     check(st, "muon_step")
 
 
+def muon_step_scheduled(params, grads, momentum, groups: Sequence, lr: float, beta: float, wd: float,
+                        ns_steps: int, coeffs, flags: int, workspace, schedule_state,
+                        workspace_bytes: Optional[int] = None, stream=None) -> None:
+    """muon_step with the learning rate multiplied by the device schedule
+    state's lr_mult (schedule_state: a 16-byte device tensor, see
+    new_schedule_state)."""
+    g = make_groups(groups)
+    ca = _coeff_array(coeffs, ns_steps)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
+    st = N.lib().muon_step_scheduled(_ptrs(params), _ptrs(grads), _ptrs(momentum), g, len(groups),
+                                     float(lr), float(beta), float(wd), int(ns_steps), ca, int(flags),
+                                     c_void_p(ws), wsb, c_void_p(schedule_state.data_ptr()),
+                                     c_void_p(_stream_handle(stream)))
+    check(st, "muon_step_scheduled")
+
+
+def new_schedule_state(device, lr_mult: float = 1.0, step: int = 0):
+    """A device-resident schedule state {float lr_mult; float reserved; int64 step}."""
+    import struct
+    import torch
+    raw = struct.pack("<ffq", float(lr_mult), 0.0, int(step))
+    return torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(device)
+
+
+def read_schedule_state(state):
+    import struct
+    lr_mult, _, step = struct.unpack("<ffq", bytes(state.cpu().numpy().tobytes()))
+    return lr_mult, step
+
+
+def muon_schedule_advance(schedule_state, total_steps: int, warmup_frac: float = 0.1,
+                          warmdown_frac: float = 0.2, final_frac: float = 0.1, stream=None) -> None:
+    st = N.lib().muon_schedule_advance(c_void_p(schedule_state.data_ptr()), int(total_steps),
+                                       float(warmup_frac), float(warmdown_frac), float(final_frac),
+                                       c_void_p(_stream_handle(stream)))
+    check(st, "muon_schedule_advance")
+
+
 def muon_orthogonalize(inputs, outputs, groups: Sequence, ns_steps: int, coeffs, flags: int,
                        workspace, workspace_bytes: Optional[int] = None, stream=None) -> None:
     g = make_groups(groups)
@@ -102,7 +141,7 @@ class AdamWSpec:
         self.grad_dtype = grad_dtype
 
 
-def adamw_step(groups: Sequence[AdamWSpec], step: int, stream=None) -> None:
+def _adamw_groups(groups: Sequence[AdamWSpec]):
     n = len(groups)
     arr = (AdamWGroup * max(n, 1))()
     keep = []
@@ -116,8 +155,21 @@ def adamw_step(groups: Sequence[AdamWSpec], step: int, stream=None) -> None:
                             ctypes.cast(v, ctypes.POINTER(c_void_p)),
                             numel, len(g.params), int(g.grad_dtype), float(g.lr), float(g.beta1),
                             float(g.beta2), float(g.eps), float(g.wd))
-    st = N.lib().adamw_step(arr, n, int(step), c_void_p(_stream_handle(stream)))
+    return arr, keep
+
+
+def adamw_step(groups: Sequence[AdamWSpec], step: int, stream=None) -> None:
+    arr, keep = _adamw_groups(groups)
+    st = N.lib().adamw_step(arr, len(groups), int(step), c_void_p(_stream_handle(stream)))
     check(st, "adamw_step")
+
+
+def adamw_step_scheduled(groups: Sequence[AdamWSpec], schedule_state, stream=None) -> None:
+    """adamw_step with lr * lr_mult and t = step read from the device schedule state."""
+    arr, keep = _adamw_groups(groups)
+    st = N.lib().adamw_step_scheduled(arr, len(groups), c_void_p(schedule_state.data_ptr()),
+                                      c_void_p(_stream_handle(stream)))
+    check(st, "adamw_step_scheduled")
 
 
 def muon_query_status(workspace, stream=None) -> int:

@@ -19,6 +19,14 @@ constexpr int kMaxNsSteps = 16;
 // Status word bits recorded by device code (OR-ed into workspace word 0).
 constexpr uint32_t kDevTimeout = 1u;
 
+// Device-resident schedule state (layout of muon_schedule_state): every
+// learning rate is multiplied by lr_mult; AdamW's bias correction uses step.
+struct DevSched {
+  float lr_mult;
+  float reserved;
+  long long step;
+};
+
 // ------------------------------------------------- elementwise: per matrix
 struct MatRef {
   const void* g;     // gradient (or orthogonaliser input), rows x cols, dense
@@ -47,6 +55,7 @@ struct EltParams {
   int use_scale;     // update/emit: multiply X by the matrix scale (ns_steps == 0)
   float* partials;   // momentum kernel: one partial sum of squares per block
   float* scales;     // per-matrix 1/(||m~||+eps)
+  const DevSched* sched;  // nullptr, or the device schedule (lr multiplier)
 };
 
 // ------------------------------------------------------------ GEMM problems
@@ -86,6 +95,7 @@ struct alignas(64) TcGemmParams {
   unsigned int* status;
   float wd;
   int cautious;
+  const DevSched* sched;
 };
 
 struct SimtGemmParams {
@@ -97,6 +107,7 @@ struct SimtGemmParams {
   const float* scales;
   float wd;
   int cautious;
+  const DevSched* sched;
 };
 
 // ---------------------------------------------------------------- AdamW
@@ -114,6 +125,7 @@ struct AdamTensor {
   float step_size;   // lr / (1 - beta1^t)
   float sqrt_bc2;    // sqrt(1 - beta2^t)
   float eps;
+  float lr, wd;      // base values (device schedule: the scalars above are recomputed)
 };
 
 struct AdamParams {
@@ -122,6 +134,7 @@ struct AdamParams {
   int total_blocks;  // work chunks
   int grid;          // launched blocks (persistent)
   int grad_bf16;
+  const DevSched* sched;  // nullptr, or the device schedule (lr multiplier, step)
 };
 
 }  // namespace muon

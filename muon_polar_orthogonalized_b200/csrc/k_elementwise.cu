@@ -274,6 +274,7 @@ __device__ __forceinline__ float cautious_apply(float w, float u, float lr, floa
 template <bool EMIT>
 __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r, long long e0) {
   const long long numel = static_cast<long long>(r.rows) * r.cols;
+  const float lr = p.sched ? r.lr * p.sched->lr_mult : r.lr;
   const bool f32x = p.x_f32 != 0;
   const float sc = p.use_scale ? p.scales[r.sidx] : 1.f;
   auto make_u = [&](float x) {
@@ -299,10 +300,10 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
           st_stream(reinterpret_cast<float4*>(r.out + e), uu);
         } else {
           float4 w = wv[u];
-          w.x = cautious_apply(w.x, uu.x, r.lr, p.wd, p.cautious);
-          w.y = cautious_apply(w.y, uu.y, r.lr, p.wd, p.cautious);
-          w.z = cautious_apply(w.z, uu.z, r.lr, p.wd, p.cautious);
-          w.w = cautious_apply(w.w, uu.w, r.lr, p.wd, p.cautious);
+          w.x = cautious_apply(w.x, uu.x, lr, p.wd, p.cautious);
+          w.y = cautious_apply(w.y, uu.y, lr, p.wd, p.cautious);
+          w.z = cautious_apply(w.z, uu.z, lr, p.wd, p.cautious);
+          w.w = cautious_apply(w.w, uu.w, lr, p.wd, p.cautious);
           st_stream(reinterpret_cast<float4*>(r.w + e), w);
         }
       }
@@ -313,7 +314,7 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
       if (e < numel) {
         const float uu = make_u(load_x1(r.x, x_index(r, e), f32x));
         if (EMIT) r.out[e] = uu;
-        else r.w[e] = cautious_apply(r.w[e], uu, r.lr, p.wd, p.cautious);
+        else r.w[e] = cautious_apply(r.w[e], uu, lr, p.wd, p.cautious);
       }
     }
   }
@@ -368,6 +369,7 @@ normuon_update_kernel(const __grid_constant__ EltParams p) {
     };
     const long long xb = static_cast<long long>(row) * r.ldx;
     float* wrow = r.w + static_cast<long long>(row) * r.cols;
+    const float lr = p.sched ? r.lr * p.sched->lr_mult : r.lr;
     // r.vec: cols % 8 == 0 and W 16-byte aligned (X rows always are)
     float acc = 0.f;
     if (r.vec) {
@@ -395,20 +397,20 @@ normuon_update_kernel(const __grid_constant__ EltParams p) {
         ld_x8(r.x, xb + c, f32x, v);
         float4* w4 = reinterpret_cast<float4*>(wrow + c);
         float4 w0 = w4[0], w1 = w4[1];
-        w0.x = cautious_apply(w0.x, f * make_u(v[0]), r.lr, p.wd, p.cautious);
-        w0.y = cautious_apply(w0.y, f * make_u(v[1]), r.lr, p.wd, p.cautious);
-        w0.z = cautious_apply(w0.z, f * make_u(v[2]), r.lr, p.wd, p.cautious);
-        w0.w = cautious_apply(w0.w, f * make_u(v[3]), r.lr, p.wd, p.cautious);
-        w1.x = cautious_apply(w1.x, f * make_u(v[4]), r.lr, p.wd, p.cautious);
-        w1.y = cautious_apply(w1.y, f * make_u(v[5]), r.lr, p.wd, p.cautious);
-        w1.z = cautious_apply(w1.z, f * make_u(v[6]), r.lr, p.wd, p.cautious);
-        w1.w = cautious_apply(w1.w, f * make_u(v[7]), r.lr, p.wd, p.cautious);
+        w0.x = cautious_apply(w0.x, f * make_u(v[0]), lr, p.wd, p.cautious);
+        w0.y = cautious_apply(w0.y, f * make_u(v[1]), lr, p.wd, p.cautious);
+        w0.z = cautious_apply(w0.z, f * make_u(v[2]), lr, p.wd, p.cautious);
+        w0.w = cautious_apply(w0.w, f * make_u(v[3]), lr, p.wd, p.cautious);
+        w1.x = cautious_apply(w1.x, f * make_u(v[4]), lr, p.wd, p.cautious);
+        w1.y = cautious_apply(w1.y, f * make_u(v[5]), lr, p.wd, p.cautious);
+        w1.z = cautious_apply(w1.z, f * make_u(v[6]), lr, p.wd, p.cautious);
+        w1.w = cautious_apply(w1.w, f * make_u(v[7]), lr, p.wd, p.cautious);
         w4[0] = w0;
         w4[1] = w1;
       }
     } else {
       for (int c = lane; c < r.cols; c += 32)
-        wrow[c] = cautious_apply(wrow[c], f * make_u(load_x1(r.x, xb + c, f32x)), r.lr, p.wd, p.cautious);
+        wrow[c] = cautious_apply(wrow[c], f * make_u(load_x1(r.x, xb + c, f32x)), lr, p.wd, p.cautious);
     }
   }
 }
@@ -479,13 +481,58 @@ __device__ __forceinline__ void adamw_chunk(const AdamTensor& T, long long e0) {
   }
 }
 
+// With a device schedule the step-dependent scalars come from the device
+// state (lr multiplier, step t), in double like the host path, then fp32.
+__device__ __forceinline__ void sched_scalars(AdamTensor& T, const DevSched* s) {
+  const double t = static_cast<double>(s->step);
+  const double lr = static_cast<double>(T.lr) * static_cast<double>(s->lr_mult);
+  T.decay = static_cast<float>(1.0 - lr * static_cast<double>(T.wd));
+  T.step_size = static_cast<float>(lr / (1.0 - pow(static_cast<double>(T.b1), t)));
+  T.sqrt_bc2 = static_cast<float>(sqrt(1.0 - pow(static_cast<double>(T.b2), t)));
+}
+
 template <bool GBF16>
 __global__ void __launch_bounds__(kEltThreads, kAdamMinBlocks)
 adamw_kernel(const __grid_constant__ AdamParams P) {
   for (int blk = blockIdx.x; blk < P.total_blocks; blk += gridDim.x) {
-    const AdamTensor& T = P.t[find_tensor(P.t, P.ntensors, blk)];
-    adamw_chunk<GBF16>(T, static_cast<long long>(blk - T.blk_begin) * kAdamChunk);
+    const int ti = find_tensor(P.t, P.ntensors, blk);
+    if (P.sched) {
+      AdamTensor T = P.t[ti];
+      sched_scalars(T, P.sched);
+      adamw_chunk<GBF16>(T, static_cast<long long>(blk - T.blk_begin) * kAdamChunk);
+    } else {
+      const AdamTensor& T = P.t[ti];
+      adamw_chunk<GBF16>(T, static_cast<long long>(blk - T.blk_begin) * kAdamChunk);
+    }
   }
+}
+
+// ----------------------------------------------------------- schedule
+// step <- step + 1; lr_mult <- trapezoid(step - 1): linear warmup from 0 over
+// int(total*warmup_frac) steps, 1 on the flat part, linear warmdown to
+// final_frac over int(total*warmdown_frac) steps, final_frac from the end on
+// ("Chapter 4: The MuonAdamW Optimizer", trapezoidal schedule).
+__global__ void schedule_advance_kernel(DevSched* s, long long total, double warmup_frac,
+                                        double warmdown_frac, double final_frac) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const long long t = s->step + 1;
+  const long long step = t - 1;
+  const long long warm = static_cast<long long>(static_cast<double>(total) * warmup_frac);
+  const long long down = static_cast<long long>(static_cast<double>(total) * warmdown_frac);
+  const long long flat = total - warm - down;
+  double m;
+  if (step < warm) m = static_cast<double>(step) / static_cast<double>(warm);
+  else if (step < warm + flat) m = 1.0;
+  else if (down == 0 || step >= total) m = final_frac;
+  else m = final_frac + (1.0 - final_frac) * (1.0 - static_cast<double>(step - warm - flat) / static_cast<double>(down));
+  s->step = t;
+  s->lr_mult = static_cast<float>(m);
+}
+
+cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
+                                    cudaStream_t st) {
+  schedule_advance_kernel<<<1, 32, 0, st>>>(s, total, wu, wd, fin);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------- launchers

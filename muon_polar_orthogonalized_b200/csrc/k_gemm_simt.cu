@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const __grid_constant__ 
         if (EPI == EPI_AXPY_UPDATE) {
           const int wi = q.w_first + mat;
           float* w = p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j;
-          *w = cautious_w_f32(*w, val, q.lr, p.wd, p.cautious != 0);
+          *w = cautious_w_f32(*w, val, p.sched ? q.lr * p.sched->lr_mult : q.lr, p.wd, p.cautious != 0);
         } else {
           static_cast<float*>(q.out)[mat * q.out_bs + static_cast<long long>(i) * q.out_ld + j] = val;
         }

@@ -235,22 +235,23 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
     const int wi = q.w_first + mat;
     float* w = p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0;
     const bool cautious = p.cautious != 0;
+    const float lr = p.sched ? q.lr * p.sched->lr_mult : q.lr;
     if (full && wvec) {
       float4* w4 = reinterpret_cast<float4*>(w);
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
         float4 ww = in.w[c4];
-        ww.x = cautious_w(ww.x, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 0])), q.lr, p.wd, cautious);
-        ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), q.lr, p.wd, cautious);
-        ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), q.lr, p.wd, cautious);
-        ww.w = cautious_w(ww.w, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 3])), q.lr, p.wd, cautious);
+        ww.x = cautious_w(ww.x, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 0])), lr, p.wd, cautious);
+        ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), lr, p.wd, cautious);
+        ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), lr, p.wd, cautious);
+        ww.w = cautious_w(ww.w, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 3])), lr, p.wd, cautious);
         w4[c4] = ww;
       }
     } else {
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         if (j0 + c < q.N)
-          w[c] = cautious_w(w[c], __bfloat162float(__float2bfloat16_rn(v[c])), q.lr, p.wd, cautious);
+          w[c] = cautious_w(w[c], __bfloat162float(__float2bfloat16_rn(v[c])), lr, p.wd, cautious);
     }
   } else {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(q.out) + mat * q.out_bs;

@@ -31,6 +31,8 @@ cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
 cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
+cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
+                                    cudaStream_t st);
 int tc_tile_m(bool pair);
 int tc_tile_n();
 int tc_b_box_rows(bool pair);
@@ -358,6 +360,7 @@ struct StepArgs {
   char* ws;
   cudaStream_t stream;
   bool orth;  // orthogonaliser mode
+  const DevSched* sched;  // device schedule (lr multiplier), or nullptr
 };
 
 struct Ctx {
@@ -387,6 +390,7 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
     P.x_f32 = f32 ? 1 : 0;
     P.use_scale = (a.ns_steps == 0) ? 1 : 0;
     P.scales = scales;
+    P.sched = a.sched;
     cudaError_t e = cudaSuccess;
     if (kind == 0) {
       P.partials = partials + launch_blk0;
@@ -487,6 +491,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       SP.scales = scales;
       SP.wd = a.wd;
       SP.cautious = (a.flags & MUON_CAUTIOUS_WD) ? 1 : 0;
+      SP.sched = a.sched;
       const int kind = epi == EPI_GRAM ? K_GRAM_F32 : epi == EPI_POLY ? K_POLY_F32
                      : epi == EPI_AXPY ? K_AXPY_F32 : K_AXPY_UPDATE_F32;
       e = timed_launch(kind, a.stream, [&] { return launch_simt_gemm(SP, epi, C.dev.sms, a.stream); });
@@ -497,6 +502,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       TP.status = reinterpret_cast<unsigned int*>(a.ws);
       TP.wd = a.wd;
       TP.cautious = (a.flags & MUON_CAUTIOUS_WD) ? 1 : 0;
+      TP.sched = a.sched;
       const int kind = epi == EPI_GRAM ? K_GRAM : epi == EPI_POLY ? K_POLY
                      : epi == EPI_AXPY ? K_AXPY : K_AXPY_UPDATE;
       e = timed_launch(kind, a.stream, [&] { return launch_tc_gemm(TP, epi, pair, C.dev.sms, a.stream); });
@@ -698,10 +704,11 @@ size_t muon_workspace_min_size(const muon_group* groups, int n_groups, uint32_t 
   return min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
 }
 
-muon_status muon_step(float* const* params, const void* const* grads, float* const* momentum,
-                      const muon_group* groups, int n_groups, float lr, float beta, float wd,
-                      int ns_steps, const float* coeffs, uint32_t flags, void* workspace,
-                      size_t workspace_bytes, muon_stream_t stream) {
+static muon_status muon_step_impl(float* const* params, const void* const* grads,
+                                  float* const* momentum, const muon_group* groups, int n_groups,
+                                  float lr, float beta, float wd, int ns_steps, const float* coeffs,
+                                  uint32_t flags, void* workspace, size_t workspace_bytes,
+                                  muon_stream_t stream, const DevSched* sched) {
   g_err[0] = '\0';
   muon_status st = validate_common(groups, n_groups, ns_steps, coeffs, flags, workspace, workspace_bytes);
   if (st != MUON_OK) return st;
@@ -711,8 +718,30 @@ muon_status muon_step(float* const* params, const void* const* grads, float* con
   if ((st = validate_ptrs("grads", grads, groups, n_groups)) != MUON_OK) return st;
   if ((st = validate_ptrs("momentum", reinterpret_cast<const void* const*>(momentum), groups, n_groups)) != MUON_OK) return st;
   StepArgs a{params, grads, momentum, nullptr, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
-             flags, static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream), false};
+             flags, static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream), false, sched};
   return run_step(a, workspace_bytes);
+}
+
+muon_status muon_step(float* const* params, const void* const* grads, float* const* momentum,
+                      const muon_group* groups, int n_groups, float lr, float beta, float wd,
+                      int ns_steps, const float* coeffs, uint32_t flags, void* workspace,
+                      size_t workspace_bytes, muon_stream_t stream) {
+  return muon_step_impl(params, grads, momentum, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
+                        flags, workspace, workspace_bytes, stream, nullptr);
+}
+
+muon_status muon_step_scheduled(float* const* params, const void* const* grads,
+                                float* const* momentum, const muon_group* groups, int n_groups,
+                                float lr, float beta, float wd, int ns_steps, const float* coeffs,
+                                uint32_t flags, void* workspace, size_t workspace_bytes,
+                                const muon_schedule_state* state, muon_stream_t stream) {
+  if (!state || !aligned(state, 8)) {
+    g_err[0] = '\0';
+    return fail(MUON_ERR_INVALID_ARG, "schedule state is NULL or not 8-byte aligned");
+  }
+  return muon_step_impl(params, grads, momentum, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
+                        flags, workspace, workspace_bytes, stream,
+                        reinterpret_cast<const DevSched*>(state));
 }
 
 muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs, const muon_group* groups,
@@ -725,11 +754,12 @@ muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs,
   if ((st = validate_ptrs("inputs", inputs, groups, n_groups)) != MUON_OK) return st;
   if ((st = validate_ptrs("outputs", reinterpret_cast<const void* const*>(outputs), groups, n_groups)) != MUON_OK) return st;
   StepArgs a{nullptr, inputs, nullptr, outputs, groups, n_groups, 0.f, 0.f, 0.f, ns_steps, coeffs,
-             flags, static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream), true};
+             flags, static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream), true, nullptr};
   return run_step(a, workspace_bytes);
 }
 
-muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step, muon_stream_t stream) {
+static muon_status adamw_impl(const adamw_group* groups, int n_groups, int64_t step,
+                              muon_stream_t stream, const DevSched* sched) {
   g_err[0] = '\0';
   if (n_groups < 0) return fail(MUON_ERR_INVALID_ARG, "n_groups < 0");
   if (n_groups > 0 && !groups) return fail(MUON_ERR_INVALID_ARG, "groups is NULL");
@@ -764,12 +794,14 @@ muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step, mu
   for (int dt = 0; dt < 2; ++dt) {
     std::memset(&P, 0, sizeof(P));
     P.grad_bf16 = dt;
+    P.sched = sched;
     auto flush = [&]() -> muon_status {
       if (P.ntensors == 0) return MUON_OK;
       cudaError_t e = timed_launch(K_ADAMW, s, [&] { return launch_adamw(P, dev.sms, s); });
       if (e != cudaSuccess) return cuda_fail(e, "adamw launch");
       P.ntensors = 0;
       P.total_blocks = 0;
+      P.sched = sched;
       return MUON_OK;
     };
     for (int gi = 0; gi < n_groups; ++gi) {
@@ -801,11 +833,45 @@ muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step, mu
         T.step_size = static_cast<float>(g.lr / bc1);
         T.sqrt_bc2 = static_cast<float>(std::sqrt(bc2));
         T.eps = g.eps;
+        T.lr = g.lr;
+        T.wd = g.wd;
         P.total_blocks += static_cast<int>(nblk);
       }
     }
     if ((st = flush()) != MUON_OK) return st;
   }
+  return MUON_OK;
+}
+
+muon_status adamw_step(const adamw_group* groups, int n_groups, int64_t step, muon_stream_t stream) {
+  return adamw_impl(groups, n_groups, step, stream, nullptr);
+}
+
+muon_status adamw_step_scheduled(const adamw_group* groups, int n_groups,
+                                 const muon_schedule_state* state, muon_stream_t stream) {
+  if (!state || !aligned(state, 8)) {
+    g_err[0] = '\0';
+    return fail(MUON_ERR_INVALID_ARG, "schedule state is NULL or not 8-byte aligned");
+  }
+  // the host step only feeds scalars the kernel recomputes from the device state
+  return adamw_impl(groups, n_groups, 1, stream, reinterpret_cast<const DevSched*>(state));
+}
+
+muon_status muon_schedule_advance(muon_schedule_state* state, int64_t total_steps,
+                                  float warmup_frac, float warmdown_frac, float final_frac,
+                                  muon_stream_t stream) {
+  g_err[0] = '\0';
+  if (!state || !aligned(state, 8)) return fail(MUON_ERR_INVALID_ARG, "schedule state is NULL or not 8-byte aligned");
+  if (total_steps < 1) return fail(MUON_ERR_INVALID_ARG, "total_steps < 1");
+  if (!(warmup_frac >= 0.f && warmdown_frac >= 0.f && warmup_frac + warmdown_frac <= 1.f))
+    return fail(MUON_ERR_INVALID_ARG, "warmup/warmdown fractions must be >= 0 and sum to <= 1");
+  if (!std::isfinite(final_frac)) return fail(MUON_ERR_INVALID_ARG, "final_frac not finite");
+  DevInfo dev;
+  muon_status st = device_info(&dev);
+  if (st != MUON_OK) return st;
+  cudaError_t e = launch_schedule_advance(reinterpret_cast<DevSched*>(state), total_steps, warmup_frac,
+                                          warmdown_frac, final_frac, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
   return MUON_OK;
 }
 

@@ -28,6 +28,7 @@ from .muon_ref import (  # noqa: F401
     normuon_rows,
     NORMUON_EPS,
     adamw_step,
+    trapezoid_lr,
     round_bf16,
     newton_schulz_bf16_emulated,
 )

@@ -192,6 +192,30 @@ def muon_step(w: np.ndarray, g: np.ndarray, m: np.ndarray, lr: float, beta: floa
 
 
 # ----------------------------------------------------------------------------
+# learning-rate schedule (device-resident schedule state)
+# ----------------------------------------------------------------------------
+def trapezoid_lr(step: int, total_steps: int, max_lr: float, min_lr: float,
+                 warmup_frac: float = 0.1, warmdown_frac: float = 0.2) -> float:
+    """[MAC] "Learning Rate Schedule: Trapezoidal (Warmup-Flat-Warmdown)":
+    linear warmup from 0 over int(total*warmup_frac) steps, max_lr for the
+    flat middle, linear warmdown to min_lr over int(total*warmdown_frac)
+    steps.  step counts from 0.  Reading for what the page leaves open: with
+    no warmdown steps, or at and beyond total_steps, the value is min_lr.
+    """
+    warmup = int(total_steps * warmup_frac)
+    warmdown = int(total_steps * warmdown_frac)
+    flat = total_steps - warmup - warmdown
+    if step < warmup:
+        return max_lr * step / warmup
+    if step < warmup + flat:
+        return max_lr
+    if warmdown == 0 or step >= total_steps:
+        return min_lr
+    decay = step - warmup - flat
+    return min_lr + (max_lr - min_lr) * (1.0 - decay / warmdown)
+
+
+# ----------------------------------------------------------------------------
 # AdamW
 # ----------------------------------------------------------------------------
 def adamw_step(p: np.ndarray, g: np.ndarray, m: np.ndarray, v: np.ndarray, t: int,

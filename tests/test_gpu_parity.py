@@ -542,6 +542,75 @@ def test_cuda_graph_replay_matches_eager(dev):
     del graph
 
 
+def test_device_schedule_matches_trapezoid(dev):
+    """The device schedule state advances like the page's trapezoidal get_lr
+    (as a multiplier: max 1, final 0.1), step counting from 1."""
+    state = api.new_schedule_state(dev, 1.0, 0)
+    total = 25
+    for t in range(1, 31):
+        api.muon_schedule_advance(state, total, 0.1, 0.2, 0.1)
+        mult, step = api.read_schedule_state(state)
+        assert step == t
+        want = oracle.trapezoid_lr(t - 1, total, 1.0, 0.1, 0.1, 0.2)
+        assert abs(mult - want) <= 1e-7 * max(1.0, abs(want)), (t, mult, want)
+
+
+def test_scheduled_graph_replay_matches_eager(dev):
+    """A graph captured once (advance the schedule, Muon step, AdamW step)
+    replays step after step with the learning rate and AdamW's t read on the
+    device; eager calls with the host-computed lr and t agree."""
+    shapes = [(256, 512), (512, 256)]
+    groups, We, G, Me, _, _ = make_state(dev, shapes, "f32", 15)
+    Wg, Mg = [w.clone() for w in We], [m.clone() for m in Me]
+    P = [torch.randn(1000, 64, device=dev) * 0.02, torch.randn(64, device=dev)]
+    AG = [torch.randn_like(p) for p in P]
+    Pe, Pg = [p.clone() for p in P], [p.clone() for p in P]
+    me, ve = [torch.zeros_like(p) for p in P], [torch.zeros_like(p) for p in P]
+    mg, vg = [torch.zeros_like(p) for p in P], [torch.zeros_like(p) for p in P]
+    ws_e = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+    ws_g = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+    state = api.new_schedule_state(dev, 1.0, 0)
+    total, lr, alr = 8, 0.02, 3e-3
+    spec_g = [api.AdamWSpec(Pg, AG, mg, vg, alr, 0.9, 0.95, 1e-8, 0.01)]
+
+    def captured_step():
+        api.muon_schedule_advance(state, total, 0.25, 0.25, 0.1)
+        api.muon_step_scheduled(Wg, G, Mg, groups, lr, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws_g, state)
+        api.adamw_step_scheduled(spec_g, state)
+
+    # warm-up on throw-away copies (one-time set-up calls happen outside capture)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        tmp_state = api.new_schedule_state(dev, 1.0, 0)
+        Wt, Mt = [w.clone() for w in Wg], [m.clone() for m in Mg]
+        api.muon_step_scheduled(Wt, G, Mt, groups, lr, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws_g, tmp_state)
+        api.adamw_step_scheduled([api.AdamWSpec([p.clone() for p in Pg], AG, [x.clone() for x in mg],
+                                                [x.clone() for x in vg], alr, 0.9, 0.95, 1e-8, 0.01)],
+                                 api.new_schedule_state(dev, 1.0, 1))
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        captured_step()
+    for t in range(1, 6):
+        graph.replay()
+        mult = float(np.float32(oracle.trapezoid_lr(t - 1, total, 1.0, 0.1, 0.25, 0.25)))
+        api.muon_step(We, G, Me, groups, float(np.float32(lr) * np.float32(mult)), 0.95, 0.01, 5, FIXED,
+                      STEP_FLAGS, ws_e)
+        api.adamw_step([api.AdamWSpec(Pe, AG, me, ve, float(np.float32(alr) * np.float32(mult)),
+                                      0.9, 0.95, 1e-8, 0.01)], t)
+        torch.cuda.synchronize()
+        for a, b in zip(Me, Mg):
+            assert torch.equal(a, b)
+        for w0, a, b in zip(We, We, Wg):
+            assert rel(host64(b), host64(a)) <= 1e-6, t
+        for a, b in zip(Pe + me + ve, Pg + mg + vg):
+            assert rel(host64(b), host64(a)) <= 1e-6, t
+    assert api.read_schedule_state(state)[1] == 5
+    del graph
+
+
 def test_status_word_ok_after_step(dev):
     groups, W, G, M, _, _ = make_state(dev, [(128, 256)], "f32", 9)
     ws = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)

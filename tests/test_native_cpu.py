@@ -135,3 +135,15 @@ def test_selftest_validation(L):
     assert L.muon_selftest_wait_timeout(ctypes.c_void_p(0x1010), 10**6, None) == N.MUON_ERR_WORKSPACE
     assert L.muon_selftest_wait_timeout(ctypes.c_void_p(0x1000), 10, None) == N.MUON_ERR_INVALID_ARG
     assert L.muon_selftest_wait_timeout(ctypes.c_void_p(0x1000), 10**10, None) == N.MUON_ERR_INVALID_ARG
+
+
+def test_schedule_validation(L):
+    assert L.muon_schedule_advance(None, 10, 0.1, 0.2, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    st = ctypes.c_void_p(0x1000)
+    assert L.muon_schedule_advance(st, 0, 0.1, 0.2, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance(st, 10, 0.7, 0.5, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance(ctypes.c_void_p(0x1004), 10, 0.1, 0.2, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    p = (ctypes.c_void_p * 1)(0x10000)
+    n = (ctypes.c_int64 * 1)(16)
+    g = N.AdamWGroup(p, p, p, p, n, 1, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0)
+    assert L.adamw_step_scheduled(ctypes.byref(g), 1, None, None) == N.MUON_ERR_INVALID_ARG

@@ -11,7 +11,8 @@ import pytest
 
 import oracle
 from tests.test_oracle_pins import (adamw_pin_failures, momentum_pin_failures,
-                                    normuon_pin_failures, ns_pin_failures, update_pin_failures)
+                                    normuon_pin_failures, ns_pin_failures, schedule_pin_failures,
+                                    update_pin_failures)
 
 
 def _coeffs(coeffs, steps):
@@ -185,3 +186,29 @@ def test_normuon_mutant_caught(kind):
 
 def test_normuon_unmutated_copy_passes():
     assert normuon_pin_failures(_normuon_variant("none")) == []
+
+
+def _sched_variant(kind):
+    def sched(step, total, max_lr, min_lr, wu=0.1, wd=0.2):
+        warm, down = int(total * wu), int(total * wd)
+        flat = total - warm - down
+        if kind == "no_warmup_ramp" and step < warm:
+            return max_lr
+        if step < warm:
+            return max_lr * step / warm
+        if step < warm + flat:
+            return max_lr
+        if step >= total:
+            return min_lr
+        dec = step - warm - flat
+        if kind == "decay_to_zero":
+            return max_lr * (1 - dec / down)
+        if kind == "wrong_fraction":
+            return min_lr + (max_lr - min_lr) * (1 - dec / total)
+        return min_lr + (max_lr - min_lr) * (1 - dec / down)
+    return sched
+
+
+@pytest.mark.parametrize("kind", ["no_warmup_ramp", "decay_to_zero", "wrong_fraction"])
+def test_schedule_mutant_caught(kind, pages):
+    assert schedule_pin_failures(_sched_variant(kind), pages["trapezoid_chart"]) != []

@@ -398,6 +398,35 @@ def test_muon_step_with_normuon_matches_page_sequence():
 
 
 # ============================================================================
+# schedule pins
+# ============================================================================
+def schedule_pin_failures(sched, pages_chart):
+    fails = []
+    c = pages_chart
+    total = 1000
+    for frac, want in zip(c["x_frac"], c["lr"]):
+        got = sched(int(round(frac * total)), total, c["max_lr"], c["min_lr"], c["warmup_frac"],
+                    c["warmdown_frac"])
+        if abs(got - want) > 1e-12:
+            fails.append(f"chart@{frac}")
+    # linear warmup from 0, flat, linear warmdown (piecewise-linear, continuous)
+    vals = [sched(t, total, 1.0, 0.1, 0.1, 0.2) for t in range(total)]
+    if vals[0] != 0.0 or abs(vals[50] - 0.5) > 1e-12:
+        fails.append("warmup_linear")
+    if any(v != 1.0 for v in vals[100:800]):
+        fails.append("flat")
+    if abs(vals[900] - (0.1 + 0.9 * 0.5)) > 1e-12:
+        fails.append("warmdown_linear")
+    if max(abs(a - b) for a, b in zip(vals, vals[1:])) > 0.0101:
+        fails.append("continuity")
+    return fails
+
+
+def test_schedule_pins(pages):
+    assert schedule_pin_failures(oracle.trapezoid_lr, pages["trapezoid_chart"]) == []
+
+
+# ============================================================================
 # AdamW pins
 # ============================================================================
 def adamw_pin_failures(adamw):
