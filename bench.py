@@ -207,11 +207,29 @@ class DeviceWorkload:
             for h, g in zip(self.host_grads, self.flat_grads):
                 h.copy_(g)
 
-    def adam_specs(self):
+    def adam_specs(self, adam_grads=None):
         from muon_polar_orthogonalized_b200 import api
         from muon_polar_orthogonalized_b200 import workloads as W
-        return [api.AdamWSpec(ps, gs, ms, vs, W.ADAMW_LR, W.ADAMW_BETAS[0], W.ADAMW_BETAS[1],
-                              W.ADAMW_EPS, t.wd) for (ps, gs, ms, vs, t) in self.adam]
+        specs = []
+        for ti, (ps, gs, ms, vs, t) in enumerate(self.adam):
+            g = adam_grads[ti] if adam_grads is not None else gs
+            specs.append(api.AdamWSpec(ps, g, ms, vs, W.ADAMW_LR, W.ADAMW_BETAS[0], W.ADAMW_BETAS[1],
+                                       W.ADAMW_EPS, t.wd))
+        return specs
+
+    def grad_views(self, flats):
+        """(muon grads, adam grads per AdamW group) as views of `flats`, a list of
+        flat buffers laid out like self.flat_grads."""
+        muon, k = [], 0
+        for s in self.wl.muon:
+            numel = s.rows * s.cols
+            muon.extend(flats[k][j * numel:(j + 1) * numel].view(s.rows, s.cols) for j in range(s.count))
+            k += 1
+        adam = []
+        for (ps, gs, ms, vs, t) in self.adam:
+            adam.append([flats[k + j].view(p.shape) for j, p in enumerate(ps)])
+            k += len(ps)
+        return muon, adam
 
 
 class RankContext:
@@ -296,12 +314,13 @@ def run_gpu(args):
     stream = torch.cuda.current_stream()
     step_no = [0]
 
-    def step():
+    def step(grads=None, adam_specs=None):
         step_no[0] += 1
-        api.muon_step(D.params, D.grads, D.mom, D.groups, W.MUON_LR, W.MUON_BETA, W.MUON_WD,
-                      wl.ns_steps, coeffs, flags, ws, stream=stream)
-        if specs:
-            api.adamw_step(specs, step_no[0], stream=stream)
+        api.muon_step(D.params, D.grads if grads is None else grads, D.mom, D.groups, W.MUON_LR,
+                      W.MUON_BETA, W.MUON_WD, wl.ns_steps, coeffs, flags, ws, stream=stream)
+        sp = specs if adam_specs is None else adam_specs
+        if sp:
+            api.adamw_step(sp, step_no[0], stream=stream)
 
     def barrier():
         torch.cuda.synchronize()
@@ -336,17 +355,43 @@ def run_gpu(args):
     ms_step = ms_total / args.steps
 
     # ------------------------------------------------------- end to end
+    # --------------------------------------------------------- end to end
+    # Every step's gradients come from host memory.  They are copied on a copy
+    # stream into one of two device gradient buffers while the previous step
+    # computes (the next batch's gradients prefetched, as a training loop
+    # would); every copy is inside the timed region, which starts before the
+    # first copy and ends after the last step's status word is read back.
     e2e = None
     if D.host_grads is not None:
         h2d = sum(h.numel() * h.element_size() for h in D.host_grads)
         status_host = torch.empty(1, dtype=torch.int32, pin_memory=True)
+        flats = [D.flat_grads, [torch.empty_like(g) for g in D.flat_grads]]
+        views = [D.grad_views(f) for f in flats]
+        vspecs = [D.adam_specs(v[1]) for v in views]
+        copy_stream = torch.cuda.Stream(device=dev)
+        ev_copy = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_step = [torch.cuda.Event(), torch.cuda.Event()]
+
+        def copy_grads(b):
+            with torch.cuda.stream(copy_stream):
+                for g, h in zip(flats[b], D.host_grads):
+                    g.copy_(h, non_blocking=True)
+            ev_copy[b].record(copy_stream)
+
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(args.steps):
-            for g, h in zip(D.flat_grads, D.host_grads):
-                g.copy_(h, non_blocking=True)
-            step()
+        copy_stream.wait_event(a0)
+        copy_grads(0)
+        for t in range(args.steps):
+            b = t % 2
+            if t + 1 < args.steps:
+                if t >= 1:
+                    copy_stream.wait_event(ev_step[1 - b])  # buffer last used by step t-1
+                copy_grads(1 - b)
+            stream.wait_event(ev_copy[b])
+            step(views[b][0], vspecs[b])
+            ev_step[b].record(stream)
             status_host.copy_(ws[:4].view(torch.int32), non_blocking=True)
         a1.record(stream)
         barrier()
@@ -354,7 +399,9 @@ def run_gpu(args):
         e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": 4,
                "path": ("pinned" if D.host_pinned else "pageable") +
-                       " host grads -> cudaMemcpyAsync -> muon_step + adamw_step -> status word read"}
+                       " host grads -> cudaMemcpyAsync on a copy stream, double-buffered (next step's"
+                       " grads copied while this step computes) -> muon_step + adamw_step -> status"
+                       " word read back"}
 
     if rank == 0:
         work = algorithmic_work(wl)
