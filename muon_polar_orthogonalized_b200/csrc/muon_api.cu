@@ -162,8 +162,9 @@ muon_status device_info(DevInfo* out) {
     g_dev[dev] = d;
   }
   *out = g_dev[dev];
-  if (out->major != 10)
-    return fail(MUON_ERR_UNSUPPORTED, "compute capability %d.%d: this library is built for sm_100a",
+  if (out->major != 10 || out->minor != 0)
+    return fail(MUON_ERR_UNSUPPORTED,
+                "compute capability %d.%d: this library is built for sm_100a (compute capability 10.0)",
                 out->major, out->minor);
   return MUON_OK;
 }

@@ -83,6 +83,8 @@ class MuonAdamW:
         specs = []
         for g in self.adamw_groups:
             grads = [p.grad for p in g["params"]]
+            if any(x is None for x in grads):
+                raise ValueError("every AdamW parameter needs a .grad")
             specs.append(api.AdamWSpec(g["params"], grads, g["exp_avg"], g["exp_avg_sq"], g["lr"],
                                        g["betas"][0], g["betas"][1], g["eps"], g["weight_decay"]))
         if specs:
