@@ -1,0 +1,132 @@
+"""Owner-sharded Muon across data-parallel ranks.
+
+Newton-Schulz needs each whole matrix on one device, while data parallelism
+keeps a full gradient on every rank ("3.9 Optimizers: SGD, Adam, Adafactor,
+Lion, Muon & Shampoo", Wiring the hybrid recipe: a distributed Muon gathers
+each matrix's gradient before it can iterate; ZeRO-1 shards optimizer state
+across data-parallel ranks).  Here every hidden matrix has one owner rank:
+
+  1. each owner's matrices' gradients are summed onto the owner (one
+     reduce per owner over a flat bucket) and divided by the world size,
+     i.e. the data-parallel mean gradient;
+  2. the owner runs the Muon step on the matrices it owns, so momentum exists
+     only on the owner (state sharded);
+  3. each owner broadcasts its updated matrices to every rank.
+
+AdamW parameters have their gradients all-reduced (mean) and are stepped on
+every rank.  Owners are chosen by longest-processing-time over the executed
+Newton-Schulz FLOPs of each matrix (3 m^2 n + m^3 for m <= n), so ranks get
+similar work.
+
+The per-rank compute is the CUDA library (MuonAdamW); `step_fn` can replace
+it, which the CPU tests use to drive the same protocol on gloo ranks.
+"""
+from __future__ import annotations
+
+import heapq
+from typing import Callable, Dict, List, Optional, Sequence
+
+import torch
+import torch.distributed as dist
+
+
+def ns_cost(rows: int, cols: int) -> float:
+    m, n = min(rows, cols), max(rows, cols)
+    return 3.0 * m * m * n + float(m) ** 3
+
+
+def assign_owners(shapes: Sequence[Sequence[int]], world: int) -> List[int]:
+    """Owner rank of each matrix: largest cost first onto the least-loaded rank
+    (ties to the lower rank), deterministic on every rank."""
+    order = sorted(range(len(shapes)), key=lambda i: (-ns_cost(*shapes[i]), i))
+    heap = [(0.0, r) for r in range(world)]
+    owners = [0] * len(shapes)
+    for i in order:
+        load, r = heapq.heappop(heap)
+        owners[i] = r
+        heapq.heappush(heap, (load + ns_cost(*shapes[i]), r))
+    return owners
+
+
+class DistributedMuonAdamW:
+    """Data-parallel MuonAdamW with owner-sharded Muon matrices.
+
+    muon_params / adamw_groups as for MuonAdamW (identical on every rank).
+    step_fn(params, grads, momentum) -> None updates the owned params and
+    momentum in place (default: a MuonAdamW over the owned matrices, built
+    with the keyword arguments given here).  The process group must be
+    initialised unless world size is 1.
+    """
+
+    def __init__(self, muon_params: Sequence[torch.Tensor], adamw_groups: Sequence[Dict] = (),
+                 process_group=None, step_fn: Optional[Callable] = None,
+                 adamw_fn: Optional[Callable] = None, **muon_kwargs):
+        self.group = process_group
+        self.world = dist.get_world_size(process_group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(process_group) if dist.is_initialized() else 0
+        self.muon_params = list(muon_params)
+        self.owners = assign_owners([tuple(p.shape) for p in self.muon_params], self.world)
+        self.owned = [i for i, o in enumerate(self.owners) if o == self.rank]
+        self.adamw_groups = list(adamw_groups)
+        self.step_fn = step_fn
+        self.adamw_fn = adamw_fn
+        self._local = None
+        if step_fn is None:
+            from .optimizer import MuonAdamW
+            self._local = MuonAdamW([self.muon_params[i] for i in self.owned], self.adamw_groups,
+                                    **muon_kwargs)
+        self.momentum = {i: torch.zeros_like(self.muon_params[i]) for i in self.owned} \
+            if step_fn is not None else None
+
+    def _bucket(self, tensors: List[torch.Tensor]) -> torch.Tensor:
+        return torch.cat([t.reshape(-1) for t in tensors]) if tensors else torch.empty(0)
+
+    def _unbucket(self, flat: torch.Tensor, tensors: List[torch.Tensor]) -> None:
+        off = 0
+        for t in tensors:
+            n = t.numel()
+            t.copy_(flat[off:off + n].view_as(t))
+            off += n
+
+    @torch.no_grad()
+    def step(self) -> None:
+        # 1. mean gradient of each matrix onto its owner
+        for r in range(self.world):
+            idx = [i for i, o in enumerate(self.owners) if o == r]
+            if not idx:
+                continue
+            grads = [self.muon_params[i].grad for i in idx]
+            if self.world > 1:
+                flat = self._bucket(grads)
+                dist.reduce(flat, dst=r, op=dist.ReduceOp.SUM, group=self.group)
+                if r == self.rank:
+                    flat.div_(self.world)
+                    self._unbucket(flat, grads)
+        # AdamW gradients: all-reduce mean
+        adam_params = [p for g in self.adamw_groups for p in g["params"]]
+        if adam_params and self.world > 1:
+            flat = self._bucket([p.grad for p in adam_params])
+            dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=self.group)
+            flat.div_(self.world)
+            self._unbucket(flat, [p.grad for p in adam_params])
+        # 2. owners step their matrices (and every rank its AdamW params)
+        if self.step_fn is not None:
+            own = self.owned
+            if own:
+                self.step_fn([self.muon_params[i] for i in own], [self.muon_params[i].grad for i in own],
+                             [self.momentum[i] for i in own])
+            if self.adamw_fn is not None and adam_params:
+                self.adamw_fn(self.adamw_groups)
+        else:
+            self._local.step()
+        # 3. owners broadcast their updated matrices
+        if self.world > 1:
+            for r in range(self.world):
+                idx = [i for i, o in enumerate(self.owners) if o == r]
+                if not idx:
+                    continue
+                ps = [self.muon_params[i] for i in idx]
+                flat = self._bucket(ps)
+                dist.broadcast(flat, src=r, group=self.group)
+                if r != self.rank:
+                    self._unbucket(flat, ps)

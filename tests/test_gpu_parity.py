@@ -611,6 +611,28 @@ def test_scheduled_graph_replay_matches_eager(dev):
     del graph
 
 
+def test_distributed_single_rank_equals_muonadamw(dev):
+    """With one rank the owner-sharded optimizer is exactly MuonAdamW."""
+    from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
+    torch.manual_seed(3)
+    mats = [torch.randn(256, 384, device=dev) * 0.02, torch.randn(384, 256, device=dev) * 0.02]
+    emb = torch.randn(500, 64, device=dev) * 0.02
+    mats2, emb2 = [m.clone() for m in mats], emb.clone()
+    a = MuonAdamW(mats, [dict(params=[emb])])
+    b = DistributedMuonAdamW(mats2, [dict(params=[emb2])])
+    assert b.owned == [0, 1]
+    for step in range(3):
+        g = torch.Generator(device=dev)
+        g.manual_seed(step)
+        for x, y in zip(mats + [emb], mats2 + [emb2]):
+            x.grad = torch.randn(x.shape, generator=g, device=dev)
+            y.grad = x.grad.clone()
+        a.step()
+        b.step()
+    for x, y in zip(mats + [emb], mats2 + [emb2]):
+        assert torch.equal(x, y)
+
+
 def test_status_word_ok_after_step(dev):
     groups, W, G, M, _, _ = make_state(dev, [(128, 256)], "f32", 9)
     ws = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
