@@ -27,8 +27,11 @@ from .muon_ref import (  # noqa: F401
     muon_step,
     normuon_rows,
     NORMUON_EPS,
+    row_equilibrate,
+    ROWEQ_EPS,
     adamw_step,
     trapezoid_lr,
+    warmup_cosine_lr,
     round_bf16,
     newton_schulz_bf16_emulated,
 )

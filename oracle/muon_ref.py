@@ -172,18 +172,50 @@ def normuon_rows(update: np.ndarray, eps: float = NORMUON_EPS) -> np.ndarray:
     return u / (rms + eps)
 
 
+# ----------------------------------------------------------------------------
+# MuonEq row equilibration
+# ----------------------------------------------------------------------------
+ROWEQ_EPS = NS_EPS
+
+
+def row_equilibrate(x: np.ndarray, eps: float = ROWEQ_EPS) -> np.ndarray:
+    """MuonEq row equilibration.
+
+    [NC] names it as one of the two optional extras layered on the
+    orthogonalisation (leaving it out turns the update's direction by a
+    cosine of 0.986) but prints no formula.  Reading: each row of the matrix,
+    in parameter orientation, is divided by its Euclidean norm plus eps (the
+    1e-7 the Frobenius normalisation adds), so every row enters Newton-Schulz
+    with norm ~1 and a zero row stays zero.  It acts on the momentum-smoothed
+    matrix, before the Frobenius normalisation; the momentum buffer itself is
+    not changed.  The one figure the pages print for it (cos 0.986) was
+    measured with a coefficient table they do not print, so it is context
+    only; the pins are the row norms, the invariance of the result under
+    positive row scaling of the input, and the closed form for a row-scaled
+    matrix with orthonormal rows.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    n = np.sqrt(np.sum(x * x, axis=1, keepdims=True))
+    return x / (n + eps)
+
+
 def muon_step(w: np.ndarray, g: np.ndarray, m: np.ndarray, lr: float, beta: float, wd: float,
               ns_steps: int = 5, coeffs=NS_COEFFS_FIXED, nesterov: bool = True,
               cautious: bool = True, lr_scale: float = 1.0, eps: float = NS_EPS,
-              normuon: bool = False):
-    """One Muon step on one matrix: momentum -> NS -> (NorMuon) -> cautious decay + update.
+              normuon: bool = False, row_equilibrate_input: bool = False):
+    """One Muon step on one matrix: momentum -> (MuonEq) -> NS -> (NorMuon) ->
+    cautious decay + update.
 
     Returns (w_new, m_new, update) in fp64.  lr_scale is the per-matrix shape
     factor some recipes multiply the learning rate by; 1 gives W -= lr*update.
     With normuon the orthogonalised update is row-normalised first ([MAC]
     "The Full Muon Step": normalize_muon_update, then decay, then the step).
+    With row_equilibrate_input the momentum-smoothed matrix is row-equilibrated
+    before the orthogonalisation (row_equilibrate).
     """
     m_new, mt = nesterov_momentum(m, g, beta, nesterov)
+    if row_equilibrate_input:
+        mt = row_equilibrate(mt)
     u = newton_schulz(mt, coeffs, ns_steps, eps)
     if normuon:
         u = normuon_rows(u)
@@ -213,6 +245,28 @@ def trapezoid_lr(step: int, total_steps: int, max_lr: float, min_lr: float,
         return min_lr
     decay = step - warmup - flat
     return min_lr + (max_lr - min_lr) * (1.0 - decay / warmdown)
+
+
+def warmup_cosine_lr(step: int, total_steps: int, max_lr: float, warmup_steps: int,
+                     final_frac: float = 0.1) -> float:
+    """[RACE] "Muon vs AdamW, Lion and Sophia: a fair race" (the bake-off's
+    learning rate, by step): a climb to the peak over the warmup, then a
+    cosine down to a tenth of the peak by the last step.
+
+    Readings for what the page leaves open: step counts from 0; the climb is
+    linear from 0, max_lr*step/warmup_steps, as the trapezoidal schedule's; the
+    cosine's phase runs from 0 at step == warmup_steps to pi at the last step,
+    step == total_steps - 1, so lr = max_lr*(final + (1 - final)*(1 + cos(phase))/2);
+    from the last step on (and when no step is left after the warmup) the
+    value is final_frac*max_lr.
+    """
+    if step < warmup_steps:
+        return max_lr * step / warmup_steps
+    last = total_steps - 1
+    if step >= last or last <= warmup_steps:
+        return max_lr * final_frac
+    phase = np.pi * (step - warmup_steps) / (last - warmup_steps)
+    return max_lr * (final_frac + (1.0 - final_frac) * 0.5 * (1.0 + np.cos(phase)))
 
 
 # ----------------------------------------------------------------------------

@@ -10,9 +10,9 @@ import numpy as np
 import pytest
 
 import oracle
-from tests.test_oracle_pins import (adamw_pin_failures, momentum_pin_failures,
-                                    normuon_pin_failures, ns_pin_failures, schedule_pin_failures,
-                                    update_pin_failures)
+from tests.test_oracle_pins import (adamw_pin_failures, cosine_pin_failures, momentum_pin_failures,
+                                    normuon_pin_failures, ns_pin_failures, rowq_pin_failures,
+                                    schedule_pin_failures, update_pin_failures)
 
 
 def _coeffs(coeffs, steps):
@@ -212,3 +212,79 @@ def _sched_variant(kind):
 @pytest.mark.parametrize("kind", ["no_warmup_ramp", "decay_to_zero", "wrong_fraction"])
 def test_schedule_mutant_caught(kind, pages):
     assert schedule_pin_failures(_sched_variant(kind), pages["trapezoid_chart"]) != []
+
+
+def _cosine_variant(kind):
+    def sched(step, total, max_lr, warmup, final=0.1):
+        if step < warmup:
+            return max_lr * (step + 1 if kind == "warmup_from_one" else step) / warmup
+        last = total if kind == "phase_to_total" else total - 1
+        if step >= last or last <= warmup:
+            return max_lr * (0.0 if kind == "decay_to_zero" else final)
+        p = (step - warmup) / (last - warmup)
+        if kind == "linear":
+            return max_lr * (final + (1 - final) * (1 - p))
+        if kind == "sin_phase":
+            return max_lr * (final + (1 - final) * 0.5 * (1 + np.sin(np.pi * p)))
+        if kind == "decay_to_zero":
+            return max_lr * 0.5 * (1 + np.cos(np.pi * p))
+        return max_lr * (final + (1 - final) * 0.5 * (1 + np.cos(np.pi * p)))
+    return sched
+
+
+@pytest.mark.parametrize("kind", ["warmup_from_one", "phase_to_total", "decay_to_zero", "linear",
+                                  "sin_phase"])
+def test_cosine_mutant_caught(kind, pages):
+    assert cosine_pin_failures(_cosine_variant(kind), pages["race_schedule"]) != []
+
+
+def test_cosine_unmutated_copy_passes(pages):
+    assert cosine_pin_failures(_cosine_variant("none"), pages["race_schedule"]) == []
+
+
+def _rowq_variant(kind):
+    """(equilibrate, step) pair with one planted slip."""
+    def equil(x, eps=oracle.ROWEQ_EPS):
+        x = np.asarray(x, dtype=np.float64)
+        if kind == "columns":
+            return x / (np.sqrt(np.sum(x * x, axis=0, keepdims=True)) + eps)
+        if kind == "squared_norm":
+            return x / (np.sum(x * x, axis=1, keepdims=True) + eps)
+        if kind == "rms_not_norm":
+            return x / (np.sqrt(np.mean(x * x, axis=1, keepdims=True)) + eps)
+        if kind == "no_eps":
+            return x / np.sqrt(np.sum(x * x, axis=1, keepdims=True))
+        return x / (np.sqrt(np.sum(x * x, axis=1, keepdims=True)) + eps)
+
+    def step(w, g, m, lr=0.02, beta=0.95):
+        if kind == "on_grad":
+            g = equil(g)
+        m_new = beta * m + g
+        mt = beta * m_new + g
+        if kind == "into_momentum":
+            m_new = equil(m_new)
+            mt = beta * m_new + g
+        if kind == "after_frobenius":
+            mt = equil(mt / (np.linalg.norm(mt) + oracle.NS_EPS))
+        elif kind == "after_orient":
+            x = mt.T if mt.shape[0] > mt.shape[1] else mt
+            x = equil(x)
+            mt = x.T if mt.shape[0] > mt.shape[1] else x
+        elif kind != "dropped" and kind != "on_grad":
+            mt = equil(mt)
+        u = oracle.newton_schulz(mt)
+        return w - lr * u, m_new, u
+    return equil, step
+
+
+ROWQ_MUTANTS = ["columns", "squared_norm", "rms_not_norm", "no_eps", "on_grad", "into_momentum",
+                "after_frobenius", "after_orient", "dropped"]
+
+
+@pytest.mark.parametrize("kind", ROWQ_MUTANTS)
+def test_rowq_mutant_caught(kind):
+    assert rowq_pin_failures(*_rowq_variant(kind)) != []
+
+
+def test_rowq_unmutated_copy_passes():
+    assert rowq_pin_failures(*_rowq_variant("none")) == []

@@ -398,6 +398,94 @@ def test_muon_step_with_normuon_matches_page_sequence():
 
 
 # ============================================================================
+# MuonEq row-equilibration pins
+# ============================================================================
+def rowq_step(w, g, m):
+    """The oracle's Muon step with row equilibration (lr 0.02, beta 0.95,
+    wd 0, the fixed triple five times)."""
+    return oracle.muon_step(w, g, m, 0.02, 0.95, 0.0, row_equilibrate_input=True)
+
+
+def rowq_pin_failures(equil, step):
+    """equil(x): the row equilibration; step(w, g, m) -> (w_new, m_new, U): a
+    Muon step that applies it (as rowq_step).  The pages name MuonEq row
+    equilibration without a formula; these pins fix the reading (each
+    parameter row divided by its norm + 1e-7, on the momentum-smoothed matrix,
+    before the Frobenius normalisation) by its mathematical consequences."""
+    fails = []
+    rng = np.random.default_rng(21)
+    eps = oracle.ROWEQ_EPS
+    for shape in [(7, 13), (13, 7), (1, 9), (9, 1)]:
+        x = rng.standard_normal(shape) * rng.uniform(0.01, 3.0, size=(shape[0], 1))
+        out = equil(x)
+        if np.shape(out) != x.shape:
+            fails.append(f"shape{shape}")
+            continue
+        n = np.linalg.norm(x, axis=1)
+        if not np.allclose(np.linalg.norm(out, axis=1), n / (n + eps), rtol=1e-12, atol=0):
+            fails.append(f"row_norm{shape}")
+        no = np.linalg.norm(out, axis=1)
+        if np.any(np.sum(out * x, axis=1) <= 0) or \
+                not np.allclose(out * n[:, None], x * no[:, None], rtol=1e-10, atol=1e-14):
+            fails.append(f"row_direction{shape}")
+    z = np.zeros((3, 5))
+    z[1] = 2.0
+    out = equil(z)
+    if not (np.all(out[0] == 0) and np.all(out[2] == 0)):
+        fails.append("zero_row")
+    # Closed form: G = D Q with orthonormal rows (wide).  Equilibrated, the
+    # step sees Q up to eps; after the Frobenius normalisation every singular
+    # value is 1/sqrt(rows), so U = p5(1/sqrt(rows)) Q, whatever D was.
+    q = _qr_orthonormal(rng, 24, 6).T
+    d = np.array([0.03, 0.2, 1.0, 4.0, 9.0, 50.0])[:, None]
+    _, _, u = step(np.zeros((6, 24)), d * q, np.zeros((6, 24)))
+    want = oracle.ns_singular_value_map(np.array([1.0 / np.sqrt(6.0)]), FIXED, 5)[0] * q
+    if np.shape(u) != want.shape or np.abs(u - want).max() > 1e-5:
+        fails.append("closed_form_row_scaled_orthonormal")
+    # Rescaling each parameter row of G and m by a positive factor leaves U
+    # unchanged (up to eps), for tall and wide matrices alike; in a tall
+    # matrix the parameter rows are the columns of the iterated X.
+    for shape in [(30, 8), (8, 30)]:
+        g = rng.standard_normal(shape)
+        m0 = rng.standard_normal(shape)
+        dd = rng.uniform(0.05, 20.0, size=(shape[0], 1))
+        _, _, u1 = step(np.zeros(shape), g, m0)
+        _, _, u2 = step(np.zeros(shape), dd * g, dd * m0)
+        if _rel(u2, u1) > 1e-6:
+            fails.append(f"row_scale_invariance{shape}")
+        # without equilibration the same rescaling does change U
+        u3 = oracle.newton_schulz(dd * (0.95 * (0.95 * m0 + g) + g))
+        if _rel(u3, u1) < 1e-2:
+            fails.append(f"invariance_is_not_trivial{shape}")
+    # the momentum buffer itself is not equilibrated
+    g = rng.standard_normal((12, 20))
+    m0 = rng.standard_normal((12, 20)) * 3.0
+    _, m_new, _ = step(np.zeros_like(g), g, m0)
+    if _rel(m_new, 0.95 * m0 + g) > 1e-15:
+        fails.append("momentum_untouched")
+    return fails
+
+
+def test_rowq_pins():
+    assert rowq_pin_failures(oracle.row_equilibrate, rowq_step) == []
+
+
+def test_rowq_direction_change_is_small(pages):
+    """Context for the page's figure (cos 0.986 between the update with and
+    without MuonEq, measured with another coefficient table): under this
+    reading the fixed triple gives a change of the same small size on the
+    page's two inputs (iid 256x1024; rank-8 plus noise)."""
+    page_cos = pages["muoneq_drop_direction_cos"]
+    cs = []
+    for g in [wl.iid_normal((256, 1024), 1.0, 0), wl.illcond_grad(0)]:
+        u0 = oracle.newton_schulz(g)
+        u1 = oracle.newton_schulz(oracle.row_equilibrate(g))
+        cs.append(float(np.sum(u0 * u1) / np.linalg.norm(u0) / np.linalg.norm(u1)))
+    assert min(cs) < page_cos < max(cs) + 1e-3, cs
+    assert min(cs) > 0.95, cs
+
+
+# ============================================================================
 # schedule pins
 # ============================================================================
 def schedule_pin_failures(sched, pages_chart):
@@ -424,6 +512,45 @@ def schedule_pin_failures(sched, pages_chart):
 
 def test_schedule_pins(pages):
     assert schedule_pin_failures(oracle.trapezoid_lr, pages["trapezoid_chart"]) == []
+
+
+def cosine_pin_failures(sched, race):
+    """sched(step, total_steps, max_lr, warmup_steps, final_frac): the
+    bake-off's warmup + cosine ("Muon vs AdamW, Lion and Sophia: a fair race":
+    a climb to the peak over the warmup, a cosine down to a tenth of the peak
+    by the last step)."""
+    fails = []
+    T, W, f = race["steps"], race["warmup_steps"], race["final_frac"]
+    vals = [sched(t, T, 1.0, W, f) for t in range(T)]
+    last = T - 1
+    if vals[0] != 0.0 or abs(vals[W // 2] - 0.5) > 1e-12:
+        fails.append("warmup_linear")
+    if abs(vals[W] - 1.0) > 1e-12:
+        fails.append("peak_after_warmup")
+    if abs(vals[last] - f) > 1e-12:
+        fails.append("tenth_at_last_step")
+    if any(b > a + 1e-15 for a, b in zip(vals[W:], vals[W + 1:])):
+        fails.append("monotone_decay")
+    if any(b < a for a, b in zip(vals[:W], vals[1:W + 1])):
+        fails.append("monotone_warmup")
+    # cos(pi p) + cos(pi (1 - p)) = 0: lr(W + k) + lr(last - k) = (1 + f) peak
+    for k in (0, 1, 37, 200, (last - W) // 2):
+        if abs(vals[W + k] + vals[last - k] - (1.0 + f)) > 1e-12:
+            fails.append(f"symmetry{k}")
+    # middle and quarter of a decay of 900 steps: cos(pi/2) = 0, cos(pi/4) = sqrt(1/2)
+    if abs(sched(W + 450, W + 901, 1.0, W, f) - (1.0 + f) / 2) > 1e-12:
+        fails.append("midpoint")
+    if abs(sched(W + 225, W + 901, 1.0, W, f) - (f + (1.0 - f) * (1.0 + math.sqrt(0.5)) / 2)) > 1e-12:
+        fails.append("quarter")
+    if abs(sched(300, T, 3e-4, W, f) - 3e-4 * vals[300]) > 1e-18:
+        fails.append("peak_scale")
+    if abs(sched(T + 5, T, 1.0, W, f) - f) > 1e-12:
+        fails.append("after_last")
+    return fails
+
+
+def test_cosine_pins(pages):
+    assert cosine_pin_failures(oracle.warmup_cosine_lr, pages["race_schedule"]) == []
 
 
 # ============================================================================
