@@ -306,7 +306,8 @@ def run_gpu(args):
     e2e_pinned = pinned_fits(grad_bytes, min(world, torch.cuda.device_count()))
     D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e, pinned=e2e_pinned)
     flags = (N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
-             | (N.MUON_NORMUON if args.normuon else 0))
+             | (N.MUON_NORMUON if args.normuon else 0)
+             | (N.MUON_ROW_EQUILIBRATE if args.row_equilibrate else 0))
     ws_bytes = api.muon_workspace_size(D.groups, flags)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     coeffs = W.NS_COEFFS_FIXED
@@ -424,6 +425,7 @@ def run_gpu(args):
             "ns_axpy": ("tensor", work["axpy_flops"]),
             "ns_axpy_update": ("tensor", work["axpy_flops"]),
             "momentum_norm": ("hbm", work["momentum_bytes"]),
+            "momentum_rowq": ("hbm", work["momentum_bytes"]),
             "update": ("hbm", work["update_bytes"]),
             "normuon_update": ("hbm", work["update_bytes"]),
             "adamw": ("hbm", work["adamw_bytes"]),
@@ -434,7 +436,8 @@ def run_gpu(args):
             "ns_gram": work["gram_flops"] * K, "ns_poly": work["poly_flops"] * K,
             "ns_axpy": work["axpy_flops"] * (K - 1 if "ns_axpy_update" in kinds else K),
             "ns_axpy_update": work["axpy_flops"],
-            "momentum_norm": work["momentum_bytes"], "update": work["update_bytes"],
+            "momentum_norm": work["momentum_bytes"], "momentum_rowq": work["momentum_bytes"],
+            "update": work["update_bytes"],
             "normuon_update": work["update_bytes"],
             "adamw": work["adamw_bytes"]}
         roof = None
@@ -461,7 +464,7 @@ def run_gpu(args):
                         "peak_source": f"{peak_src} (HBM copy)",
                         "work_per_launch": per_launch, "work_unit": "algorithmic bytes"}
         ew = {}
-        for k in ("momentum_norm", "update", "normuon_update", "adamw"):
+        for k in ("momentum_norm", "momentum_rowq", "update", "normuon_update", "adamw"):
             if k in kinds:
                 ew[k] = round(per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e9, 1)
         for k in ("ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update"):
@@ -486,7 +489,7 @@ def run_gpu(args):
                        "ns_steps": K, "grads": "bf16", "params_state": "fp32",
                        "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
                        "gemm_tiles": "128x256 single-CTA" if args.single_cta else "256x256 CTA pair",
-                       "normuon": bool(args.normuon)},
+                       "normuon": bool(args.normuon), "row_equilibrate": bool(args.row_equilibrate)},
             "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_ms_per_step": round(ns_ms, 3),
@@ -580,6 +583,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--normuon", action="store_true",
                     help="row-normalise the orthogonalised update (NorMuon)")
+    ap.add_argument("--row-equilibrate", action="store_true",
+                    help="MuonEq row equilibration of the momentum-smoothed matrix before Newton-Schulz")
     ap.add_argument("--single-cta", action="store_true",
                     help="Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of CTA pairs")
     args = ap.parse_args()

@@ -68,9 +68,14 @@ enum {
   MUON_UNFUSED_UPDATE = 8u, /* apply the update in its own kernel instead of the last B*X epilogue */
   MUON_TC_SINGLE_CTA = 16u, /* run the Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of
                                CTA-pair (cta_group::2) 256x256 tiles; same results, for comparison */
-  MUON_NORMUON = 32u        /* NorMuon ("Chapter 4: The MuonAdamW Optimizer", NorMuon): divide every
+  MUON_NORMUON = 32u,       /* NorMuon ("Chapter 4: The MuonAdamW Optimizer", NorMuon): divide every
                                row of U (parameter orientation) by (||row||/sqrt(cols) + 1e-8) before
                                the decay and update, so each row's RMS is 1 and the step's is lr */
+  MUON_ROW_EQUILIBRATE = 64u /* MuonEq row equilibration ("Stuck at the optimizer after figuring out
+                               backward()", mira687's reply, names it without a formula): divide every
+                               row of m~ (parameter orientation) by (||row|| + 1e-7) before the
+                               Frobenius normalisation; the momentum buffer is unchanged.  muon_step
+                               only; needs the workspace sizes computed with this flag */
 };
 
 /*
@@ -102,6 +107,7 @@ size_t muon_workspace_min_size(const muon_group* groups, int n_groups, uint32_t 
  * One Muon step over every matrix of every group.
  *
  *   for each matrix:  m <- beta*m + G;   m~ <- beta*m + G  (MUON_NESTEROV) or m
+ *                     (MUON_ROW_EQUILIBRATE: m~_row <- m~_row / (||m~_row|| + 1e-7))
  *                     X0 <- m~ / (||m~||_F + 1e-7)
  *                     ns_steps x { A = X X^T; B = b_k A + c_k A A; X = a_k X + B X }
  *                     (wide orientation: rows > cols iterates on X^T)
@@ -211,6 +217,22 @@ typedef struct {
 muon_status muon_schedule_advance(muon_schedule_state* state, int64_t total_steps,
                                   float warmup_frac, float warmdown_frac, float final_frac,
                                   muon_stream_t stream);
+
+/*
+ * On the device: step <- step + 1, then lr_mult <- the warmup + cosine
+ * schedule ("Muon vs AdamW, Lion and Sophia: a fair race", the bake-off's
+ * learning rate by step) at the 0-based step s = step - 1:
+ *   s < warmup_steps              s / warmup_steps (linear climb from 0)
+ *   warmup_steps <= s < last      final_frac + (1 - final_frac) * (1 + cos(pi * p)) / 2,
+ *                                 p = (s - warmup_steps) / (last - warmup_steps)
+ *   s >= last                     final_frac
+ * with last = total_steps - 1, so the cosine reaches final_frac (a tenth of
+ * the peak on that page) at the last step.  total_steps >= 1,
+ * 0 <= warmup_steps <= total_steps, final_frac finite; computed in double.
+ * One single-thread kernel on `stream`.
+ */
+muon_status muon_schedule_advance_cosine(muon_schedule_state* state, int64_t total_steps,
+                                         int64_t warmup_steps, float final_frac, muon_stream_t stream);
 
 /* muon_step with the learning rate lr * state->lr_mult read on the device. */
 muon_status muon_step_scheduled(float* const* params, const void* const* grads,

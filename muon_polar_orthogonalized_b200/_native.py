@@ -31,6 +31,7 @@ MUON_FP32_DEBUG = 4
 MUON_UNFUSED_UPDATE = 8
 MUON_TC_SINGLE_CTA = 16
 MUON_NORMUON = 32
+MUON_ROW_EQUILIBRATE = 64
 
 
 class MuonGroup(ctypes.Structure):
@@ -60,6 +61,7 @@ SIGNATURES = {
                                    c_int, POINTER(c_float), c_uint32, c_void_p, c_size_t, c_void_p]),
     "adamw_step": (c_int, [POINTER(AdamWGroup), c_int, c_int64, c_void_p]),
     "muon_schedule_advance": (c_int, [c_void_p, c_int64, c_float, c_float, c_float, c_void_p]),
+    "muon_schedule_advance_cosine": (c_int, [c_void_p, c_int64, c_int64, c_float, c_void_p]),
     "muon_step_scheduled": (c_int, [POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p),
                                     POINTER(MuonGroup), c_int, c_float, c_float, c_float, c_int,
                                     POINTER(c_float), c_uint32, c_void_p, c_size_t, c_void_p,

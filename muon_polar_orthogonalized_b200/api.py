@@ -117,6 +117,14 @@ def muon_schedule_advance(schedule_state, total_steps: int, warmup_frac: float =
     check(st, "muon_schedule_advance")
 
 
+def muon_schedule_advance_cosine(schedule_state, total_steps: int, warmup_steps: int,
+                                 final_frac: float = 0.1, stream=None) -> None:
+    st = N.lib().muon_schedule_advance_cosine(c_void_p(schedule_state.data_ptr()), int(total_steps),
+                                              int(warmup_steps), float(final_frac),
+                                              c_void_p(_stream_handle(stream)))
+    check(st, "muon_schedule_advance_cosine")
+
+
 def muon_orthogonalize(inputs, outputs, groups: Sequence, ns_steps: int, coeffs, flags: int,
                        workspace, workspace_bytes: Optional[int] = None, stream=None) -> None:
     g = make_groups(groups)

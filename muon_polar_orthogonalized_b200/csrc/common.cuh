@@ -39,6 +39,7 @@ struct MatRef {
   int blk_begin;     // first block of this matrix in the launch
   int sidx;          // index of this matrix's scale in the wave's scale array
   float lr;          // lr * lr_scale (update kernel)
+  int pbase;         // MuonEq momentum: index of the first row's partial in `partials`
 };
 
 struct EltParams {
@@ -53,7 +54,8 @@ struct EltParams {
   float wd;
   int cautious;
   int use_scale;     // update/emit: multiply X by the matrix scale (ns_steps == 0)
-  float* partials;   // momentum kernel: one partial sum of squares per block
+  int row_eq;        // MuonEq: momentum kernel row-wise, one partial sum per row
+  float* partials;   // momentum kernel: one partial sum of squares per block (or row)
   float* scales;     // per-matrix 1/(||m~||+eps)
   const DevSched* sched;  // nullptr, or the device schedule (lr multiplier)
 };

@@ -4,6 +4,10 @@
 //                  X0 <- m~ stored in the workspace (bf16, or fp32 in debug
 //                  mode) and one partial sum of m~^2 per block.
 //                  ("Chapter 4: The MuonAdamW Optimizer", The Muon Update Rule)
+//   momentum_rowq  the same momentum, then MuonEq row equilibration: every
+//                  parameter row of m~ divided by (||row|| + 1e-7) before it
+//                  is stored as X0; one partial sum per row
+//                  (nanochat discussion, mira687's reply: MuonEq)
 //   norm_finalize  s <- 1 / (sqrt(sum of partials) + 1e-7), one block per
 //                  matrix, fixed summation order (deterministic).
 //                  ("Chapter 4", Polar Express: X / (||X|| + 1e-7))
@@ -237,12 +241,239 @@ momentum_norm_kernel(const __grid_constant__ EltParams p) {
   }
 }
 
+// ------------------------------------------------------------ momentum_rowq
+// MuonEq: the momentum update, then every parameter row of m~ divided by
+// (||row|| + 1e-7) as it is stored as X0.  Each row's partial is
+// (||m~_row|| f)^2 with f = 1/(||m~_row|| + 1e-7), the squared norm of the
+// equilibrated row, stored at partials[pbase + row]; norm_finalize then
+// yields the Frobenius scale of the equilibrated matrix.  Rows are numbered
+// consecutively over the matrices of a launch (MatRef.blk_begin = first row).
+// Row sums of squares are taken in a fixed order.  The host sorts rows into
+// four launches by width, so that each keeps enough loads in flight:
+//   rowq_warp   vector rows of <= 768 columns: one warp per row, m~ in
+//               registers (6 float4 per lane), shuffle reduction;
+//   rowq_block  vector rows of <= 4096 columns: one block per row, m~ in
+//               registers (4 float4 per thread);
+//   momentum_rowq_kernel, vector rows of <= 16384 columns: one block per row,
+//               m~ in dynamic shared memory (each thread reads back only the
+//               entries it wrote);
+//   momentum_rowq_kernel, longer or unaligned rows: pass 2 recomputes m~ from
+//               G and the momentum this thread just wrote (the same fp32
+//               operations, so the same values).
+constexpr int kRowEqWarpCols = 768;                       // 32 lanes x 6 float4
+constexpr int kRowEqWarpVec = kRowEqWarpCols / 128;
+constexpr int kRowEqBlockVec = 4;
+constexpr int kRowEqBlockCols = kEltThreads * 4 * kRowEqBlockVec;  // 4096
+constexpr int kRowEqSmemCols = 16384;
+constexpr int kRowEqUnroll = 4;  // float4 units in flight per thread (shared-memory path)
+constexpr float kRowEqEps = 1e-7f;
+
+__device__ __forceinline__ float4 momentum4(const EltParams& p, float* m, long long e, float4 g, float4 mv) {
+  if (!m) return g;
+  float4 mn;
+  mn.x = fmaf(p.beta, mv.x, g.x);
+  mn.y = fmaf(p.beta, mv.y, g.y);
+  mn.z = fmaf(p.beta, mv.z, g.z);
+  mn.w = fmaf(p.beta, mv.w, g.w);
+  st_stream(reinterpret_cast<float4*>(m + e), mn);
+  if (!p.nesterov) return mn;
+  return make_float4(fmaf(p.beta, mn.x, g.x), fmaf(p.beta, mn.y, g.y), fmaf(p.beta, mn.z, g.z),
+                     fmaf(p.beta, mn.w, g.w));
+}
+// m~ again from G and the momentum already written by momentum4
+__device__ __forceinline__ float4 lookahead4(const EltParams& p, const float* m, long long e, float4 g) {
+  if (!m) return g;
+  const float4 mn = *reinterpret_cast<const float4*>(m + e);
+  if (!p.nesterov) return mn;
+  return make_float4(fmaf(p.beta, mn.x, g.x), fmaf(p.beta, mn.y, g.y), fmaf(p.beta, mn.z, g.z),
+                     fmaf(p.beta, mn.w, g.w));
+}
+__device__ __forceinline__ float sumsq4(float4 v, float acc) {
+  acc = fmaf(v.x, v.x, acc);
+  acc = fmaf(v.y, v.y, acc);
+  acc = fmaf(v.z, v.z, acc);
+  return fmaf(v.w, v.w, acc);
+}
+__device__ __forceinline__ float4 scale4(float4 v, float f) {
+  return make_float4(v.x * f, v.y * f, v.z * f, v.w * f);
+}
+__device__ __forceinline__ float4 load_m4(const float* m, long long e) {
+  return m ? ld_stream(reinterpret_cast<const float4*>(m + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Loads NV float4 units of one row (unit u at column base + u*stride + lane4),
+// runs the momentum update, keeps m~ in `keep` and returns this thread's sum
+// of squares (units in order).
+template <bool GBF16, int NV>
+__device__ __forceinline__ float rowq_load_regs(const EltParams& p, const MatRef& r, long long e0,
+                                                int first, int stride, float4 (&keep)[NV]) {
+  float4 gv[NV];
+#pragma unroll
+  for (int u = 0; u < NV; ++u) {
+    const int c = first + u * stride;
+    if (c < r.cols) {
+      gv[u] = load_g4<GBF16>(r.g, e0 + c);
+      keep[u] = load_m4(r.m, e0 + c);
+    }
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < NV; ++u) {
+    const int c = first + u * stride;
+    if (c < r.cols) {
+      keep[u] = momentum4(p, r.m, e0 + c, gv[u], keep[u]);
+      acc = sumsq4(keep[u], acc);
+    }
+  }
+  return acc;
+}
+
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads, 3)
+rowq_warp_kernel(const __grid_constant__ EltParams p) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = kEltThreads / 32;
+  const bool f32x = p.x_f32 != 0;
+  for (int row_g = blockIdx.x * wpb + static_cast<int>(threadIdx.x >> 5); row_g < p.total_blocks;
+       row_g += gridDim.x * wpb) {
+    const MatRef& r = p.mats[find_mat(p.mats, p.nmats, row_g)];
+    const int row = row_g - r.blk_begin;
+    const long long e0 = static_cast<long long>(row) * r.cols;
+    float4 keep[kRowEqWarpVec];
+    float acc = rowq_load_regs<GBF16, kRowEqWarpVec>(p, r, e0, lane * 4, 128, keep);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const float nrm = sqrtf(acc);
+    const float f = 1.f / (nrm + kRowEqEps);
+    if (lane == 0) {
+      const float q = nrm * f;
+      p.partials[r.pbase + row] = q * q;
+    }
+    const long long x0 = static_cast<long long>(row) * r.ldx;
+#pragma unroll
+    for (int u = 0; u < kRowEqWarpVec; ++u) {
+      const int c = lane * 4 + u * 128;
+      if (c < r.cols) store_x4(r.x, x0 + c, scale4(keep[u], f), f32x);
+    }
+  }
+}
+
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads)
+rowq_block_kernel(const __grid_constant__ EltParams p) {
+  __shared__ float row_ss;
+  const bool f32x = p.x_f32 != 0;
+  for (int row_g = blockIdx.x; row_g < p.total_blocks; row_g += gridDim.x) {
+    const MatRef& r = p.mats[find_mat(p.mats, p.nmats, row_g)];
+    const int row = row_g - r.blk_begin;
+    const long long e0 = static_cast<long long>(row) * r.cols;
+    float4 keep[kRowEqBlockVec];
+    const float acc = rowq_load_regs<GBF16, kRowEqBlockVec>(p, r, e0, static_cast<int>(threadIdx.x) * 4,
+                                                            kEltThreads * 4, keep);
+    const float tot = block_sum(acc);
+    if (threadIdx.x == 0) row_ss = tot;
+    __syncthreads();
+    const float nrm = sqrtf(row_ss);
+    const float f = 1.f / (nrm + kRowEqEps);
+    if (threadIdx.x == 0) {
+      const float q = nrm * f;
+      p.partials[r.pbase + row] = q * q;
+    }
+    const long long x0 = static_cast<long long>(row) * r.ldx;
+#pragma unroll
+    for (int u = 0; u < kRowEqBlockVec; ++u) {
+      const int c = static_cast<int>(threadIdx.x) * 4 + u * kEltThreads * 4;
+      if (c < r.cols) store_x4(r.x, x0 + c, scale4(keep[u], f), f32x);
+    }
+  }
+}
+
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads)
+momentum_rowq_kernel(const __grid_constant__ EltParams p) {
+  extern __shared__ float4 rowbuf[];  // kRowEqSmemCols / 4 entries at most
+  __shared__ float row_ss;
+  const bool f32x = p.x_f32 != 0;
+  constexpr int kStep = kEltThreads * 4;  // columns per unit
+  for (int row_g = blockIdx.x; row_g < p.total_blocks; row_g += gridDim.x) {
+    const MatRef& r = p.mats[find_mat(p.mats, p.nmats, row_g)];
+    const int row = row_g - r.blk_begin;
+    const long long e0 = static_cast<long long>(row) * r.cols;
+    const long long x0 = static_cast<long long>(row) * r.ldx;
+    const bool in_smem = r.vec && r.cols <= kRowEqSmemCols;
+    float acc = 0.f;
+    if (r.vec) {
+      for (int base = 0; base < r.cols; base += kStep * kRowEqUnroll) {
+        float4 gv[kRowEqUnroll], mv[kRowEqUnroll];
+#pragma unroll
+        for (int u = 0; u < kRowEqUnroll; ++u) {
+          const int c = base + u * kStep + static_cast<int>(threadIdx.x) * 4;
+          if (c < r.cols) {
+            gv[u] = load_g4<GBF16>(r.g, e0 + c);
+            mv[u] = load_m4(r.m, e0 + c);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kRowEqUnroll; ++u) {
+          const int c = base + u * kStep + static_cast<int>(threadIdx.x) * 4;
+          if (c < r.cols) {
+            const float4 mt = momentum4(p, r.m, e0 + c, gv[u], mv[u]);
+            acc = sumsq4(mt, acc);
+            if (in_smem) rowbuf[c >> 2] = mt;
+          }
+        }
+      }
+    } else {
+      for (int c = threadIdx.x; c < r.cols; c += kEltThreads) {
+        const float g = load_g1<GBF16>(r.g, e0 + c);
+        float mt = g;
+        if (r.m) {
+          const float mn = fmaf(p.beta, r.m[e0 + c], g);
+          r.m[e0 + c] = mn;
+          mt = p.nesterov ? fmaf(p.beta, mn, g) : mn;
+        }
+        acc = fmaf(mt, mt, acc);
+      }
+    }
+    const float tot = block_sum(acc);
+    if (threadIdx.x == 0) row_ss = tot;
+    __syncthreads();
+    const float nrm = sqrtf(row_ss);
+    const float f = 1.f / (nrm + kRowEqEps);
+    if (threadIdx.x == 0) {
+      const float q = nrm * f;
+      p.partials[r.pbase + row] = q * q;
+    }
+    if (in_smem) {
+      for (int c = threadIdx.x * 4; c < r.cols; c += kStep)
+        store_x4(r.x, x0 + c, scale4(rowbuf[c >> 2], f), f32x);
+    } else if (r.vec) {
+      for (int c = threadIdx.x * 4; c < r.cols; c += kStep) {
+        const float4 g = load_g4<GBF16>(r.g, e0 + c);
+        store_x4(r.x, x0 + c, scale4(lookahead4(p, r.m, e0 + c, g), f), f32x);
+      }
+    } else {
+      for (int c = threadIdx.x; c < r.cols; c += kEltThreads) {
+        const float g = load_g1<GBF16>(r.g, e0 + c);
+        float mt = g;
+        if (r.m) {
+          const float mn = r.m[e0 + c];
+          mt = p.nesterov ? fmaf(p.beta, mn, g) : mn;
+        }
+        store_x1(r.x, x0 + c, mt * f, f32x);
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------ norm_finalize
+// Sums the matrix's partials (one per momentum block, or one per row with
+// MuonEq) in fp64 in a fixed order.
 __global__ void __launch_bounds__(kEltThreads)
 norm_finalize_kernel(const __grid_constant__ EltParams p) {
   const MatRef& r = p.mats[blockIdx.x];
   const long long numel = static_cast<long long>(r.rows) * r.cols;
-  const int nblk = static_cast<int>((numel + kEltChunk - 1) / kEltChunk);
+  const int nblk = p.row_eq ? r.rows : static_cast<int>((numel + kEltChunk - 1) / kEltChunk);
   double acc = 0.0;
   for (int i = threadIdx.x; i < nblk; i += kEltThreads) acc += p.partials[r.blk_begin + i];
   __shared__ double red[kEltThreads];
@@ -535,6 +766,31 @@ cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, dou
   return cudaGetLastError();
 }
 
+// step <- step + 1; lr_mult <- linear climb over `warm` steps, then a cosine
+// from 1 to final_frac at the last step, total - 1 ("Muon vs AdamW, Lion and
+// Sophia: a fair race", the bake-off's schedule by step).
+__global__ void schedule_cosine_kernel(DevSched* s, long long total, long long warm, double final_frac) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const long long step = s->step;  // 0-based index of the step being taken
+  const long long last = total - 1;
+  double m;
+  if (step < warm) {
+    m = static_cast<double>(step) / static_cast<double>(warm);
+  } else if (step >= last || last <= warm) {
+    m = final_frac;
+  } else {
+    const double phase = 3.141592653589793 * static_cast<double>(step - warm) / static_cast<double>(last - warm);
+    m = final_frac + (1.0 - final_frac) * 0.5 * (1.0 + cos(phase));
+  }
+  s->step = step + 1;
+  s->lr_mult = static_cast<float>(m);
+}
+
+cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm, double fin, cudaStream_t st) {
+  schedule_cosine_kernel<<<1, 32, 0, st>>>(s, total, warm, fin);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- launchers
 int elt_chunk() { return kEltChunk; }
 int adam_chunk() { return kAdamChunk; }
@@ -566,6 +822,65 @@ cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s) {
     k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
   }
   return cudaGetLastError();
+}
+
+int rowq_class(int cols, bool vec) {
+  if (!vec) return 3;
+  if (cols <= kRowEqWarpCols) return 0;
+  if (cols <= kRowEqBlockCols) return 1;
+  if (cols <= kRowEqSmemCols) return 2;
+  return 3;
+}
+
+// Grid for a persistent row kernel: every SM filled to the occupancy the
+// block's dynamic shared memory allows, never more blocks than work items.
+template <typename K>
+static int rowq_grid(K k, int items, size_t smem, int sms) {
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kEltThreads, smem) != cudaSuccess || occ < 1)
+    occ = 1;
+  const long long g = static_cast<long long>(sms) * occ;
+  return static_cast<int>(g < items ? g : items);
+}
+
+// Classes 2 and 3 share momentum_rowq_kernel; its dynamic shared memory is
+// sized for the longest on-chip row of the launch (none for class 3).
+template <bool GBF16>
+static cudaError_t launch_rowq(const EltParams& p, int cls, int sms, cudaStream_t s) {
+  if (cls == 0) {
+    auto k = rowq_warp_kernel<GBF16>;
+    const int wpb = kEltThreads / 32;
+    k<<<rowq_grid(k, (p.total_blocks + wpb - 1) / wpb, 0, sms), kEltThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  if (cls == 1) {
+    auto k = rowq_block_kernel<GBF16>;
+    k<<<rowq_grid(k, p.total_blocks, 0, sms), kEltThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  auto k = momentum_rowq_kernel<GBF16>;
+  static bool attr_set[64] = {};  // per device (the attribute is per device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowEqSmemCols * 4)) !=
+        cudaSuccess)
+      return e;
+    attr_set[dev] = true;
+  }
+  int cols = 0;
+  for (int i = 0; i < p.nmats; ++i)
+    if (p.mats[i].vec && p.mats[i].cols <= kRowEqSmemCols && p.mats[i].cols > cols) cols = p.mats[i].cols;
+  const size_t smem = static_cast<size_t>((cols + 3) / 4) * sizeof(float4);
+  k<<<rowq_grid(k, p.total_blocks, smem, sms), kEltThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_momentum_rowq(const EltParams& p, int cls, int sms, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  return p.grad_bf16 ? launch_rowq<true>(p, cls, sms, s) : launch_rowq<false>(p, cls, sms, s);
 }
 
 cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s) {

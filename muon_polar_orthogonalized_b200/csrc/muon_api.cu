@@ -27,12 +27,15 @@ namespace muon {
 int elt_chunk();
 int adam_chunk();
 cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s);
+cudaError_t launch_momentum_rowq(const EltParams& p, int cls, int sms, cudaStream_t s);
+int rowq_class(int cols, bool vec);
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
 cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
 cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
                                     cudaStream_t st);
+cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm, double fin, cudaStream_t st);
 int tc_tile_m(bool pair);
 int tc_tile_n();
 int tc_b_box_rows(bool pair);
@@ -65,12 +68,12 @@ void muon_set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s",
 namespace {
 enum Kind {
   K_MOMENTUM = 0, K_NORM, K_GRAM, K_POLY, K_AXPY, K_AXPY_UPDATE, K_UPDATE, K_EMIT, K_ADAMW,
-  K_GRAM_F32, K_POLY_F32, K_AXPY_F32, K_AXPY_UPDATE_F32, K_NORMUON_UPDATE, K_COUNT
+  K_GRAM_F32, K_POLY_F32, K_AXPY_F32, K_AXPY_UPDATE_F32, K_NORMUON_UPDATE, K_MOMENTUM_ROWEQ, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
     "momentum_norm", "norm_finalize", "ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update",
     "update", "emit", "adamw", "ns_gram_f32", "ns_poly_f32", "ns_axpy_f32", "ns_axpy_update_f32",
-    "normuon_update"};
+    "normuon_update", "momentum_rowq"};
 
 struct ProfRec {
   int kind;
@@ -179,9 +182,10 @@ struct GroupGeom {
   int r, c, m, n, tall, ldc, ldm, esz;
   size_t xstride, bstride;  // bytes per matrix
   long long nblk;           // momentum-kernel blocks per matrix
+  long long npart;          // Frobenius partial sums per matrix: one per block, or per row (MuonEq)
 };
 
-GroupGeom geom_of(const muon_group& g, bool f32) {
+GroupGeom geom_of(const muon_group& g, bool f32, bool row_eq) {
   GroupGeom q;
   q.r = g.rows;
   q.c = g.cols;
@@ -195,6 +199,7 @@ GroupGeom geom_of(const muon_group& g, bool f32) {
   q.bstride = static_cast<size_t>(q.m) * q.ldm * q.esz;
   const long long numel = static_cast<long long>(g.rows) * g.cols;
   q.nblk = (numel + elt_chunk() - 1) / elt_chunk();
+  q.npart = row_eq ? q.r : q.nblk;
   return q;
 }
 
@@ -202,14 +207,14 @@ struct WaveItem {
   int g, first, count;  // matrices [first, first+count) of group g (group-relative)
   size_t x0, x1, b;     // byte offsets in the workspace
   int sbase;            // index of the item's first matrix in the wave's scale array
-  long long pbase;      // first momentum block of the item's first matrix (wave-relative)
+  long long pbase;      // first partial sum of the item's first matrix (wave-relative)
 };
 
 struct Wave {
   std::vector<WaveItem> items;
   size_t scales_off = 0, partials_off = 0, total = 0;
   int nmats = 0;
-  long long nblocks = 0;
+  long long nblocks = 0;  // partial sums of the wave
 };
 
 // Lay out a wave and return its byte size.
@@ -220,7 +225,7 @@ size_t layout_wave(Wave& w, const std::vector<GroupGeom>& geo) {
     it.sbase = w.nmats;
     it.pbase = w.nblocks;
     w.nmats += it.count;
-    w.nblocks += geo[it.g].nblk * it.count;
+    w.nblocks += geo[it.g].npart * it.count;
   }
   size_t off = kWsHeaderBytes;
   w.scales_off = off;
@@ -258,10 +263,10 @@ muon_status validate_groups(const muon_group* groups, int n_groups) {
 }
 
 // Greedy waves: whole groups in order, split only where the workspace runs out.
-muon_status plan_waves(const muon_group* groups, int n_groups, bool f32, size_t ws_bytes,
+muon_status plan_waves(const muon_group* groups, int n_groups, bool f32, bool row_eq, size_t ws_bytes,
                        std::vector<GroupGeom>& geo, std::vector<Wave>& waves) {
   geo.clear();
-  for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32));
+  for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32, row_eq));
   waves.clear();
   Wave cur;
   for (int gi = 0; gi < n_groups; ++gi) {
@@ -295,9 +300,9 @@ muon_status plan_waves(const muon_group* groups, int n_groups, bool f32, size_t 
   return MUON_OK;
 }
 
-size_t full_wave_size(const muon_group* groups, int n_groups, bool f32) {
+size_t full_wave_size(const muon_group* groups, int n_groups, bool f32, bool row_eq) {
   std::vector<GroupGeom> geo;
-  for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32));
+  for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32, row_eq));
   Wave w;
   for (int gi = 0; gi < n_groups; ++gi) {
     int left = groups[gi].count, first = 0;
@@ -311,10 +316,10 @@ size_t full_wave_size(const muon_group* groups, int n_groups, bool f32) {
   return layout_wave(w, geo);
 }
 
-size_t min_wave_size(const muon_group* groups, int n_groups, bool f32) {
+size_t min_wave_size(const muon_group* groups, int n_groups, bool f32, bool row_eq) {
   size_t mx = kWsHeaderBytes;
   std::vector<GroupGeom> geo;
-  for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32));
+  for (int i = 0; i < n_groups; ++i) geo.push_back(geom_of(groups[i], f32, row_eq));
   for (int gi = 0; gi < n_groups; ++gi) {
     if (groups[gi].count == 0) continue;
     Wave w;
@@ -364,16 +369,84 @@ struct StepArgs {
   const DevSched* sched;  // device schedule (lr multiplier), or nullptr
 };
 
+// MuonEq row equilibration applies to muon_step only (the orthogonaliser has
+// no momentum stage).
+inline bool row_equilibrate(const StepArgs& a) { return !a.orth && (a.flags & MUON_ROW_EQUILIBRATE) != 0; }
+
 struct Ctx {
   const StepArgs& a;
   const std::vector<GroupGeom>& geo;
   const DevInfo& dev;
 };
 
+// MuonEq momentum: one launch per row class (rowq_class: by row width and
+// alignment) and grad dtype, at most kMaxMatsPerLaunch matrices each.  Rows
+// are numbered per launch; each matrix's partials start at its wave-relative
+// first row (pbase), the order norm_finalize reads them in.
+muon_status run_momentum_rowq(const Ctx& C, const Wave& w) {
+  const StepArgs& a = C.a;
+  float* partials = reinterpret_cast<float*>(a.ws + w.partials_off);
+  EltParams P;
+  std::memset(&P, 0, sizeof(P));
+  int pending_dtype = -1;
+  auto flush = [&](int cls) -> muon_status {
+    if (P.nmats == 0) return MUON_OK;
+    P.beta = a.beta;
+    P.nesterov = (a.flags & MUON_NESTEROV) ? 1 : 0;
+    P.x_f32 = (a.flags & MUON_FP32_DEBUG) ? 1 : 0;
+    P.row_eq = 1;
+    P.partials = partials;
+    P.grad_bf16 = pending_dtype == MUON_BF16;
+    cudaError_t e = timed_launch(K_MOMENTUM_ROWEQ, a.stream,
+                                 [&] { return launch_momentum_rowq(P, cls, C.dev.sms, a.stream); });
+    if (e != cudaSuccess) return cuda_fail(e, "MuonEq momentum launch");
+    std::memset(&P, 0, sizeof(P));
+    pending_dtype = -1;
+    return MUON_OK;
+  };
+  for (int cls = 0; cls < 4; ++cls) {
+    long long pbase = 0;
+    for (const auto& it : w.items) {
+      const GroupGeom& q = C.geo[it.g];
+      const muon_group& g = a.groups[it.g];
+      for (int j = 0; j < it.count; ++j, pbase += q.npart) {
+        const int pi = g.first + it.first + j;
+        const size_t ga = (g.grad_dtype == MUON_BF16) ? 8 : 16;
+        const bool vec = (q.c % 4) == 0 && aligned(a.grads[pi], ga) && aligned(a.momentum[pi], 16);
+        if (rowq_class(q.c, vec) != cls) continue;
+        if (P.nmats == kMaxMatsPerLaunch || (pending_dtype != -1 && pending_dtype != g.grad_dtype)) {
+          muon_status st = flush(cls);
+          if (st != MUON_OK) return st;
+        }
+        pending_dtype = g.grad_dtype;
+        MatRef& r = P.mats[P.nmats];
+        r.rows = q.r;
+        r.cols = q.c;
+        r.ldx = q.ldc;
+        r.sidx = it.sbase + j;
+        r.x = a.ws + it.x0 + q.xstride * j;
+        r.g = a.grads[pi];
+        r.m = a.momentum[pi];
+        r.vec = vec ? 1 : 0;
+        r.blk_begin = P.total_blocks;  // rows, numbered across the launch
+        r.pbase = static_cast<int>(pbase);
+        P.total_blocks += q.r;
+        P.nmats += 1;
+      }
+    }
+    muon_status st = flush(cls);
+    if (st != MUON_OK) return st;
+  }
+  return MUON_OK;
+}
+
 muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
-  // kind: 0 momentum_norm, 1 finalize, 2 update, 3 emit, 4 NorMuon update (row-wise)
+  // kind: 0 momentum_norm (row-wise with MuonEq), 1 finalize, 2 update, 3 emit,
+  // 4 NorMuon update (row-wise)
   const StepArgs& a = C.a;
   const bool f32 = (a.flags & MUON_FP32_DEBUG) != 0;
+  const bool row_eq = row_equilibrate(a);
+  if (kind == 0 && row_eq) return run_momentum_rowq(C, w);
   float* scales = reinterpret_cast<float*>(a.ws + w.scales_off);
   float* partials = reinterpret_cast<float*>(a.ws + w.partials_off);
   // matrices of the wave in order, batched <= kMaxMatsPerLaunch per launch and,
@@ -392,6 +465,7 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
     P.use_scale = (a.ns_steps == 0) ? 1 : 0;
     P.scales = scales;
     P.sched = a.sched;
+    P.row_eq = row_eq ? 1 : 0;
     cudaError_t e = cudaSuccess;
     if (kind == 0) {
       P.partials = partials + launch_blk0;
@@ -459,7 +533,7 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
         r.blk_begin = P.total_blocks;
         P.total_blocks += static_cast<int>(q.nblk);
       }
-      wave_blk += q.nblk;
+      wave_blk += q.npart;
       P.nmats += 1;
     }
   }
@@ -632,7 +706,7 @@ muon_status run_step(const StepArgs& a, size_t ws_bytes) {
   std::vector<GroupGeom> geo;
   std::vector<Wave> waves;
   const bool normuon = (a.flags & MUON_NORMUON) != 0 && !a.orth;
-  muon_status st = plan_waves(a.groups, a.n_groups, f32, ws_bytes, geo, waves);
+  muon_status st = plan_waves(a.groups, a.n_groups, f32, row_equilibrate(a), ws_bytes, geo, waves);
   if (st != MUON_OK) return st;
   DevInfo dev;
   if ((st = device_info(&dev)) != MUON_OK) return st;
@@ -665,7 +739,7 @@ muon_status validate_common(const muon_group* groups, int n_groups, int ns_steps
   muon_status st = validate_groups(groups, n_groups);
   if (st != MUON_OK) return st;
   if (flags & ~(MUON_NESTEROV | MUON_CAUTIOUS_WD | MUON_FP32_DEBUG | MUON_UNFUSED_UPDATE |
-                MUON_TC_SINGLE_CTA | MUON_NORMUON))
+                MUON_TC_SINGLE_CTA | MUON_NORMUON | MUON_ROW_EQUILIBRATE))
     return fail(MUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (ns_steps < 0 || ns_steps > kMaxNsSteps)
     return fail(MUON_ERR_INVALID_ARG, "ns_steps %d outside [0, %d]", ns_steps, kMaxNsSteps);
@@ -674,7 +748,8 @@ muon_status validate_common(const muon_group* groups, int n_groups, int ns_steps
     if (!std::isfinite(coeffs[i])) return fail(MUON_ERR_INVALID_ARG, "coeffs[%d] not finite", i);
   if (!workspace) return fail(MUON_ERR_WORKSPACE, "workspace is NULL");
   if (!aligned(workspace, 256)) return fail(MUON_ERR_WORKSPACE, "workspace not 256-byte aligned");
-  const size_t need = min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
+  const size_t need = min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0,
+                                    (flags & MUON_ROW_EQUILIBRATE) != 0);
   if (workspace_bytes < need)
     return fail(MUON_ERR_WORKSPACE, "workspace of %zu bytes < minimum %zu", workspace_bytes, need);
   return MUON_OK;
@@ -697,12 +772,14 @@ extern "C" {
 
 size_t muon_workspace_size(const muon_group* groups, int n_groups, uint32_t flags) {
   if (validate_groups(groups, n_groups) != MUON_OK) return 0;
-  return full_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
+  return full_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0,
+                        (flags & MUON_ROW_EQUILIBRATE) != 0);
 }
 
 size_t muon_workspace_min_size(const muon_group* groups, int n_groups, uint32_t flags) {
   if (validate_groups(groups, n_groups) != MUON_OK) return 0;
-  return min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0);
+  return min_wave_size(groups, n_groups, (flags & MUON_FP32_DEBUG) != 0,
+                       (flags & MUON_ROW_EQUILIBRATE) != 0);
 }
 
 static muon_status muon_step_impl(float* const* params, const void* const* grads,
@@ -872,6 +949,23 @@ muon_status muon_schedule_advance(muon_schedule_state* state, int64_t total_step
   if (st != MUON_OK) return st;
   cudaError_t e = launch_schedule_advance(reinterpret_cast<DevSched*>(state), total_steps, warmup_frac,
                                           warmdown_frac, final_frac, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+  return MUON_OK;
+}
+
+muon_status muon_schedule_advance_cosine(muon_schedule_state* state, int64_t total_steps,
+                                         int64_t warmup_steps, float final_frac, muon_stream_t stream) {
+  g_err[0] = '\0';
+  if (!state || !aligned(state, 8)) return fail(MUON_ERR_INVALID_ARG, "schedule state is NULL or not 8-byte aligned");
+  if (total_steps < 1) return fail(MUON_ERR_INVALID_ARG, "total_steps < 1");
+  if (warmup_steps < 0 || warmup_steps > total_steps)
+    return fail(MUON_ERR_INVALID_ARG, "warmup_steps must be in [0, total_steps]");
+  if (!std::isfinite(final_frac)) return fail(MUON_ERR_INVALID_ARG, "final_frac not finite");
+  DevInfo dev;
+  muon_status st = device_info(&dev);
+  if (st != MUON_OK) return st;
+  cudaError_t e = launch_schedule_cosine(reinterpret_cast<DevSched*>(state), total_steps, warmup_steps,
+                                         final_frac, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
   return MUON_OK;
 }

@@ -24,18 +24,21 @@ class MuonAdamW:
                  lr: float = 0.02, momentum: float = 0.95, weight_decay: float = 0.01,
                  ns_steps: int = 5, coeffs=DEFAULT_COEFFS, nesterov: bool = True,
                  cautious: bool = True, lr_scale_fn=None, fp32_debug: bool = False,
-                 fused_update: bool = True, normuon: bool = False,
+                 fused_update: bool = True, normuon: bool = False, row_equilibrate: bool = False,
                  workspace_bytes: Optional[int] = None):
         """muon_params: fp32 2-D CUDA tensors.  adamw_groups: dicts with keys
         params, lr, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.  lr_scale_fn:
         optional (rows, cols) -> float learning-rate multiplier per shape.
-        normuon: row-normalise the orthogonalised update (NorMuon)."""
+        normuon: row-normalise the orthogonalised update (NorMuon).
+        row_equilibrate: row-equilibrate the momentum-smoothed matrix before
+        the orthogonalisation (MuonEq)."""
         self.lr, self.beta, self.wd = lr, momentum, weight_decay
         self.ns_steps, self.coeffs = ns_steps, coeffs
         self.flags = ((N.MUON_NESTEROV if nesterov else 0) | (N.MUON_CAUTIOUS_WD if cautious else 0)
                       | (N.MUON_FP32_DEBUG if fp32_debug else 0)
                       | (0 if fused_update else N.MUON_UNFUSED_UPDATE)
-                      | (N.MUON_NORMUON if normuon else 0))
+                      | (N.MUON_NORMUON if normuon else 0)
+                      | (N.MUON_ROW_EQUILIBRATE if row_equilibrate else 0))
         # shape groups: matrices with equal (rows, cols) are contiguous in the pointer arrays
         order: Dict[tuple, List[torch.Tensor]] = {}
         for p in muon_params:

@@ -374,6 +374,105 @@ def test_normuon_parity(dev, fp32, ns):
         print((r, c), "ns", ns, "fp32" if fp32 else "bf16", "normuon step rel err", e)
 
 
+# ---------------------------------------------------------------- MuonEq
+# row classes of the MuonEq momentum kernels: <= 768 columns (one warp per
+# row), <= 4096 (one block, registers), <= 16384 (one block, shared memory),
+# longer or unaligned (recomputed)
+ROWEQ_SHAPES = [(1024, 256), (130, 200), (4100, 36), (256, 1024), (40, 3000), (24, 5000),
+                (66, 130), (8, 20000)]
+
+
+def bf16_gate(r, c, ns, e_emul):
+    """bf16-mode tolerance: 2e-2 (tol_bf16), or, where the method's own bf16
+    arithmetic (the bf16-emulated oracle on the same input) is already
+    further than that from fp64, 1.15 x that error + 1e-3.  At some widths
+    (m = 32..36, e.g. 4100 x 36) the emulated oracle is 2.0-2.5e-2 from fp64
+    for well-conditioned input, because the five-step map amplifies bf16
+    storage error there."""
+    return max(tol_bf16(r, c, ns), 1.15 * e_emul + 1e-3)
+
+
+def rowq_grad(shape, seed, step):
+    """iid rows scaled by 10^U(-2, 2), so that equilibration matters; row 5
+    of a matrix with more than 5 rows is zero."""
+    rng = np.random.default_rng(wl.seed_of("rowq", seed, step, *shape))
+    g = rng.standard_normal(shape) * 10.0 ** rng.uniform(-2, 2, size=(shape[0], 1))
+    if shape[0] > 5:
+        g[5] = 0.0
+    return g
+
+
+@pytest.mark.parametrize("gdt", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["bf16", "fp32", "fp32_ns0", "bf16_normuon"])
+def test_row_equilibrate_parity(dev, gdt, mode):
+    """MuonEq row equilibration (nanochat discussion, mira687's reply) on
+    every row path of the kernel: rows kept on chip (wide, tall, ragged),
+    unaligned rows (130 columns), rows longer than the on-chip limit (20000
+    columns) and many short rows (4100 x 36).  Three steps with the momentum
+    carried; each step is compared with the oracle run from the GPU's own
+    W and m before it."""
+    fp32 = mode.startswith("fp32")
+    ns = 0 if mode == "fp32_ns0" else 5
+    normuon = mode == "bf16_normuon"
+    shapes = ROWEQ_SHAPES
+    groups, W, G, M, hW, hG = make_state(dev, shapes, gdt, 31)
+    flags = STEP_FLAGS | N.MUON_ROW_EQUILIBRATE | (N.MUON_FP32_DEBUG if fp32 else 0) \
+        | (N.MUON_NORMUON if normuon else 0)
+    ws = workspace(api.muon_workspace_size(groups, flags), dev)
+    lr, wd = 0.02, 0.01
+    for step in range(3):
+        w_old = [host64(w) for w in W]
+        m_old = [host64(m) for m in M]
+        hg = []
+        for i, shp in enumerate(shapes):
+            g = wl.round_through_dtype(rowq_grad(shp, i, step), gdt)
+            hg.append(g)
+            G[i].copy_(dev_tensor(g, gdt, dev))
+        api.muon_step(W, G, M, groups, lr, 0.95, wd, ns, FIXED, flags, ws)
+        torch.cuda.synchronize()
+        for i, (r, c) in enumerate(shapes):
+            rw, rm, _ = oracle.muon_step(w_old[i], hg[i], m_old[i], lr, 0.95, wd, ns_steps=ns,
+                                         normuon=normuon, row_equilibrate_input=True)
+            if fp32:
+                tol = TOL_F32
+                if ns == 0:
+                    # U = s X0 is tiny (entries ~ 1/sqrt(rows cols)), so the
+                    # fp32 rounding of the stored W dominates W_old - W_new;
+                    # gate the stored tensor itself
+                    assert rel(host64(W[i]), rw) <= 1e-7
+            else:
+                _, mt = oracle.nesterov_momentum(m_old[i], hg[i], 0.95)
+                ue = oracle.newton_schulz_bf16_emulated(oracle.row_equilibrate(mt), FIXED, ns)
+                if normuon:
+                    ue = oracle.normuon_rows(ue)
+                rwe = oracle.cautious_weight_decay_update(w_old[i], ue, lr, wd, True)
+                tol = bf16_gate(r, c, ns, rel(w_old[i] - rwe, w_old[i] - rw))
+            e = check_step(w_old[i], host64(W[i]), host64(M[i]), rw, rm, tol=tol)
+            print((r, c), mode, gdt, "step", step, "rel err", e, "tol", tol)
+
+
+def test_row_equilibrate_matters_and_is_row_scale_invariant(dev):
+    """Rescaling each row of G by a positive factor leaves the MuonEq update
+    unchanged (the step from zero momentum), while the plain update changes."""
+    shapes = [(192, 640), (640, 192)]
+    outs = {}
+    for variant in ["plain", "scaled"]:
+        for eq in [False, True]:
+            groups, W, G, M, hW, hG = make_state(dev, shapes, "f32", 33)
+            if variant == "scaled":
+                for i, (r, c) in enumerate(shapes):
+                    d = np.random.default_rng(40 + i).uniform(0.1, 10.0, size=(r, 1))
+                    G[i].copy_(dev_tensor(hG[i] * d, "f32", dev))
+            flags = N.MUON_NESTEROV | (N.MUON_ROW_EQUILIBRATE if eq else 0)
+            ws = workspace(api.muon_workspace_size(groups, flags), dev)
+            api.muon_step(W, G, M, groups, 0.02, 0.95, 0.0, 5, FIXED, flags, ws)
+            torch.cuda.synchronize()
+            outs[(variant, eq)] = [(hW[i] - host64(W[i])) / 0.02 for i in range(len(shapes))]
+    for i in range(len(shapes)):
+        assert rel(outs[("scaled", True)][i], outs[("plain", True)][i]) < 2e-2
+        assert rel(outs[("scaled", False)][i], outs[("plain", False)][i]) > 5e-2
+
+
 # ---------------------------------------------------------------- AdamW
 @pytest.mark.parametrize("gdt", ["f32", "bf16"])
 def test_adamw_parity(dev, gdt):
@@ -553,6 +652,24 @@ def test_device_schedule_matches_trapezoid(dev):
         assert step == t
         want = oracle.trapezoid_lr(t - 1, total, 1.0, 0.1, 0.1, 0.2)
         assert abs(mult - want) <= 1e-7 * max(1.0, abs(want)), (t, mult, want)
+
+
+def test_device_cosine_schedule_matches_oracle(dev, pages):
+    """The device warmup + cosine schedule follows the bake-off's ("Muon vs
+    AdamW, Lion and Sophia: a fair race": 1000 steps, warmup 100, down to a
+    tenth of the peak by the last step) step by step, and beyond the end."""
+    race = pages["race_schedule"]
+    T, Wu, f = race["steps"], race["warmup_steps"], race["final_frac"]
+    state = api.new_schedule_state(dev, 1.0, 0)
+    got = []
+    for _ in range(T + 3):
+        api.muon_schedule_advance_cosine(state, T, Wu, f)
+        got.append(api.read_schedule_state(state))
+    for t, (mult, step) in enumerate(got):
+        assert step == t + 1
+        want = oracle.warmup_cosine_lr(t, T, 1.0, Wu, f)
+        assert abs(mult - want) <= 1e-7 + 1e-6 * abs(want), (t, mult, want)
+    assert abs(got[Wu][0] - 1.0) < 1e-7 and abs(got[T - 1][0] - f) < 1e-7
 
 
 def test_scheduled_graph_replay_matches_eager(dev):

@@ -78,7 +78,7 @@ def _call_step(L, groups, ptr_count, ns=5, coeffs=True, flags=3, ws=0x1000, wsb=
     (dict(ns=17), N.MUON_ERR_INVALID_ARG),
     (dict(ns=-1), N.MUON_ERR_INVALID_ARG),
     (dict(coeffs=False), N.MUON_ERR_INVALID_ARG),
-    (dict(flags=64), N.MUON_ERR_INVALID_ARG),
+    (dict(flags=128), N.MUON_ERR_INVALID_ARG),
     (dict(ws=0), N.MUON_ERR_WORKSPACE),
     (dict(ws=0x1010), N.MUON_ERR_WORKSPACE),                                 # misaligned
     (dict(wsb=100), N.MUON_ERR_WORKSPACE),
@@ -92,6 +92,20 @@ def test_muon_step_validation(L, case, expect):
     st = _call_step(L, groups, 2, **case)
     assert st == expect, N.last_error()
     assert N.last_error() != ""
+
+
+def test_row_equilibrate_workspace_holds_one_partial_per_row():
+    """MuonEq keeps one Frobenius partial per parameter row: for short rows
+    (768 columns, fewer elements per row than a momentum block) the
+    workspace grows by the extra partials, never shrinks, and a flag-less
+    size is too small for a flagged call."""
+    groups = [(768, 768, 48, 0, 1, 1.0), (3072, 768, 12, 48, 1, 1.0)]
+    plain = api.muon_workspace_size(groups, 0)
+    eq = api.muon_workspace_size(groups, N.MUON_ROW_EQUILIBRATE)
+    assert eq > plain
+    rows = 48 * 768 + 12 * 3072
+    assert eq - plain <= 4 * rows + 2048
+    assert api.muon_workspace_min_size(groups, N.MUON_ROW_EQUILIBRATE) > api.muon_workspace_min_size(groups, 0)
 
 
 def test_adamw_validation(L):
@@ -143,6 +157,11 @@ def test_schedule_validation(L):
     assert L.muon_schedule_advance(st, 0, 0.1, 0.2, 0.1, None) == N.MUON_ERR_INVALID_ARG
     assert L.muon_schedule_advance(st, 10, 0.7, 0.5, 0.1, None) == N.MUON_ERR_INVALID_ARG
     assert L.muon_schedule_advance(ctypes.c_void_p(0x1004), 10, 0.1, 0.2, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance_cosine(None, 10, 1, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance_cosine(st, 0, 0, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance_cosine(st, 10, 11, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance_cosine(st, 10, -1, 0.1, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_schedule_advance_cosine(st, 10, 1, float("nan"), None) == N.MUON_ERR_INVALID_ARG
     p = (ctypes.c_void_p * 1)(0x10000)
     n = (ctypes.c_int64 * 1)(16)
     g = N.AdamWGroup(p, p, p, p, n, 1, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0)
