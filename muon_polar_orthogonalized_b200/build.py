@@ -26,7 +26,7 @@ LIB_NAME = "libmuon_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
 SOURCES = ["muon_api.cu", "k_elementwise.cu", "k_gemm_tc.cu", "k_gemm_simt.cu", "muon_noalloc.cu"]
-HEADERS = ["common.cuh", "sm100.cuh"]
+HEADERS = ["common.cuh", "elt_params.cuh", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
           "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]

@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "elt_params.cuh"
 
 namespace muon {
 

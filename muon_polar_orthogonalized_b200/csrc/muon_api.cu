@@ -21,6 +21,7 @@
 
 #include "../../include/muon_b200.h"
 #include "common.cuh"
+#include "elt_params.cuh"
 
 namespace muon {
 // kernels (k_elementwise.cu, k_gemm_tc.cu, k_gemm_simt.cu)
