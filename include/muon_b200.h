@@ -67,10 +67,13 @@ enum {
   MUON_FP32_DEBUG = 4u,     /* fp32 operands and fp32 FMA GEMMs (slow; tolerance 1e-4 mode) */
   MUON_UNFUSED_UPDATE = 8u, /* apply the update in its own kernel instead of the last B*X epilogue */
   MUON_TC_SINGLE_CTA = 16u, /* run the Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of
-                               CTA-pair (cta_group::2) 256x256 tiles; same results, for comparison */
+                               CTA-pair (cta_group::2) tiles; same results, for comparison */
   MUON_NORMUON = 32u,       /* NorMuon ("Chapter 4: The MuonAdamW Optimizer", NorMuon): divide every
                                row of U (parameter orientation) by (||row||/sqrt(cols) + 1e-8) before
                                the decay and update, so each row's RMS is 1 and the step's is lr */
+  MUON_TC_NARROW_TILES = 128u, /* run the Gram products on 256x256 CTA-pair tiles with two TMEM
+                               accumulators (as the other products always are) instead of 256x512
+                               tiles with one; same results, for comparison */
   MUON_ROW_EQUILIBRATE = 64u /* MuonEq row equilibration ("Stuck at the optimizer after figuring out
                                backward()", mira687's reply, names it without a formula): divide every
                                row of m~ (parameter orientation) by (||row|| + 1e-7) before the
@@ -160,8 +163,8 @@ muon_status muon_step_noalloc(float* const* params, const void* const* grads,
 /*
  * The orthogonaliser alone: outputs[i] <- NS(inputs[i]) as fp32, rows x cols,
  * with the same normalisation, orientation, iteration and bf16 rounding of
- * the result as muon_step.  inputs[i] dtype per group.  Only MUON_FP32_DEBUG
- * and MUON_TC_SINGLE_CTA are honoured in `flags`.
+ * the result as muon_step.  inputs[i] dtype per group.  Only MUON_FP32_DEBUG,
+ * MUON_TC_SINGLE_CTA and MUON_TC_NARROW_TILES are honoured in `flags`.
  */
 muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs,
                                const muon_group* groups, int n_groups,

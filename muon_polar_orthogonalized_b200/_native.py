@@ -32,6 +32,7 @@ MUON_UNFUSED_UPDATE = 8
 MUON_TC_SINGLE_CTA = 16
 MUON_NORMUON = 32
 MUON_ROW_EQUILIBRATE = 64
+MUON_TC_NARROW_TILES = 128
 
 
 class MuonGroup(ctypes.Structure):

@@ -16,13 +16,17 @@
 // s is the Frobenius scale 1/(||m~||+1e-7), applied on the first iteration
 // only (X0 is stored unscaled; bf16 rounding is scale-free up to exponent).
 //
-// Structure: persistent grouped kernel, one CTA per SM, 128x256 output tiles,
-// BK = 64, 4-stage TMA -> shared-memory ring, tcgen05.mma kind::f16 (bf16 in,
-// fp32 accumulate) issued by one thread into a double-buffered TMEM
-// accumulator (2 x 256 columns), and four epilogue warps that drain TMEM with
-// tcgen05.ld while the next tile's MMAs run.
+// Structure: persistent grouped kernel, one CTA per SM (CTA pairs by
+// default), BK = 64, a TMA -> shared-memory ring, tcgen05.mma kind::f16 (bf16
+// in, fp32 accumulate) issued by one thread into TMEM, and eight epilogue
+// warps that drain TMEM with tcgen05.ld.  Tiles: 256x256 on a CTA pair with
+// two 256-column accumulators (one tile's epilogue overlaps the next tile's
+// MMAs) and a 6-stage ring; the Gram products use 256x512 pair tiles (two
+// N=256 MMAs per K step into one 512-column accumulator, 4-stage ring).
+// Single-CTA mode: 128x256 tiles, 4-stage ring.
 //   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
-//   warps 2-5: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31)
+//   warps 2-9: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31; two warps
+//              per lane quadrant split the tile's columns)
 // No multicast is used anywhere.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,31 +37,41 @@
 namespace muon {
 
 // Tile geometry.  Single-CTA mode: 128x256 tiles, one SM per tile.  Pair mode
-// (cta_group::2): 256x256 tiles on a CTA pair; each CTA stages 128 rows of A
-// and 128 rows (N/2) of B, the leader issues one 256x256x16 MMA per K step
-// that reads both CTAs' shared memory, and each CTA's TMEM holds its 128
-// accumulator rows.
+// (cta_group::2): 256 x (256*NSUB) tiles on a CTA pair; each CTA stages 128
+// rows of A and, per 256-column sub-tile, 128 rows (half) of B; the leader
+// issues NSUB 256x256x16 MMAs per K step that read both CTAs' shared memory,
+// and each CTA's TMEM holds its 128 accumulator rows.  NSUB = 1: two
+// accumulators of 256 columns, so one tile's epilogue overlaps the next
+// tile's MMAs.  NSUB = 2: one 512-column accumulator (all of TMEM), 25% fewer
+// operand bytes per FLOP from L2, the epilogue drain no longer overlapped.
 #ifndef MUON_TC_PAIR_STAGES
 #define MUON_TC_PAIR_STAGES 6
+#endif
+#ifndef MUON_TC_WIDE_STAGES
+#define MUON_TC_WIDE_STAGES 4
 #endif
 #ifndef MUON_TC_RASTER_GN
 #define MUON_TC_RASTER_GN 8
 #endif
 
-template <bool PAIR>
+template <bool PAIR, int NSUB>
 struct TcCfg {
+  static_assert(NSUB == 1 || (PAIR && NSUB == 2), "512-column tiles need CTA pairs");
   static constexpr int BM = PAIR ? 256 : 128;        // tile rows
-  static constexpr int BN = 256;                     // tile columns
+  static constexpr int BN = 256 * NSUB;              // tile columns
   static constexpr int BK = 64;
   static constexpr int A_ROWS = 128;                 // A rows staged per CTA
-  static constexpr int B_ROWS = PAIR ? 128 : 256;    // B rows staged per CTA
+  static constexpr int SUB_B_ROWS = PAIR ? 128 : 256;  // B rows staged per CTA per 256-column sub-tile
+  static constexpr int B_ROWS = SUB_B_ROWS * NSUB;
   static constexpr int A_BYTES = A_ROWS * BK * 2;
+  static constexpr int SUB_B_BYTES = SUB_B_ROWS * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = PAIR ? MUON_TC_PAIR_STAGES : 4;
+  static constexpr int STAGES = NSUB == 2 ? MUON_TC_WIDE_STAGES : PAIR ? MUON_TC_PAIR_STAGES : 4;
+  static constexpr int ACC_BUFS = NSUB == 1 ? 2 : 1;   // TMEM accumulators (512 columns in all)
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 };
-constexpr int TC_BN = 256;
+constexpr int TC_BN = 256;   // columns of one MMA (N) and of a narrow tile
 #ifndef MUON_TC_EPI_WARPS
 #define MUON_TC_EPI_WARPS 8
 #endif
@@ -77,7 +91,7 @@ struct TileCoord {
 // Linear tile index -> (problem, matrix, tile row, tile column).  Symmetric
 // problems enumerate, per tile row I, only the tile columns that reach the
 // upper triangle: J >= I*BM/BN.
-template <int BM>
+template <int BM, int BN>
 __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
   int pi = 0;
   while (pi + 1 < p.nprob && t >= p.prob[pi + 1].tile_begin) ++pi;
@@ -89,13 +103,13 @@ __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
   if (q.sym) {
     int I = 0;
     for (;;) {
-      const int cnt = q.tiles_n - (I * BM) / TC_BN;
+      const int cnt = q.tiles_n - (I * BM) / BN;
       if (r < cnt) break;
       r -= cnt;
       ++I;
     }
     tm = I;
-    tn = (I * BM) / TC_BN + r;
+    tn = (I * BM) / BN + r;
   } else {
     const int band_tiles = q.tiles_m * TC_RASTER_GN;
     const int band = r / band_tiles;
@@ -165,12 +179,15 @@ __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const G
 
 struct EpiIn {
   uint4 e[4];     // 32 bf16 of the epilogue operand (A or X)
+};
+struct EpiW {
   float4 w[8];    // 32 fp32 parameters (fused update)
 };
 
+// The bf16 operand (A or X) of one chunk.
 template <int EPI>
 __device__ __forceinline__ void epilogue_load(const TcGemmParams& p, const GemmProblem& q, int mat,
-                                              int i, int j0, bool full, bool wvec, EpiIn& in) {
+                                              int i, int j0, bool full, EpiIn& in) {
   if (i >= q.M) return;
   if (EPI != EPI_GRAM && full) {
     const uint4* e4 = reinterpret_cast<const uint4*>(
@@ -178,6 +195,13 @@ __device__ __forceinline__ void epilogue_load(const TcGemmParams& p, const GemmP
 #pragma unroll
     for (int k = 0; k < 4; ++k) in.e[k] = e4[k];
   }
+}
+
+// The parameters W of one chunk (fused update).
+template <int EPI>
+__device__ __forceinline__ void epilogue_load_w(const TcGemmParams& p, const GemmProblem& q, int mat,
+                                                int i, int j0, bool full, bool wvec, EpiW& in) {
+  if (i >= q.M) return;
   if (EPI == EPI_AXPY_UPDATE && full && wvec) {
     const int wi = q.w_first + mat;
     const float4* w4 = reinterpret_cast<const float4*>(p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0);
@@ -202,7 +226,7 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&e)[4], float (&a)[3
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const GemmProblem& q, int mat,
                                                int i, int j0, bool full, bool wvec, bool mirror,
-                                               const EpiIn& in, float (&v)[32]) {
+                                               const EpiIn& in, const EpiW& win, float (&v)[32]) {
   if (i >= q.M) return;
   float f = 1.f;
   if (q.scale_mode) {
@@ -240,7 +264,7 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
       float4* w4 = reinterpret_cast<float4*>(w);
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
-        float4 ww = in.w[c4];
+        float4 ww = win.w[c4];
         ww.x = cautious_w(ww.x, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 0])), lr, p.wd, cautious);
         ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), lr, p.wd, cautious);
         ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), lr, p.wd, cautious);
@@ -273,10 +297,10 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
   }
 }
 
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, int NSUB>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
-  using C = TcCfg<PAIR>;
+  using C = TcCfg<PAIR, NSUB>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -331,11 +355,11 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       uint32_t issued_mask = 0, issued_phase_mask = 0;  // per stage: loads issued / their phase
       bool ok = true;
       for (int t = unit; t < p.total_tiles && ok; t += nunits) {
-        const TileCoord tc = decode_tile<C::BM>(p, t);
+        const TileCoord tc = decode_tile<C::BM, C::BN>(p, t);
         const GemmProblem& q = p.prob[tc.prob];
         const int kblocks = (q.K + C::BK - 1) / C::BK;
         const int arow = tc.tm * C::BM + rank * C::A_ROWS;
-        const int brow = tc.tn * TC_BN + rank * C::B_ROWS;
+        const int brow = tc.tn * C::BN + rank * C::SUB_B_ROWS;   // sub-tile n adds n * TC_BN
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!sm100::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
             record_timeout(p.status, abort_flag);
@@ -360,11 +384,16 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
 #pragma unroll
             for (int h = 0; h < C::A_ROWS / 64; ++h) load(sa + h * 8192, &p.tmA[tc.prob], arow + h * 64, k0);
           }
-          if (!q.b_mn) {
-            load(sb, &p.tmB[tc.prob], k0, brow);
-          } else {
 #pragma unroll
-            for (int h = 0; h < C::B_ROWS / 64; ++h) load(sb + h * 8192, &p.tmB[tc.prob], brow + h * 64, k0);
+          for (int n = 0; n < NSUB; ++n) {
+            uint8_t* sbn = sb + n * C::SUB_B_BYTES;
+            const int brow_n = brow + n * TC_BN;
+            if (!q.b_mn) {
+              load(sbn, &p.tmB[tc.prob], k0, brow_n);
+            } else {
+#pragma unroll
+              for (int h = 0; h < C::SUB_B_ROWS / 64; ++h) load(sbn + h * 8192, &p.tmB[tc.prob], brow_n + h * 64, k0);
+            }
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -392,7 +421,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = unit; t < p.total_tiles && ok; t += nunits) {
-        const TileCoord tc = decode_tile<C::BM>(p, t);
+        const TileCoord tc = decode_tile<C::BM, C::BN>(p, t);
         const GemmProblem& q = p.prob[tc.prob];
         const int kblocks = (q.K + C::BK - 1) / C::BK;
         const uint32_t idesc = sm100::make_idesc_bf16(C::BM, TC_BN, q.a_mn, q.b_mn);
@@ -401,7 +430,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           break;
         }
         sm100::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * TC_BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!sm100::mbar_wait(&full_bar[stage], phase, abort_flag)) {
             record_timeout(p.status, abort_flag);
@@ -415,10 +444,15 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             const uint64_t ad = q.a_mn ? sm100::make_sdesc(sa + kk * 2048, 8192, 1024)
                                        : sm100::make_sdesc(sa + kk * 32, 16, 1024);
-            const uint64_t bd = q.b_mn ? sm100::make_sdesc(sb + kk * 2048, 8192, 1024)
-                                       : sm100::make_sdesc(sb + kk * 32, 16, 1024);
-            if (PAIR) sm100::umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
-            else sm100::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+#pragma unroll
+            for (int n = 0; n < NSUB; ++n) {
+              const uint32_t sbn = sb + n * C::SUB_B_BYTES;
+              const uint64_t bd = q.b_mn ? sm100::make_sdesc(sbn + kk * 2048, 8192, 1024)
+                                         : sm100::make_sdesc(sbn + kk * 32, 16, 1024);
+              const uint32_t dn = d_tmem + static_cast<uint32_t>(n * TC_BN);
+              if (PAIR) sm100::umma_bf16_pair(dn, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+              else sm100::umma_bf16(dn, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+            }
           }
           if (PAIR) sm100::umma_commit_pair_both(&empty_bar[stage]);
           else sm100::umma_commit(&empty_bar[stage]);
@@ -430,24 +464,26 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         if (!ok) break;
         if (PAIR) sm100::umma_commit_pair_both(&tfull_bar[acc]);
         else sm100::umma_commit(&tfull_bar[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == C::ACC_BUFS) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
     }
   } else {
     // ----------------------------------------------------------- epilogue
     const int quad = warp & 3;                          // TMEM lane quadrant this warp may read
     const int slice = (warp - 2) / 4;                   // which column slice of the tile
-    constexpr int kChunks = TC_BN / 32 / TC_EPI_SPLIT;  // 32-column chunks per warp
+    constexpr int kChunks = C::BN / 32 / TC_EPI_SPLIT;  // 32-column chunks per warp
     const int row_in_cta = quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = unit; t < p.total_tiles; t += nunits) {
-      const TileCoord tc = decode_tile<C::BM>(p, t);
+      const TileCoord tc = decode_tile<C::BM, C::BN>(p, t);
       const GemmProblem& q = p.prob[tc.prob];
       const int row0 = tc.tm * C::BM + rank * 128;   // first row this CTA holds
       const int i = row0 + row_in_cta;
-      const int jslice = tc.tn * TC_BN + slice * kChunks * 32;
+      const int jslice = tc.tn * C::BN + slice * kChunks * 32;
       if (jslice < q.N) epilogue_prefetch<EPI>(p, q, tc.mat, i, jslice, kChunks * 32);
       bool wvec = true;
       if (EPI == EPI_AXPY_UPDATE && i < q.M) {
@@ -460,25 +496,48 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       }
       sm100::tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                             static_cast<uint32_t>(acc * TC_BN);
-#pragma unroll 1
-      for (int cc = 0; cc < kChunks; ++cc) {
-        const int c = slice * kChunks + cc;
-        const int j0 = tc.tn * TC_BN + c * 32;
-        if (j0 >= q.N) break;  // warp-uniform
-        bool mirror = false;
-        if (q.sym) {
-          const int ib = row0 / 128;        // 128-row block of this CTA's rows
-          const int jb = j0 / 128;          // 128-wide column block
-          if (jb < ib) continue;            // strictly lower block: produced by its mirror
-          mirror = jb > ib;
-        }
+                             static_cast<uint32_t>(acc * C::BN);
+      // Active chunks form one range [c_lo, c_hi): a symmetric tile skips the
+      // chunks of strictly lower 128-blocks (a prefix) and a ragged tile stops
+      // at N.  The bf16 operand of chunk c+1 is loaded while chunk c is
+      // combined and stored, so one L2 round trip is in flight at all times.
+      // The fused update loads X and W (prefetched to L2 above) with each chunk.
+      const int ib = row0 / 128;   // 128-row block of this CTA's rows
+      int c_hi = 0;
+      if (jslice < q.N) c_hi = min(kChunks, (q.N - jslice + 31) / 32);
+      int c_lo = 0;
+      if (q.sym) c_lo = max(0, (128 * ib - jslice) / 32);
+      auto chunk_j0 = [&](int cc) { return jslice + cc * 32; };
+      auto process = [&](int cc, const EpiIn& in) {
+        const int j0 = chunk_j0(cc);
+        const bool mirror = q.sym && (j0 / 128) > ib;
         const bool full = (j0 + 32 <= q.N);
-        EpiIn in;
-        epilogue_load<EPI>(p, q, tc.mat, i, j0, full, wvec, in);
+        EpiW win;
+        epilogue_load_w<EPI>(p, q, tc.mat, i, j0, full, wvec, win);
         float v[32];
-        sm100::tmem_ld32(t_row + static_cast<uint32_t>(c * 32), v);
-        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, mirror, in, v);
+        sm100::tmem_ld32(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), v);
+        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, mirror, in, win, v);
+      };
+      if constexpr (EPI == EPI_AXPY_UPDATE) {
+        // no room for a second operand buffer next to W: one chunk at a time
+#pragma unroll 1
+        for (int cc = c_lo; cc < c_hi; ++cc) {
+          EpiIn in;
+          epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc), chunk_j0(cc) + 32 <= q.N, in);
+          process(cc, in);
+        }
+      } else {
+        EpiIn in0, in1;
+        if (c_lo < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(c_lo), chunk_j0(c_lo) + 32 <= q.N, in0);
+#pragma unroll 1
+        for (int cc = c_lo; cc < c_hi; cc += 2) {
+          if (cc + 1 < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc + 1), chunk_j0(cc + 1) + 32 <= q.N, in1);
+          process(cc, in0);
+          if (cc + 1 < c_hi) {
+            if (cc + 2 < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc + 2), chunk_j0(cc + 2) + 32 <= q.N, in0);
+            process(cc + 1, in1);
+          }
+        }
       }
       sm100::tc_fence_before();
       __syncwarp();
@@ -486,8 +545,10 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         if (PAIR) sm100::mbar_arrive_cluster(sm100::mapa_shared(sm100::smem_u32(&tempty_bar[acc]), 0));
         else sm100::mbar_arrive(&tempty_bar[acc]);
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == C::ACC_BUFS) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -521,14 +582,14 @@ cudaError_t launch_selftest_wait(unsigned int* status, unsigned long long limit_
 }
 
 // ---------------------------------------------------------------- launcher
-int tc_tile_m(bool pair) { return pair ? TcCfg<true>::BM : TcCfg<false>::BM; }
-int tc_tile_n() { return TC_BN; }
-int tc_b_box_rows(bool pair) { return pair ? TcCfg<true>::B_ROWS : TcCfg<false>::B_ROWS; }
+int tc_tile_m(bool pair) { return pair ? TcCfg<true, 1>::BM : TcCfg<false, 1>::BM; }
+int tc_tile_n(bool wide) { return wide ? TcCfg<true, 2>::BN : TC_BN; }
+int tc_b_box_rows(bool pair) { return pair ? TcCfg<true, 1>::SUB_B_ROWS : TcCfg<false, 1>::SUB_B_ROWS; }
 
-template <int EPI, bool PAIR>
+template <int EPI, bool PAIR, int NSUB>
 static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_t s) {
-  using C = TcCfg<PAIR>;
-  auto kern = tc_gemm_kernel<EPI, PAIR>;
+  using C = TcCfg<PAIR, NSUB>;
+  auto kern = tc_gemm_kernel<EPI, PAIR, NSUB>;
   static thread_local int max_units = 0;   // co-resident tile units (CTAs or CTA pairs)
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -561,21 +622,29 @@ static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_
   return cudaGetLastError();
 }
 
-cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, int num_sms, cudaStream_t s) {
+cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, bool wide, int num_sms, cudaStream_t s) {
   if (p.total_tiles <= 0) return cudaSuccess;
-  if (pair) {
+  if (wide && !pair) return cudaErrorInvalidValue;
+  if (wide) {
     switch (epi) {
-      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, true>(p, num_sms, s);
-      case EPI_POLY: return launch_tc_epi<EPI_POLY, true>(p, num_sms, s);
-      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, true>(p, num_sms, s);
-      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, true>(p, num_sms, s);
+      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, true, 2>(p, num_sms, s);
+      case EPI_POLY: return launch_tc_epi<EPI_POLY, true, 2>(p, num_sms, s);
+      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, true, 2>(p, num_sms, s);
+      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, true, 2>(p, num_sms, s);
+    }
+  } else if (pair) {
+    switch (epi) {
+      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, true, 1>(p, num_sms, s);
+      case EPI_POLY: return launch_tc_epi<EPI_POLY, true, 1>(p, num_sms, s);
+      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, true, 1>(p, num_sms, s);
+      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, true, 1>(p, num_sms, s);
     }
   } else {
     switch (epi) {
-      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, false>(p, num_sms, s);
-      case EPI_POLY: return launch_tc_epi<EPI_POLY, false>(p, num_sms, s);
-      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, false>(p, num_sms, s);
-      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, false>(p, num_sms, s);
+      case EPI_GRAM: return launch_tc_epi<EPI_GRAM, false, 1>(p, num_sms, s);
+      case EPI_POLY: return launch_tc_epi<EPI_POLY, false, 1>(p, num_sms, s);
+      case EPI_AXPY: return launch_tc_epi<EPI_AXPY, false, 1>(p, num_sms, s);
+      case EPI_AXPY_UPDATE: return launch_tc_epi<EPI_AXPY_UPDATE, false, 1>(p, num_sms, s);
     }
   }
   return cudaErrorInvalidValue;

@@ -38,9 +38,9 @@ cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, dou
                                     cudaStream_t st);
 cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm, double fin, cudaStream_t st);
 int tc_tile_m(bool pair);
-int tc_tile_n();
+int tc_tile_n(bool wide);
 int tc_b_box_rows(bool pair);
-cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, int num_sms, cudaStream_t s);
+cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, bool wide, int num_sms, cudaStream_t s);
 cudaError_t launch_selftest_wait(unsigned int* status, unsigned long long limit_ns, cudaStream_t s);
 int simt_tile();
 cudaError_t launch_simt_gemm(const SimtGemmParams& p, int epi, int num_sms, cudaStream_t s);
@@ -542,14 +542,26 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
 }
 
 // Build and launch one NS product (epi) for every item of the wave.
+// Products that run on 512-column CTA-pair tiles (bit per EpiKind) unless
+// MUON_TC_NARROW_TILES or single-CTA mode is requested.  Measured at the
+// 8B shapes under the 1 kW cap: the Gram (K = n, up to 14336) takes the same
+// SM cycles on either tile and 8% less time on the wide one, which draws less
+// power per cycle (25% fewer operand bytes from L2 per FLOP); A*A and B*X
+// (K = m = 4096) take ~10-25% more cycles on it, because the drain of the
+// single 512-column accumulator is no longer hidden behind the next tile.
+#ifndef MUON_TC_WIDE_EPIS
+#define MUON_TC_WIDE_EPIS 0x1
+#endif
+
 muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
   const StepArgs& a = C.a;
   const bool f32 = (a.flags & MUON_FP32_DEBUG) != 0;
   const float ca = a.coeffs[3 * k], cb = a.coeffs[3 * k + 1], cc = a.coeffs[3 * k + 2];
   const float* scales = reinterpret_cast<const float*>(a.ws + w.scales_off);
   const bool pair = (a.flags & MUON_TC_SINGLE_CTA) == 0;
+  const bool wide = pair && !f32 && (a.flags & MUON_TC_NARROW_TILES) == 0 && ((MUON_TC_WIDE_EPIS >> epi) & 1);
   const int BM = f32 ? simt_tile() : tc_tile_m(pair);
-  const int BN = f32 ? simt_tile() : tc_tile_n();
+  const int BN = f32 ? simt_tile() : tc_tile_n(wide);
   const int b_rows = tc_b_box_rows(pair);
 
   static thread_local TcGemmParams TP;
@@ -581,7 +593,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       TP.sched = a.sched;
       const int kind = epi == EPI_GRAM ? K_GRAM : epi == EPI_POLY ? K_POLY
                      : epi == EPI_AXPY ? K_AXPY : K_AXPY_UPDATE;
-      e = timed_launch(kind, a.stream, [&] { return launch_tc_gemm(TP, epi, pair, C.dev.sms, a.stream); });
+      e = timed_launch(kind, a.stream, [&] { return launch_tc_gemm(TP, epi, pair, wide, C.dev.sms, a.stream); });
     }
     if (e != cudaSuccess) return cuda_fail(e, "NS GEMM launch");
     reset();
@@ -740,7 +752,7 @@ muon_status validate_common(const muon_group* groups, int n_groups, int ns_steps
   muon_status st = validate_groups(groups, n_groups);
   if (st != MUON_OK) return st;
   if (flags & ~(MUON_NESTEROV | MUON_CAUTIOUS_WD | MUON_FP32_DEBUG | MUON_UNFUSED_UPDATE |
-                MUON_TC_SINGLE_CTA | MUON_NORMUON | MUON_ROW_EQUILIBRATE))
+                MUON_TC_SINGLE_CTA | MUON_NORMUON | MUON_ROW_EQUILIBRATE | MUON_TC_NARROW_TILES))
     return fail(MUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (ns_steps < 0 || ns_steps > kMaxNsSteps)
     return fail(MUON_ERR_INVALID_ARG, "ns_steps %d outside [0, %d]", ns_steps, kMaxNsSteps);
@@ -827,7 +839,7 @@ muon_status muon_orthogonalize(const void* const* inputs, float* const* outputs,
                                int n_groups, int ns_steps, const float* coeffs, uint32_t flags,
                                void* workspace, size_t workspace_bytes, muon_stream_t stream) {
   g_err[0] = '\0';
-  flags &= (MUON_FP32_DEBUG | MUON_TC_SINGLE_CTA);
+  flags &= (MUON_FP32_DEBUG | MUON_TC_SINGLE_CTA | MUON_TC_NARROW_TILES);
   muon_status st = validate_common(groups, n_groups, ns_steps, coeffs, flags, workspace, workspace_bytes);
   if (st != MUON_OK) return st;
   if ((st = validate_ptrs("inputs", inputs, groups, n_groups)) != MUON_OK) return st;
