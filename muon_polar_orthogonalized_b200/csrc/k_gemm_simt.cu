@@ -1,7 +1,7 @@
 // k_gemm_simt.cu -- fp32-operand Newton-Schulz products for the debug mode.
 //
-// Same three products and epilogues as the tensor-core kernels (Gram, b*A +
-// c*A*A, a*X + B*X, and the fused cautious update), but with fp32 operands and
+// Same three products and epilogues as the tensor-core kernels (Gram,
+// B' = a*I + b*A + c*A*A, B'*X, and the fused cautious update), but with fp32 operands and
 // fp32 FMA accumulation on the CUDA cores, so the whole iteration can be
 // checked to ~1e-6 against the fp64 oracle.  Correctness scaffold, not a fast
 // path: 64x64 tiles, 16x16 threads with 4x4 outputs each, full (not
@@ -83,10 +83,9 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const __grid_constant__ 
           val *= f;
         } else if (EPI == EPI_POLY) {
           const float a = static_cast<const float*>(q.ein)[mat * q.ein_bs + eo];
-          val = fmaf(q.cb, a, q.cc * val);
+          val = fmaf(q.cb, a, q.cc * val) + (i == j ? q.ca : 0.f);
         } else {
-          const float x = static_cast<const float*>(q.ein)[mat * q.ein_bs + eo];
-          val = f * fmaf(q.ca, x, val);
+          val *= f;
         }
         if (EPI == EPI_AXPY_UPDATE) {
           const int wi = q.w_first + mat;

@@ -6,11 +6,14 @@
 //   gram  A = s^2 X X^T          symmetric: only tiles touching the upper
 //                                triangle run; off-diagonal blocks are also
 //                                stored transposed (mirrored)
-//   poly  B = b A + c A A        symmetric likewise; A A = A A^T since A is
+//   poly  B' = a I + b A + c A A symmetric likewise; A A = A A^T since A is
 //                                symmetric, so both operands are rows of A;
-//                                the epilogue reads the A tile for b*A
-//   axpy  X' = s (a X + B X)     wide matrices; tall ones (iterated as X^T)
-//                                compute X' = s (a X + X B) in parameter layout
+//                                the epilogue reads the A tile for b*A and
+//                                adds a on the diagonal
+//   axpy  X' = s B' X            = s (a X + B X); wide matrices; tall ones
+//                                (iterated as X^T) compute X' = s X B' in
+//                                parameter layout.  The epilogue only scales
+//                                and converts: a X rides in the product
 //   axpy_update                  last iteration: U = bf16(X') feeds the
 //                                cautious-decay update of W directly
 // s is the Frobenius scale 1/(||m~||+1e-7), applied on the first iteration
@@ -21,8 +24,9 @@
 // in, fp32 accumulate) issued by one thread into TMEM, and eight epilogue
 // warps that drain TMEM with tcgen05.ld.  Tiles: 256x256 on a CTA pair with
 // two 256-column accumulators (one tile's epilogue overlaps the next tile's
-// MMAs) and a 6-stage ring; the Gram products use 256x512 pair tiles (two
-// N=256 MMAs per K step into one 512-column accumulator, 4-stage ring).
+// MMAs) and a 6-stage ring; the Gram and plain B'X products use 256x512 pair
+// tiles (two N=256 MMAs per K step into one 512-column accumulator, 4-stage
+// ring).
 // Single-CTA mode: 128x256 tiles, 4-stage ring.
 //   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
 //   warps 2-9: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31; two warps
@@ -165,11 +169,13 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
 template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const GemmProblem& q,
                                                   int mat, int i, int jt, int width) {
-  if (EPI == EPI_GRAM || i >= q.M) return;
+  if (EPI == EPI_GRAM || EPI == EPI_AXPY || i >= q.M) return;
   const int ncols = min(width, q.N - jt);  // jt < N
-  const char* ein = reinterpret_cast<const char*>(
-      static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
-  for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
+  if (EPI == EPI_POLY) {
+    const char* ein = reinterpret_cast<const char*>(
+        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
+    for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
+  }
   if (EPI == EPI_AXPY_UPDATE) {
     const int wi = q.w_first + mat;
     const char* w = reinterpret_cast<const char*>(p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + jt);
@@ -178,18 +184,18 @@ __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const G
 }
 
 struct EpiIn {
-  uint4 e[4];     // 32 bf16 of the epilogue operand (A or X)
+  uint4 e[4];     // 32 bf16 of the epilogue operand A (A*A products)
 };
 struct EpiW {
   float4 w[8];    // 32 fp32 parameters (fused update)
 };
 
-// The bf16 operand (A or X) of one chunk.
+// The bf16 operand A of one chunk (A*A products only).
 template <int EPI>
 __device__ __forceinline__ void epilogue_load(const TcGemmParams& p, const GemmProblem& q, int mat,
                                               int i, int j0, bool full, EpiIn& in) {
   if (i >= q.M) return;
-  if (EPI != EPI_GRAM && full) {
+  if (EPI == EPI_POLY && full) {
     const uint4* e4 = reinterpret_cast<const uint4*>(
         static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0);
 #pragma unroll
@@ -233,10 +239,7 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
     const float s = p.scales[q.scale_base + mat];
     f = (q.scale_mode == 1) ? s * s : s;
   }
-  if constexpr (EPI == EPI_GRAM) {
-#pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] *= f;
-  } else {
+  if constexpr (EPI == EPI_POLY) {
     float a[32];
     if (full) {
       unpack_bf16x32(in.e, a);
@@ -246,13 +249,12 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
 #pragma unroll
       for (int c = 0; c < 32; ++c) a[c] = (j0 + c < q.N) ? __bfloat162float(ein[c]) : 0.f;
     }
-    if constexpr (EPI == EPI_POLY) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]);
-    } else {
+    for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]) + ((j0 + c == i) ? q.ca : 0.f);
+  } else {
+    // Gram: s^2 on the first iteration; axpy: s on the first iteration
 #pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] = f * fmaf(q.ca, a[c], v[c]);
-    }
+    for (int c = 0; c < 32; ++c) v[c] *= f;
   }
 
   if constexpr (EPI == EPI_AXPY_UPDATE) {

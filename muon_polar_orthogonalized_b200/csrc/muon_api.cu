@@ -543,14 +543,16 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
 
 // Build and launch one NS product (epi) for every item of the wave.
 // Products that run on 512-column CTA-pair tiles (bit per EpiKind) unless
-// MUON_TC_NARROW_TILES or single-CTA mode is requested.  Measured at the
-// 8B shapes under the 1 kW cap: the Gram (K = n, up to 14336) takes the same
-// SM cycles on either tile and 8% less time on the wide one, which draws less
-// power per cycle (25% fewer operand bytes from L2 per FLOP); A*A and B*X
-// (K = m = 4096) take ~10-25% more cycles on it, because the drain of the
-// single 512-column accumulator is no longer hidden behind the next tile.
+// MUON_TC_NARROW_TILES or single-CTA mode is requested.  The wide tile reads
+// 25% fewer operand bytes from L2 per FLOP, so at the same SM cycles it draws
+// less power and runs at a higher clock under the 1 kW cap; its single
+// 512-column accumulator is drained without overlap.  Measured on 8 layers
+// of the 8B shapes: the Gram and B'X (whose epilogue only scales and stores)
+// take the same cycles on either tile and less time on the wide one; A*A
+// (epilogue reads A) and the fused-update B'X (reads and writes W) take
+// 25-35% more time on it.
 #ifndef MUON_TC_WIDE_EPIS
-#define MUON_TC_WIDE_EPIS 0x1
+#define MUON_TC_WIDE_EPIS 0x5
 #endif
 
 muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
@@ -638,21 +640,21 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       P.a_bs = P.b_bs = xs_el;
       P.a_ld = P.b_ld = q.ldm;
       P.sym = 1;
-      P.out = bbuf; P.out_bs = bs_el; P.out_ld = q.ldm;
+      P.out = bbuf; P.out_bs = bs_el; P.out_ld = q.ldm;   // B' = a I + b A + c A A
       P.ein = xoth; P.ein_bs = xs_el; P.ein_ld = q.ldm;
     } else {
       P.M = q.r;
       P.N = q.c;
       P.K = q.m;
-      if (!q.tall) {  // X' = a X + B X : Aop = B (K-major), Bop = X (MN-major)
+      // a X + B X = B' X with B' = a I + B from the A*A epilogue
+      if (!q.tall) {  // X' = B' X : Aop = B' (K-major), Bop = X (MN-major)
         P.a = bbuf; P.a_bs = bs_el; P.a_ld = q.ldm; P.a_mn = 0;
         P.b = xcur; P.b_bs = xs_el; P.b_ld = q.ldc; P.b_mn = 1;
-      } else {        // X' = a X + X B : Aop = X (K-major), Bop = B (K-major, symmetric)
+      } else {        // X' = X B' : Aop = X (K-major), Bop = B' (K-major, symmetric)
         P.a = xcur; P.a_bs = xs_el; P.a_ld = q.ldc; P.a_mn = 0;
         P.b = bbuf; P.b_bs = bs_el; P.b_ld = q.ldm; P.b_mn = 0;
       }
       P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldc;
-      P.ein = xcur; P.ein_bs = xs_el; P.ein_ld = q.ldc;
       P.scale_mode = (k == 0) ? 2 : 0;
     }
     if (f32) P.sym = 0;  // the fp32 scaffold computes full outputs

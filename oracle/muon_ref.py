@@ -307,7 +307,7 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 
 
 def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: int = 5,
-                                eps: float = NS_EPS) -> np.ndarray:
+                                eps: float = NS_EPS, fold_a: bool = False) -> np.ndarray:
     """The iteration with bf16 rounding wherever a bf16 matrix is stored.
 
     [MAC] casts to bf16 before iterating and keeps X, A, B in bf16.  Storage
@@ -315,6 +315,10 @@ def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: in
     scalar into the first Gram product and the first X update, A, B and each
     new X; products are exact (fp64) between roundings.  Used to tell bf16
     precision apart from kernel bugs; the gate is always the fp64 oracle.
+
+    fold_a: the stored B holds a on its diagonal, B' = bf16(a I + b A + c A A),
+    and X' = bf16(B' X): the same algebra, a*X + B X = (a I + B) X, with the
+    rounding moved, as a kernel that folds a into B stores it.
     """
     g = np.asarray(g, dtype=np.float64)
     s = 1.0 / (np.sqrt(np.sum(g * g)) + eps)
@@ -325,8 +329,12 @@ def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: in
     for k, (a, b, c) in enumerate(_coeff_list(coeffs, steps)):
         sk = s if k == 0 else 1.0
         A = round_bf16(sk * sk * (x @ x.T))
-        B = round_bf16(b * A + c * (A @ A))
-        x = round_bf16(sk * (a * x + B @ x))
+        if fold_a:
+            B = round_bf16(a * np.eye(A.shape[0]) + b * A + c * (A @ A))
+            x = round_bf16(sk * (B @ x))
+        else:
+            B = round_bf16(b * A + c * (A @ A))
+            x = round_bf16(sk * (a * x + B @ x))
     if steps == 0:
         x = round_bf16(s * x)
     if transposed:
