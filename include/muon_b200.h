@@ -134,6 +134,30 @@ muon_status muon_step(float* const* params, const void* const* grads, float* con
                       muon_stream_t stream);
 
 /*
+ * muon_step that also writes every updated parameter matrix into
+ * n_replicas further copies ("3.9 Optimizers: SGD, Adam, Adafactor, Lion,
+ * Muon & Shampoo", Wiring the hybrid recipe: a distributed Muon steps each
+ * matrix on one rank, which must then hand the result to every
+ * data-parallel rank).  replicas: host array of n_replicas host arrays of
+ * device pointers, in the order of `params`: replicas[r][i] is copy r of
+ * params[i] (same shape, fp32, 16-byte aligned).  The copies may live in
+ * another GPU's memory that this device can address (peer access or a
+ * mapped IPC / symmetric-memory allocation): on the default path the last
+ * Newton-Schulz product's epilogue stores each updated W tile to W and to
+ * every copy with plain stores, so the exchange over NVLink overlaps the
+ * GEMM tile by tile; other paths (MUON_UNFUSED_UPDATE, MUON_NORMUON,
+ * MUON_FP32_DEBUG, ns_steps == 0) copy W after the update.  No multicast.
+ * The copies hold the new values once `stream` passes this call; a reader
+ * on another device must order itself after it (an event or a collective).
+ * n_replicas in [0, 7]; 0 is muon_step.  Other arguments as muon_step.
+ */
+muon_status muon_step_replicated(float* const* params, const void* const* grads,
+                                 float* const* momentum, const muon_group* groups, int n_groups,
+                                 float lr, float beta, float wd, int ns_steps, const float* coeffs,
+                                 uint32_t flags, void* workspace, size_t workspace_bytes,
+                                 float* const* const* replicas, int n_replicas, muon_stream_t stream);
+
+/*
  * muon_step without a caller workspace, for callers that cannot allocate
  * device memory (no counterpart on the optimizer pages: it is a deployment
  * aid).  Programs whose device-memory budget is fixed at start-up by another

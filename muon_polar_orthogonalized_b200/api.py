@@ -78,6 +78,25 @@ def muon_step(params, grads, momentum, groups: Sequence, lr: float, beta: float,
     check(st, "muon_step")
 
 
+def muon_step_replicated(params, grads, momentum, groups: Sequence, lr: float, beta: float, wd: float,
+                         ns_steps: int, coeffs, flags: int, workspace, replicas: Sequence[Sequence],
+                         workspace_bytes: Optional[int] = None, stream=None) -> None:
+    """muon_step that also writes each updated matrix into every replica list
+    (replicas[r][i] is copy r of params[i]; tensors or raw device pointers,
+    possibly in peer GPUs' memory)."""
+    g = make_groups(groups)
+    ca = _coeff_array(coeffs, ns_steps)
+    wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    ws = workspace if isinstance(workspace, int) else workspace.data_ptr()
+    rows = [_ptrs(rep) for rep in replicas]
+    table = (ctypes.POINTER(c_void_p) * max(len(rows), 1))(
+        *[ctypes.cast(r, ctypes.POINTER(c_void_p)) for r in rows])
+    st = N.lib().muon_step_replicated(_ptrs(params), _ptrs(grads), _ptrs(momentum), g, len(groups),
+                                      float(lr), float(beta), float(wd), int(ns_steps), ca, int(flags),
+                                      c_void_p(ws), wsb, table, len(rows), c_void_p(_stream_handle(stream)))
+    check(st, "muon_step_replicated")
+
+
 def muon_step_scheduled(params, grads, momentum, groups: Sequence, lr: float, beta: float, wd: float,
                         ns_steps: int, coeffs, flags: int, workspace, schedule_state,
                         workspace_bytes: Optional[int] = None, stream=None) -> None:

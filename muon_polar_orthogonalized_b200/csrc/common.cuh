@@ -16,6 +16,7 @@ constexpr int kMaxUpdMats = 256;         // fused-update pointer table
 constexpr int kMaxAdamTensors = 128;     // AdamW tensors per launch
 constexpr int kWsHeaderBytes = 4096;     // workspace header: status word + reserve
 constexpr int kMaxNsSteps = 16;
+constexpr int kMaxReplicas = 7;          // copies of W written with the update (the other ranks of a node)
 
 // Status word bits recorded by device code (OR-ed into workspace word 0).
 constexpr uint32_t kDevTimeout = 1u;
@@ -59,6 +60,8 @@ struct alignas(64) TcGemmParams {
   GemmProblem prob[kMaxProblems];
   float* wptr[kMaxUpdMats];
   int wcols[kMaxUpdMats];   // param row pitch (= cols)
+  float* rptr[kMaxReplicas][kMaxUpdMats];   // fused update: copies of each W written with it
+  int nrep;                 // copies in rptr (0: none)
   int nprob;
   int total_tiles;
   const float* scales;
@@ -67,6 +70,7 @@ struct alignas(64) TcGemmParams {
   int cautious;
   const DevSched* sched;
 };
+static_assert(sizeof(TcGemmParams) <= 32764, "kernel parameter limit");
 
 struct SimtGemmParams {
   GemmProblem prob[kMaxProblems];

@@ -66,4 +66,18 @@ struct AdamParams {
   const DevSched* sched;  // nullptr, or the device schedule (lr multiplier, step)
 };
 
+// ------------------------------------------------------------- replicate
+// Copies of parameter matrices: dst[r][i] <- src[i] for r < nrep, for the
+// update paths that do not write the copies themselves.
+constexpr int kReplMats = 64;
+struct ReplParams {
+  const float* src[kReplMats];
+  float* dst[kMaxReplicas][kReplMats];
+  long long numel[kReplMats];
+  int blk_begin[kReplMats];   // first work chunk of matrix i
+  int nmats;
+  int nrep;
+  int total_blocks;
+};
+
 }  // namespace muon

@@ -761,6 +761,44 @@ __global__ void schedule_advance_kernel(DevSched* s, long long total, double war
   s->lr_mult = static_cast<float>(m);
 }
 
+// ------------------------------------------------------------- replicate
+// dst[r][i] <- src[i]: persistent, 4096-element chunks, 16-byte accesses
+// (every pointer is 16-byte aligned; a matrix's scalar tail is copied last).
+constexpr int kReplChunk = kEltThreads * 4 * 4;
+
+__global__ void __launch_bounds__(kEltThreads)
+replicate_kernel(const __grid_constant__ ReplParams p) {
+  for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
+    int mi = 0;
+    while (mi + 1 < p.nmats && p.blk_begin[mi + 1] <= blk) ++mi;
+    const long long e0 = static_cast<long long>(blk - p.blk_begin[mi]) * kReplChunk;
+    const long long n = p.numel[mi];
+    const long long nvec = n & ~3ll;
+    const float* src = p.src[mi];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
+      if (e < nvec) {
+        const float4 v = *reinterpret_cast<const float4*>(src + e);
+        for (int r = 0; r < p.nrep; ++r) *reinterpret_cast<float4*>(p.dst[r][mi] + e) = v;
+      }
+    }
+    if (e0 + kReplChunk >= n && threadIdx.x < n - nvec) {   // the matrix's last chunk: scalar tail
+      const long long e = nvec + threadIdx.x;
+      for (int r = 0; r < p.nrep; ++r) p.dst[r][mi][e] = src[e];
+    }
+  }
+}
+
+int repl_chunk() { return kReplChunk; }
+
+cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s) {
+  if (p.total_blocks <= 0 || p.nrep <= 0) return cudaSuccess;
+  const long long g = static_cast<long long>(sms) * 4;
+  replicate_kernel<<<static_cast<int>(g < p.total_blocks ? g : p.total_blocks), kEltThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
                                     cudaStream_t st) {
   schedule_advance_kernel<<<1, 32, 0, st>>>(s, total, wu, wd, fin);

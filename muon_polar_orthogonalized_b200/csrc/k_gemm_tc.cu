@@ -258,12 +258,16 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
   }
 
   if constexpr (EPI == EPI_AXPY_UPDATE) {
+    // W and each of its copies (rptr: the other ranks' replicas, possibly in
+    // peer GPUs' memory) receive the same new values, with plain stores
     const int wi = q.w_first + mat;
-    float* w = p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0;
+    const long long roff = static_cast<long long>(i) * p.wcols[wi] + j0;
+    float* w = p.wptr[wi] + roff;
     const bool cautious = p.cautious != 0;
     const float lr = p.sched ? q.lr * p.sched->lr_mult : q.lr;
     if (full && wvec) {
       float4* w4 = reinterpret_cast<float4*>(w);
+      float4 nw[8];
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
         float4 ww = win.w[c4];
@@ -271,13 +275,22 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
         ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), lr, p.wd, cautious);
         ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), lr, p.wd, cautious);
         ww.w = cautious_w(ww.w, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 3])), lr, p.wd, cautious);
+        nw[c4] = ww;
         w4[c4] = ww;
+      }
+      for (int r = 0; r < p.nrep; ++r) {
+        float4* d4 = reinterpret_cast<float4*>(p.rptr[r][wi] + roff);
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) d4[c4] = nw[c4];
       }
     } else {
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        if (j0 + c < q.N)
-          w[c] = cautious_w(w[c], __bfloat162float(__float2bfloat16_rn(v[c])), lr, p.wd, cautious);
+        if (j0 + c < q.N) {
+          const float nv = cautious_w(w[c], __bfloat162float(__float2bfloat16_rn(v[c])), lr, p.wd, cautious);
+          w[c] = nv;
+          for (int r = 0; r < p.nrep; ++r) p.rptr[r][wi][roff + c] = nv;
+        }
     }
   } else {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(q.out) + mat * q.out_bs;

@@ -34,6 +34,8 @@ cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
 cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
+cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s);
+int repl_chunk();
 cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
                                     cudaStream_t st);
 cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm, double fin, cudaStream_t st);
@@ -368,6 +370,8 @@ struct StepArgs {
   cudaStream_t stream;
   bool orth;  // orthogonaliser mode
   const DevSched* sched;  // device schedule (lr multiplier), or nullptr
+  float* const* const* replicas = nullptr;  // [nrep][pointer index]: copies of each param
+  int nrep = 0;
 };
 
 // MuonEq row equilibration applies to muon_step only (the orthogonaliser has
@@ -593,6 +597,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       TP.wd = a.wd;
       TP.cautious = (a.flags & MUON_CAUTIOUS_WD) ? 1 : 0;
       TP.sched = a.sched;
+      TP.nrep = (epi == EPI_AXPY_UPDATE) ? a.nrep : 0;
       const int kind = epi == EPI_GRAM ? K_GRAM : epi == EPI_POLY ? K_POLY
                      : epi == EPI_AXPY ? K_AXPY : K_AXPY_UPDATE;
       e = timed_launch(kind, a.stream, [&] { return launch_tc_gemm(TP, epi, pair, wide, C.dev.sms, a.stream); });
@@ -706,12 +711,47 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
         } else {
           TP.wptr[nw + j] = a.params[pi];
           TP.wcols[nw + j] = q.c;
+          for (int r = 0; r < a.nrep; ++r) TP.rptr[r][nw + j] = a.replicas[r][pi];
         }
       }
     }
     nw += it.count;
     tiles += static_cast<int>(add);
     nprob += 1;
+  }
+  return flush();
+}
+
+// dst[r][i] <- params[i] for every matrix of the wave (update paths that do
+// not write the copies in their own epilogue).
+muon_status run_replicate(const Ctx& C, const Wave& w) {
+  const StepArgs& a = C.a;
+  ReplParams R;
+  std::memset(&R, 0, sizeof(R));
+  R.nrep = a.nrep;
+  auto flush = [&]() -> muon_status {
+    if (R.nmats == 0) return MUON_OK;
+    cudaError_t e = launch_replicate(R, C.dev.sms, a.stream);
+    if (e != cudaSuccess) return cuda_fail(e, "replicate launch");
+    R.nmats = R.total_blocks = 0;
+    return MUON_OK;
+  };
+  for (const auto& it : w.items) {
+    const muon_group& g = a.groups[it.g];
+    for (int j = 0; j < it.count; ++j) {
+      if (R.nmats == kReplMats) {
+        muon_status st = flush();
+        if (st != MUON_OK) return st;
+      }
+      const int pi = g.first + it.first + j;
+      const long long numel = static_cast<long long>(g.rows) * g.cols;
+      R.src[R.nmats] = a.params[pi];
+      for (int r = 0; r < a.nrep; ++r) R.dst[r][R.nmats] = a.replicas[r][pi];
+      R.numel[R.nmats] = numel;
+      R.blk_begin[R.nmats] = R.total_blocks;
+      R.total_blocks += static_cast<int>((numel + repl_chunk() - 1) / repl_chunk());
+      R.nmats += 1;
+    }
   }
   return flush();
 }
@@ -745,6 +785,9 @@ muon_status run_step(const StepArgs& a, size_t ws_bytes) {
     } else if (!fused) {
       if ((st = run_elementwise(C, w, normuon ? 4 : 2)) != MUON_OK) return st;
     }
+    // the tensor-core fused update writes the copies itself
+    if (a.nrep > 0 && !(fused && !f32))
+      if ((st = run_replicate(C, w)) != MUON_OK) return st;
   }
   return MUON_OK;
 }
@@ -801,7 +844,8 @@ static muon_status muon_step_impl(float* const* params, const void* const* grads
                                   float* const* momentum, const muon_group* groups, int n_groups,
                                   float lr, float beta, float wd, int ns_steps, const float* coeffs,
                                   uint32_t flags, void* workspace, size_t workspace_bytes,
-                                  muon_stream_t stream, const DevSched* sched) {
+                                  muon_stream_t stream, const DevSched* sched,
+                                  float* const* const* replicas = nullptr, int n_replicas = 0) {
   g_err[0] = '\0';
   muon_status st = validate_common(groups, n_groups, ns_steps, coeffs, flags, workspace, workspace_bytes);
   if (st != MUON_OK) return st;
@@ -810,9 +854,28 @@ static muon_status muon_step_impl(float* const* params, const void* const* grads
   if ((st = validate_ptrs("params", reinterpret_cast<const void* const*>(params), groups, n_groups)) != MUON_OK) return st;
   if ((st = validate_ptrs("grads", grads, groups, n_groups)) != MUON_OK) return st;
   if ((st = validate_ptrs("momentum", reinterpret_cast<const void* const*>(momentum), groups, n_groups)) != MUON_OK) return st;
+  if (n_replicas < 0 || n_replicas > kMaxReplicas)
+    return fail(MUON_ERR_INVALID_ARG, "n_replicas %d outside [0, %d]", n_replicas, kMaxReplicas);
+  if (n_replicas > 0 && !replicas) return fail(MUON_ERR_INVALID_ARG, "replicas is NULL");
+  for (int r = 0; r < n_replicas; ++r) {
+    char what[32];
+    snprintf(what, sizeof(what), "replicas[%d]", r);
+    if ((st = validate_ptrs(what, reinterpret_cast<const void* const*>(replicas[r]), groups, n_groups)) != MUON_OK)
+      return st;
+  }
   StepArgs a{params, grads, momentum, nullptr, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
-             flags, static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream), false, sched};
+             flags, static_cast<char*>(workspace), reinterpret_cast<cudaStream_t>(stream), false, sched,
+             replicas, n_replicas};
   return run_step(a, workspace_bytes);
+}
+
+muon_status muon_step_replicated(float* const* params, const void* const* grads, float* const* momentum,
+                                 const muon_group* groups, int n_groups, float lr, float beta, float wd,
+                                 int ns_steps, const float* coeffs, uint32_t flags, void* workspace,
+                                 size_t workspace_bytes, float* const* const* replicas, int n_replicas,
+                                 muon_stream_t stream) {
+  return muon_step_impl(params, grads, momentum, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
+                        flags, workspace, workspace_bytes, stream, nullptr, replicas, n_replicas);
 }
 
 muon_status muon_step(float* const* params, const void* const* grads, float* const* momentum,

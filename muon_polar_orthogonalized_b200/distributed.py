@@ -13,6 +13,12 @@ across data-parallel ranks).  Here every hidden matrix has one owner rank:
      only on the owner (state sharded);
   3. each owner broadcasts its updated matrices to every rank.
 
+With peer_params (every other rank's parameter tensors, addressable from
+this GPU through peer access or symmetric memory), step 3 becomes part of
+step 2: the owner's last Newton-Schulz epilogue stores each updated tile into
+every rank's replica over NVLink (muon_step_replicated), and one barrier
+orders the ranks after all owners' writes.
+
 AdamW parameters have their gradients all-reduced (mean) and are stepped on
 every rank.  Owners are chosen by longest-processing-time over the executed
 Newton-Schulz FLOPs of each matrix (3 m^2 n + m^3 for m <= n), so ranks get
@@ -52,15 +58,20 @@ class DistributedMuonAdamW:
     """Data-parallel MuonAdamW with owner-sharded Muon matrices.
 
     muon_params / adamw_groups as for MuonAdamW (identical on every rank).
-    step_fn(params, grads, momentum) -> None updates the owned params and
-    momentum in place (default: a MuonAdamW over the owned matrices, built
-    with the keyword arguments given here).  The process group must be
-    initialised unless world size is 1.
+    step_fn(params, grads, momentum[, replicas]) -> None updates the owned
+    params and momentum in place, and each replica list's tensors too when
+    given (default: a MuonAdamW over the owned matrices, built with the
+    keyword arguments given here).  peer_params: optional {rank: that rank's
+    muon_params tensors in the same order} for every other rank, writable
+    from this process (peer GPU memory); owners then write every rank's copy
+    in their update and the broadcasts are skipped.  The process group must
+    be initialised unless world size is 1.
     """
 
     def __init__(self, muon_params: Sequence[torch.Tensor], adamw_groups: Sequence[Dict] = (),
                  process_group=None, step_fn: Optional[Callable] = None,
-                 adamw_fn: Optional[Callable] = None, **muon_kwargs):
+                 adamw_fn: Optional[Callable] = None,
+                 peer_params: Optional[Dict[int, Sequence[torch.Tensor]]] = None, **muon_kwargs):
         self.group = process_group
         self.world = dist.get_world_size(process_group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(process_group) if dist.is_initialized() else 0
@@ -77,6 +88,16 @@ class DistributedMuonAdamW:
                                     **muon_kwargs)
         self.momentum = {i: torch.zeros_like(self.muon_params[i]) for i in self.owned} \
             if step_fn is not None else None
+        self.peer_params = None
+        if peer_params is not None:
+            others = sorted(r for r in range(self.world) if r != self.rank)
+            if sorted(peer_params) != others:
+                raise ValueError(f"peer_params must hold exactly the other ranks {others}")
+            for r in others:
+                if len(peer_params[r]) != len(self.muon_params) or any(
+                        tuple(a.shape) != tuple(b.shape) for a, b in zip(peer_params[r], self.muon_params)):
+                    raise ValueError(f"peer_params[{r}] does not match muon_params")
+            self.peer_params = {r: list(peer_params[r]) for r in others}
 
     def _bucket(self, tensors: List[torch.Tensor]) -> torch.Tensor:
         return torch.cat([t.reshape(-1) for t in tensors]) if tensors else torch.empty(0)
@@ -109,16 +130,29 @@ class DistributedMuonAdamW:
             dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=self.group)
             flat.div_(self.world)
             self._unbucket(flat, [p.grad for p in adam_params])
-        # 2. owners step their matrices (and every rank its AdamW params)
+        # 2. owners step their matrices (and every rank its AdamW params); with
+        #    peer_params they write every other rank's copy as well
+        replicas = None
+        if self.peer_params is not None:
+            replicas = [[self.peer_params[r][i] for i in self.owned] for r in sorted(self.peer_params)]
         if self.step_fn is not None:
             own = self.owned
             if own:
-                self.step_fn([self.muon_params[i] for i in own], [self.muon_params[i].grad for i in own],
-                             [self.momentum[i] for i in own])
+                args = ([self.muon_params[i] for i in own], [self.muon_params[i].grad for i in own],
+                        [self.momentum[i] for i in own])
+                if replicas is not None:
+                    self.step_fn(*args, replicas)
+                else:
+                    self.step_fn(*args)
             if self.adamw_fn is not None and adam_params:
                 self.adamw_fn(self.adamw_groups)
         else:
-            self._local.step()
+            self._local.step(replicas=replicas)
+        if self.peer_params is not None:
+            # 3. every owner's writes into this rank's replica are done
+            if self.world > 1:
+                dist.barrier(group=self.group)
+            return
         # 3. owners broadcast their updated matrices
         if self.world > 1:
             for r in range(self.world):

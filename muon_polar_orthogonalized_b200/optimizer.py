@@ -40,17 +40,20 @@ class MuonAdamW:
                       | (N.MUON_NORMUON if normuon else 0)
                       | (N.MUON_ROW_EQUILIBRATE if row_equilibrate else 0))
         # shape groups: matrices with equal (rows, cols) are contiguous in the pointer arrays
-        order: Dict[tuple, List[torch.Tensor]] = {}
-        for p in muon_params:
+        muon_params = list(muon_params)
+        order: Dict[tuple, List[int]] = {}
+        for k, p in enumerate(muon_params):
             if p.dim() != 2 or p.dtype != torch.float32 or not p.is_cuda or not p.is_contiguous():
                 raise ValueError("Muon parameters must be contiguous fp32 2-D CUDA tensors")
-            order.setdefault(tuple(p.shape), []).append(p)
+            order.setdefault(tuple(p.shape), []).append(k)
         self.muon_params: List[torch.Tensor] = []
+        self._order: List[int] = []   # internal position -> position in muon_params as given
         self._shapes = []
-        for (r, c), ps in order.items():
-            self._shapes.append((r, c, len(ps), len(self.muon_params),
+        for (r, c), ks in order.items():
+            self._shapes.append((r, c, len(ks), len(self.muon_params),
                                  float(lr_scale_fn(r, c)) if lr_scale_fn else 1.0))
-            self.muon_params.extend(ps)
+            self.muon_params.extend(muon_params[k] for k in ks)
+            self._order.extend(ks)
         self.momentum = [torch.zeros_like(p) for p in self.muon_params]
         self.adamw_groups = []
         for g in adamw_groups:
@@ -71,7 +74,11 @@ class MuonAdamW:
         return [(r, c, n, first, dt, ls) for (r, c, n, first, ls) in self._shapes]
 
     @torch.no_grad()
-    def step(self, stream=None) -> None:
+    def step(self, stream=None, replicas: Optional[Sequence[Sequence[torch.Tensor]]] = None) -> None:
+        """One MuonAdamW step.  replicas: optional copies of the Muon
+        parameters (replicas[r][k] is copy r of the k-th tensor given at
+        construction, e.g. another data-parallel rank's replica in peer
+        memory); each receives the updated values (muon_step_replicated)."""
         self.step_count += 1
         if self.muon_params:
             grads = [p.grad for p in self.muon_params]
@@ -80,9 +87,15 @@ class MuonAdamW:
             gd = grads[0].dtype
             if any(g.dtype != gd for g in grads):
                 raise ValueError("Muon grads must share one dtype")
-            api.muon_step(self.muon_params, grads, self.momentum, self._groups(gd), self.lr,
-                          self.beta, self.wd, self.ns_steps, self.coeffs, self.flags,
-                          self.workspace, stream=stream)
+            if replicas:
+                reps = [[rep[k] for k in self._order] for rep in replicas]
+                api.muon_step_replicated(self.muon_params, grads, self.momentum, self._groups(gd), self.lr,
+                                         self.beta, self.wd, self.ns_steps, self.coeffs, self.flags,
+                                         self.workspace, reps, stream=stream)
+            else:
+                api.muon_step(self.muon_params, grads, self.momentum, self._groups(gd), self.lr,
+                              self.beta, self.wd, self.ns_steps, self.coeffs, self.flags,
+                              self.workspace, stream=stream)
         specs = []
         for g in self.adamw_groups:
             grads = [p.grad for p in g["params"]]

@@ -111,6 +111,76 @@ def test_owner_sharded_step_equals_single_process(tmp_path):
         assert res[r]["momentum_keys"] == res[r]["owned"]
 
 
+def _worker_peer(rank, world, port, out_dir, all_params):
+    """As _worker, with every rank's Muon parameters in shared memory standing
+    in for peer GPU memory: owners write the other rank's copies in their
+    step (peer_params) instead of broadcasting."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    import oracle
+    from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    params = all_params[rank]
+    peers = {r: all_params[r] for r in range(world) if r != rank}
+    calls = {"replicated": 0}
+
+    def step_fn(ps, gs, ms, replicas):
+        calls["replicated"] += 1
+        for k, (p, g, m) in enumerate(zip(ps, gs, ms)):
+            w_new, m_new, _ = oracle.muon_step(p.numpy(), g.numpy(), m.numpy(), LR, BETA, WD)
+            p.copy_(torch.from_numpy(w_new))
+            m.copy_(torch.from_numpy(m_new))
+            for rep in replicas:
+                rep[k].copy_(torch.from_numpy(w_new))
+
+    opt = DistributedMuonAdamW(params, [], step_fn=step_fn, peer_params=peers)
+    for step in range(2):
+        for p, g in zip(params, _grads(rank, step)):
+            p.grad = g
+        opt.step()
+    out = {"params": [p.numpy().tolist() for p in params], "calls": calls["replicated"]}
+    with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+        json.dump(out, f)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_owner_writes_peer_replicas_equals_single_process(tmp_path):
+    world, port = 2, _free_port()
+    all_params = []
+    for r in range(world):
+        ps = [p.clone() for p in _params()]
+        for p in ps:
+            p.share_memory_()
+        all_params.append(ps)
+    mp.start_processes(_worker_peer, args=(world, port, str(tmp_path), all_params), nprocs=world,
+                       join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
+    ref_params, _ = _reference()
+    for r in range(world):
+        assert res[r]["calls"] == 2
+        for got, want in zip(res[r]["params"], ref_params):
+            np.testing.assert_allclose(np.array(got), want, rtol=0, atol=1e-15)
+
+
+def test_peer_params_must_cover_other_ranks():
+    sys.path.insert(0, ROOT)
+    from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
+    ps = _params()
+    import pytest
+    with pytest.raises(ValueError):
+        DistributedMuonAdamW(ps, [], step_fn=lambda *a: None, peer_params={1: ps})   # world 1: no peers
+    seen = []
+    opt = DistributedMuonAdamW(ps, [], step_fn=lambda p, g, m, reps: seen.append(len(reps)),
+                               peer_params={})                                    # world 1: none needed
+    for p in ps:
+        p.grad = torch.zeros_like(p)
+    opt.step()
+    assert seen == [0]
+
+
 def test_owner_assignment_balances_ns_cost():
     sys.path.insert(0, ROOT)
     from muon_polar_orthogonalized_b200.distributed import assign_owners, ns_cost

@@ -356,6 +356,67 @@ def test_illcond_high_condition_fp32_debug(dev):
               "vs bf16-emulated:", rel(u, oracle.newton_schulz_bf16_emulated(x, FIXED, 5)))
 
 
+@pytest.mark.parametrize("mode", ["fused", "unfused", "normuon", "fp32", "ns0"])
+def test_replicated_step_writes_every_copy(dev, mode):
+    """muon_step_replicated leaves W exactly as muon_step does and every copy
+    equal to W, bit for bit: on the fused path the last product's epilogue
+    writes the copies (vector and, for 198 columns, scalar stores); the other
+    paths copy W after the update.  Copies start as garbage."""
+    shapes = [(256, 1024), (1024, 256), (130, 198)]
+    flags = STEP_FLAGS | {"fused": 0, "unfused": N.MUON_UNFUSED_UPDATE, "normuon": N.MUON_NORMUON,
+                          "fp32": N.MUON_FP32_DEBUG, "ns0": 0}[mode]
+    ns = 0 if mode == "ns0" else 5
+    ref_w = None
+    for replicated in (False, True):
+        groups, W, G, M, _, _ = make_state(dev, shapes, "bf16", 41, counts=[2, 1, 1])
+        ws = workspace(api.muon_workspace_size(groups, flags), dev)
+        if replicated:
+            reps = [[torch.full_like(w, float("nan")) for w in W] for _ in range(2)]
+            api.muon_step_replicated(W, G, M, groups, 0.02, 0.95, 0.01, ns, FIXED, flags, ws, reps)
+        else:
+            api.muon_step(W, G, M, groups, 0.02, 0.95, 0.01, ns, FIXED, flags, ws)
+        torch.cuda.synchronize()
+        if not replicated:
+            ref_w = [w.clone() for w in W]
+    for i, w in enumerate(W):
+        assert torch.equal(w, ref_w[i]), i
+        for rep in reps:
+            assert torch.equal(rep[i], w), i
+
+
+def test_optimizer_replicas_follow_construction_order(dev):
+    """MuonAdamW groups matrices by shape internally; replicas given in the
+    construction order still land on the right copies."""
+    from muon_polar_orthogonalized_b200.optimizer import MuonAdamW
+    shapes = [(256, 512), (512, 256), (256, 512), (128, 128), (512, 256)]
+    ps = [torch.randn(s, device=dev) * 0.02 for s in shapes]
+    for k, p in enumerate(ps):
+        p.grad = torch.randn(shapes[k], device=dev)
+    twin = [p.clone() for p in ps]
+    for p, t in zip(ps, twin):
+        t.grad = p.grad.clone()
+    reps = [[torch.zeros_like(p) for p in ps] for _ in range(3)]
+    MuonAdamW(ps).step(replicas=reps)
+    MuonAdamW(twin).step()
+    torch.cuda.synchronize()
+    for k in range(len(ps)):
+        assert torch.equal(ps[k], twin[k])
+        for rep in reps:
+            assert torch.equal(rep[k], ps[k]), k
+
+
+def test_replicated_step_multi_wave(dev):
+    """A workspace that holds one matrix at a time: copies still complete."""
+    shapes = [(256, 512), (512, 256)]
+    groups, W, G, M, _, _ = make_state(dev, shapes, "bf16", 42, counts=[3, 2])
+    ws = workspace(api.muon_workspace_min_size(groups, STEP_FLAGS), dev)
+    reps = [[torch.zeros_like(w) for w in W]]
+    api.muon_step_replicated(W, G, M, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws, reps)
+    torch.cuda.synchronize()
+    for w, c in zip(W, reps[0]):
+        assert torch.equal(w, c)
+
+
 def test_multi_wave_matches_single_wave(dev):
     """A workspace too small for all matrices forces several waves: same bits."""
     shapes = [(256, 512), (512, 256)]

@@ -108,6 +108,26 @@ def test_row_equilibrate_workspace_holds_one_partial_per_row():
     assert api.muon_workspace_min_size(groups, N.MUON_ROW_EQUILIBRATE) > api.muon_workspace_min_size(groups, 0)
 
 
+def test_replicated_step_validation(L):
+    groups = api.make_groups([(64, 128, 2, 0, 0, 1.0)])
+    arr = (ctypes.c_void_p * 2)(0x10000, 0x10000)
+    ca = (ctypes.c_float * 15)(*([1.0] * 15))
+    bad = (ctypes.c_void_p * 2)(0x10000, 0x10008)          # misaligned copy
+    good = (ctypes.c_void_p * 2)(0x20000, 0x20000)
+
+    def call(table, n):
+        return L.muon_step_replicated(arr, arr, arr, groups, 1, 0.02, 0.95, 0.01, 5, ca, 3,
+                                      ctypes.c_void_p(0x1000), 1 << 40, table, n, None)
+    T = ctypes.POINTER(ctypes.c_void_p) * 8
+    assert call(None, 1) == N.MUON_ERR_INVALID_ARG
+    assert call(T(*[ctypes.cast(good, ctypes.POINTER(ctypes.c_void_p))] * 8), 8) == N.MUON_ERR_INVALID_ARG
+    assert call(T(ctypes.cast(bad, ctypes.POINTER(ctypes.c_void_p))), 1) == N.MUON_ERR_INVALID_ARG
+    assert "replicas[0]" in N.last_error()
+    assert call(T(ctypes.cast(good, ctypes.POINTER(ctypes.c_void_p)),
+                  ctypes.POINTER(ctypes.c_void_p)()), 2) == N.MUON_ERR_INVALID_ARG
+    assert "replicas[1]" in N.last_error()
+
+
 def test_adamw_validation(L):
     p = (ctypes.c_void_p * 1)(0x10000)
     n = (ctypes.c_int64 * 1)(16)
