@@ -343,15 +343,25 @@ def run_gpu(args):
     api.muon_profiler_reset()
     api.muon_profiler_enable(True)
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for k in range(args.steps):
         step()
-    e1.record(stream)
+        evs[k + 1].record(stream)
+    e0, e1 = evs[0], evs[-1]
     barrier()
     api.muon_profiler_enable(False)
     clk = clocks.stop()
     ms_total = max_over_ranks(e0.elapsed_time(e1))
+    per_step = sorted(evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps))
+
+    def quantile(q):
+        x = q * (len(per_step) - 1)
+        lo = int(x)
+        hi = min(lo + 1, len(per_step) - 1)
+        return per_step[lo] + (per_step[hi] - per_step[lo]) * (x - lo)
+    step_quantiles = {name: round(max_over_ranks(quantile(q)), 3)
+                      for name, q in (("p10", 0.1), ("p50", 0.5), ("p90", 0.9))}
     prof = api.muon_profiler_read()
     ms_step = ms_total / args.steps
 
@@ -479,6 +489,7 @@ def run_gpu(args):
             "steps": args.steps,
             "warmup": args.warmup,
             "ms_per_step": round(ms_step, 3),
+            "step_ms_quantiles": step_quantiles,
             "higher_is_better": False,
             "scaling": "weak",
             "vs_baseline": None,
@@ -488,7 +499,8 @@ def run_gpu(args):
                        "muon_groups": [[s.rows, s.cols, s.count] for s in wl.muon],
                        "ns_steps": K, "grads": "bf16", "params_state": "fp32",
                        "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
-                       "gemm_tiles": "128x256 single-CTA" if args.single_cta else "256x256 CTA pair",
+                       "gemm_tiles": "128x256 single-CTA" if args.single_cta else
+                       "CTA pairs: 256x512 (Gram, B'X), 256x256 (A*A, fused update)",
                        "normuon": bool(args.normuon), "row_equilibrate": bool(args.row_equilibrate)},
             "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
@@ -508,6 +520,17 @@ def run_gpu(args):
 
 
 # --------------------------------------------------------- CPU (oracle)
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(wl, reps: int = 1):
     """The oracle, as it stands, on a bounded sample of the workload, scaled to
     ms per full step: one Muon matrix of the cheapest shape group (timed
@@ -546,6 +569,7 @@ def cpu_baseline(wl, reps: int = 1):
         oracle.adamw_step(p, g, z, z, 1, W.ADAMW_LR, 0.9, 0.95, 1e-8, 0.0)
         adam_ms = (time.perf_counter() - t0) * (n_adam / k) * 1e3
     return {"value": round(muon_ms + adam_ms, 1), "unit": "ms", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"fp64 NumPy muon_step on one {s.rows}x{s.cols} matrix ({t_mat:.2f} s) scaled by "
                       f"nominal NS FLOPs to all {sum(x.count for x in wl.muon)} matrices, plus AdamW on "
                       f"{min(n_adam, 1 << 22)} elements scaled to {n_adam}",
