@@ -158,6 +158,25 @@ muon_status muon_step_replicated(float* const* params, const void* const* grads,
                                  float* const* const* replicas, int n_replicas, muon_stream_t stream);
 
 /*
+ * Mean of `count` tensors over n_sources copies, computed by this GPU:
+ *   dst[i][e] <- (sources[0][i][e] + ... + sources[n_sources-1][i][e]) * (1/n_sources)
+ * summed in fp32 in that order and stored in `dtype` (round to nearest even
+ * for bf16).  The data-parallel mean gradient that the owner of a matrix
+ * needs before its Muon step ("3.9 Optimizers: SGD, Adam, Adafactor, Lion,
+ * Muon & Shampoo", Wiring the hybrid recipe): the sources may be the other
+ * ranks' gradient buffers in peer GPU memory (peer access or a mapped IPC /
+ * symmetric-memory allocation), read with plain loads over NVLink; no
+ * multicast.  dst[i] may be one of sources[r][i] (each element is read
+ * before it is written by the same thread).  The sources must not change
+ * until `stream` passes this call.
+ * dst: host array of `count` device pointers; sources: host array of
+ * n_sources host arrays of `count` device pointers; numel: host, elements
+ * per tensor.  Every pointer 16-byte aligned.  n_sources in [1, 8].
+ */
+muon_status muon_reduce_mean(void* const* dst, const void* const* const* sources, int n_sources,
+                             const int64_t* numel, int count, int32_t dtype, muon_stream_t stream);
+
+/*
  * muon_step without a caller workspace, for callers that cannot allocate
  * device memory (no counterpart on the optimizer pages: it is a deployment
  * aid).  Programs whose device-memory budget is fixed at start-up by another

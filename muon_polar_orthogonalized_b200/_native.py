@@ -65,6 +65,8 @@ SIGNATURES = {
                                      POINTER(MuonGroup), c_int, c_float, c_float, c_float, c_int,
                                      POINTER(c_float), c_uint32, c_void_p, c_size_t,
                                      POINTER(POINTER(c_void_p)), c_int, c_void_p]),
+    "muon_reduce_mean": (c_int, [POINTER(c_void_p), POINTER(POINTER(c_void_p)), c_int, POINTER(c_int64),
+                                 c_int, c_int32, c_void_p]),
     "muon_schedule_advance": (c_int, [c_void_p, c_int64, c_float, c_float, c_float, c_void_p]),
     "muon_schedule_advance_cosine": (c_int, [c_void_p, c_int64, c_int64, c_float, c_void_p]),
     "muon_step_scheduled": (c_int, [POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p),

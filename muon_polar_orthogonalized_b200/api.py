@@ -97,6 +97,25 @@ def muon_step_replicated(params, grads, momentum, groups: Sequence, lr: float, b
     check(st, "muon_step_replicated")
 
 
+def muon_reduce_mean(dst: Sequence, sources: Sequence[Sequence], stream=None) -> None:
+    """dst[i] <- mean over r of sources[r][i] (fp32 or bf16 tensors of one
+    dtype; sources may live in peer GPUs' memory)."""
+    import torch
+    if not dst:
+        return
+    dt = N.MUON_BF16 if dst[0].dtype == torch.bfloat16 else N.MUON_F32
+    for t in list(dst) + [x for src in sources for x in src]:
+        if t.dtype != dst[0].dtype or not t.is_contiguous():
+            raise ValueError("muon_reduce_mean: tensors must be contiguous and share one dtype")
+    numel = (c_int64 * len(dst))(*[t.numel() for t in dst])
+    rows = [_ptrs(src) for src in sources]
+    table = (ctypes.POINTER(c_void_p) * max(len(rows), 1))(
+        *[ctypes.cast(r, ctypes.POINTER(c_void_p)) for r in rows])
+    st = N.lib().muon_reduce_mean(_ptrs(dst), table, len(rows), numel, len(dst), dt,
+                                  c_void_p(_stream_handle(stream)))
+    check(st, "muon_reduce_mean")
+
+
 def muon_step_scheduled(params, grads, momentum, groups: Sequence, lr: float, beta: float, wd: float,
                         ns_steps: int, coeffs, flags: int, workspace, schedule_state,
                         workspace_bytes: Optional[int] = None, stream=None) -> None:

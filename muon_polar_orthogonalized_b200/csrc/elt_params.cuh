@@ -80,4 +80,21 @@ struct ReplParams {
   int total_blocks;
 };
 
+// ------------------------------------------------------------ reduce_mean
+// dst[i] <- (src[0][i] + src[1][i] + ... + src[n-1][i]) * (1/n), summed in
+// fp32 in that order; tensors fp32 or bf16 (one dtype per launch).
+constexpr int kMaxSources = 8;
+constexpr int kMeanTensors = 64;
+struct MeanParams {
+  const void* src[kMaxSources][kMeanTensors];
+  void* dst[kMeanTensors];
+  long long numel[kMeanTensors];
+  int blk_begin[kMeanTensors];
+  int ntensors;
+  int nsrc;
+  int total_blocks;
+  int bf16;
+  float inv_n;
+};
+
 }  // namespace muon

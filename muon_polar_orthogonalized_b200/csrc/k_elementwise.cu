@@ -792,6 +792,50 @@ replicate_kernel(const __grid_constant__ ReplParams p) {
 
 int repl_chunk() { return kReplChunk; }
 
+// ------------------------------------------------------------ reduce_mean
+// Persistent, 4096-element chunks; each thread handles 4 groups of 4
+// consecutive elements (16-byte fp32 / 8-byte bf16 accesses; every pointer
+// is 16-byte aligned), the tail of a tensor element by element.
+template <bool BF16>
+__global__ void __launch_bounds__(kEltThreads)
+reduce_mean_kernel(const __grid_constant__ MeanParams p) {
+  for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
+    int ti = 0;
+    while (ti + 1 < p.ntensors && p.blk_begin[ti + 1] <= blk) ++ti;
+    const long long e0 = static_cast<long long>(blk - p.blk_begin[ti]) * kReplChunk;
+    const long long n = p.numel[ti];
+    const long long nvec = n & ~3ll;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long e = e0 + (static_cast<long long>(u) * kEltThreads + threadIdx.x) * 4;
+      if (e < nvec) {
+        float4 acc = load_g4<BF16>(p.src[0][ti], e);
+        for (int r = 1; r < p.nsrc; ++r) {
+          const float4 g = load_g4<BF16>(p.src[r][ti], e);
+          acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
+        }
+        acc.x *= p.inv_n; acc.y *= p.inv_n; acc.z *= p.inv_n; acc.w *= p.inv_n;
+        store_x4(p.dst[ti], e, acc, !BF16);
+      }
+    }
+    if (e0 + kReplChunk >= n && threadIdx.x < n - nvec) {   // the tensor's last chunk: scalar tail
+      const long long e = nvec + threadIdx.x;
+      float acc = load_g1<BF16>(p.src[0][ti], e);
+      for (int r = 1; r < p.nsrc; ++r) acc += load_g1<BF16>(p.src[r][ti], e);
+      store_x1(p.dst[ti], e, acc * p.inv_n, !BF16);
+    }
+  }
+}
+
+cudaError_t launch_reduce_mean(const MeanParams& p, int sms, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  const long long g = static_cast<long long>(sms) * 4;
+  const int grid = static_cast<int>(g < p.total_blocks ? g : p.total_blocks);
+  if (p.bf16) reduce_mean_kernel<true><<<grid, kEltThreads, 0, s>>>(p);
+  else reduce_mean_kernel<false><<<grid, kEltThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0 || p.nrep <= 0) return cudaSuccess;
   const long long g = static_cast<long long>(sms) * 4;

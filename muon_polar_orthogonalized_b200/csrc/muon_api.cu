@@ -35,6 +35,7 @@ cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
 cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s);
+cudaError_t launch_reduce_mean(const MeanParams& p, int sms, cudaStream_t s);
 int repl_chunk();
 cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
                                     cudaStream_t st);
@@ -876,6 +877,55 @@ muon_status muon_step_replicated(float* const* params, const void* const* grads,
                                  muon_stream_t stream) {
   return muon_step_impl(params, grads, momentum, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
                         flags, workspace, workspace_bytes, stream, nullptr, replicas, n_replicas);
+}
+
+muon_status muon_reduce_mean(void* const* dst, const void* const* const* sources, int n_sources,
+                             const int64_t* numel, int count, int32_t dtype, muon_stream_t stream) {
+  g_err[0] = '\0';
+  if (count < 0) return fail(MUON_ERR_INVALID_ARG, "count < 0");
+  if (n_sources < 1 || n_sources > kMaxSources)
+    return fail(MUON_ERR_INVALID_ARG, "n_sources %d outside [1, %d]", n_sources, kMaxSources);
+  if (dtype != MUON_F32 && dtype != MUON_BF16) return fail(MUON_ERR_INVALID_ARG, "dtype %d unknown", dtype);
+  if (count > 0 && (!dst || !sources || !numel)) return fail(MUON_ERR_INVALID_ARG, "dst, sources or numel is NULL");
+  for (int r = 0; r < n_sources; ++r)
+    if (count > 0 && !sources[r]) return fail(MUON_ERR_INVALID_ARG, "sources[%d] is NULL", r);
+  for (int i = 0; i < count; ++i) {
+    if (numel[i] < 0 || numel[i] >= (1ll << 40)) return fail(MUON_ERR_INVALID_ARG, "numel[%d] out of range", i);
+    if (!dst[i] || !aligned(dst[i], 16)) return fail(MUON_ERR_INVALID_ARG, "dst[%d] NULL or not 16-byte aligned", i);
+    for (int r = 0; r < n_sources; ++r)
+      if (!sources[r][i] || !aligned(sources[r][i], 16))
+        return fail(MUON_ERR_INVALID_ARG, "sources[%d][%d] NULL or not 16-byte aligned", r, i);
+  }
+  DevInfo dev;
+  muon_status st = device_info(&dev);
+  if (st != MUON_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MeanParams P;
+  std::memset(&P, 0, sizeof(P));
+  auto flush = [&]() -> muon_status {
+    if (P.ntensors == 0) return MUON_OK;
+    P.nsrc = n_sources;
+    P.bf16 = dtype == MUON_BF16;
+    P.inv_n = 1.0f / static_cast<float>(n_sources);
+    cudaError_t e = launch_reduce_mean(P, dev.sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "reduce_mean launch");
+    std::memset(&P, 0, sizeof(P));
+    return MUON_OK;
+  };
+  for (int i = 0; i < count; ++i) {
+    if (numel[i] == 0) continue;
+    const long long nblk = (numel[i] + repl_chunk() - 1) / repl_chunk();
+    if (P.ntensors == kMeanTensors || P.total_blocks + nblk > (1ll << 30))
+      if ((st = flush()) != MUON_OK) return st;
+    const int t = P.ntensors;
+    for (int r = 0; r < n_sources; ++r) P.src[r][t] = sources[r][i];
+    P.dst[t] = dst[i];
+    P.numel[t] = numel[i];
+    P.blk_begin[t] = P.total_blocks;
+    P.total_blocks += static_cast<int>(nblk);
+    P.ntensors += 1;
+  }
+  return flush();
 }
 
 muon_status muon_step(float* const* params, const void* const* grads, float* const* momentum,

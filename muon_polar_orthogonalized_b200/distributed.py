@@ -17,7 +17,10 @@ With peer_params (every other rank's parameter tensors, addressable from
 this GPU through peer access or symmetric memory), step 3 becomes part of
 step 2: the owner's last Newton-Schulz epilogue stores each updated tile into
 every rank's replica over NVLink (muon_step_replicated), and one barrier
-orders the ranks after all owners' writes.
+orders the ranks after all owners' writes.  With peer_grads (every other
+rank's gradient tensors, addressable likewise), step 1 becomes a barrier
+(every rank's gradients are written) and a kernel on the owner that averages
+its matrices' gradients from all ranks over NVLink (muon_reduce_mean).
 
 AdamW parameters have their gradients all-reduced (mean) and are stepped on
 every rank.  Owners are chosen by longest-processing-time over the executed
@@ -64,14 +67,21 @@ class DistributedMuonAdamW:
     keyword arguments given here).  peer_params: optional {rank: that rank's
     muon_params tensors in the same order} for every other rank, writable
     from this process (peer GPU memory); owners then write every rank's copy
-    in their update and the broadcasts are skipped.  The process group must
-    be initialised unless world size is 1.
+    in their update and the broadcasts are skipped.  peer_grads: likewise
+    every other rank's gradient tensors of muon_params (their .grad buffers,
+    which must stay the same tensors across steps); owners then average
+    their matrices' gradients from all ranks themselves instead of the
+    per-owner reduces.  reduce_fn(dst, sources) replaces that average
+    (default muon_reduce_mean).  The process group must be initialised
+    unless world size is 1.
     """
 
     def __init__(self, muon_params: Sequence[torch.Tensor], adamw_groups: Sequence[Dict] = (),
                  process_group=None, step_fn: Optional[Callable] = None,
                  adamw_fn: Optional[Callable] = None,
-                 peer_params: Optional[Dict[int, Sequence[torch.Tensor]]] = None, **muon_kwargs):
+                 peer_params: Optional[Dict[int, Sequence[torch.Tensor]]] = None,
+                 peer_grads: Optional[Dict[int, Sequence[torch.Tensor]]] = None,
+                 reduce_fn: Optional[Callable] = None, **muon_kwargs):
         self.group = process_group
         self.world = dist.get_world_size(process_group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(process_group) if dist.is_initialized() else 0
@@ -98,6 +108,17 @@ class DistributedMuonAdamW:
                         tuple(a.shape) != tuple(b.shape) for a, b in zip(peer_params[r], self.muon_params)):
                     raise ValueError(f"peer_params[{r}] does not match muon_params")
             self.peer_params = {r: list(peer_params[r]) for r in others}
+        self.peer_grads = None
+        if peer_grads is not None:
+            others = sorted(r for r in range(self.world) if r != self.rank)
+            if sorted(peer_grads) != others:
+                raise ValueError(f"peer_grads must hold exactly the other ranks {others}")
+            for r in others:
+                if len(peer_grads[r]) != len(self.muon_params) or any(
+                        tuple(a.shape) != tuple(b.shape) for a, b in zip(peer_grads[r], self.muon_params)):
+                    raise ValueError(f"peer_grads[{r}] does not match muon_params")
+            self.peer_grads = {r: list(peer_grads[r]) for r in others}
+        self.reduce_fn = reduce_fn
 
     def _bucket(self, tensors: List[torch.Tensor]) -> torch.Tensor:
         return torch.cat([t.reshape(-1) for t in tensors]) if tensors else torch.empty(0)
@@ -109,20 +130,41 @@ class DistributedMuonAdamW:
             t.copy_(flat[off:off + n].view_as(t))
             off += n
 
+    def _owner_mean_from_peers(self) -> None:
+        """Every rank's gradients are written (barrier); then each owner
+        averages its matrices' gradients over all ranks, in rank order, into
+        its own .grad tensors."""
+        if self.world > 1:
+            dist.barrier(group=self.group)
+        own = self.owned
+        if not own:
+            return
+        dst = [self.muon_params[i].grad for i in own]
+        sources = [dst if r == self.rank else [self.peer_grads[r][i] for i in own]
+                   for r in range(self.world)]
+        if self.reduce_fn is not None:
+            self.reduce_fn(dst, sources)
+        else:
+            from . import api
+            api.muon_reduce_mean(dst, sources)
+
     @torch.no_grad()
     def step(self) -> None:
         # 1. mean gradient of each matrix onto its owner
-        for r in range(self.world):
-            idx = [i for i, o in enumerate(self.owners) if o == r]
-            if not idx:
-                continue
-            grads = [self.muon_params[i].grad for i in idx]
-            if self.world > 1:
-                flat = self._bucket(grads)
-                dist.reduce(flat, dst=r, op=dist.ReduceOp.SUM, group=self.group)
-                if r == self.rank:
-                    flat.div_(self.world)
-                    self._unbucket(flat, grads)
+        if self.peer_grads is not None:
+            self._owner_mean_from_peers()
+        else:
+            for r in range(self.world):
+                idx = [i for i, o in enumerate(self.owners) if o == r]
+                if not idx:
+                    continue
+                grads = [self.muon_params[i].grad for i in idx]
+                if self.world > 1:
+                    flat = self._bucket(grads)
+                    dist.reduce(flat, dst=r, op=dist.ReduceOp.SUM, group=self.group)
+                    if r == self.rank:
+                        flat.div_(self.world)
+                        self._unbucket(flat, grads)
         # AdamW gradients: all-reduce mean
         adam_params = [p for g in self.adamw_groups for p in g["params"]]
         if adam_params and self.world > 1:

@@ -13,6 +13,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -111,10 +112,12 @@ def test_owner_sharded_step_equals_single_process(tmp_path):
         assert res[r]["momentum_keys"] == res[r]["owned"]
 
 
-def _worker_peer(rank, world, port, out_dir, all_params):
-    """As _worker, with every rank's Muon parameters in shared memory standing
-    in for peer GPU memory: owners write the other rank's copies in their
-    step (peer_params) instead of broadcasting."""
+def _worker_peer(rank, world, port, out_dir, all_params, all_grads):
+    """As _worker, with every rank's Muon parameters (and, if given, gradients)
+    in shared memory standing in for peer GPU memory: owners write the other
+    rank's copies in their step (peer_params) instead of broadcasting, and
+    average the gradients from every rank themselves (peer_grads) instead of
+    the reduces."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -124,7 +127,16 @@ def _worker_peer(rank, world, port, out_dir, all_params):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     params = all_params[rank]
     peers = {r: all_params[r] for r in range(world) if r != rank}
-    calls = {"replicated": 0}
+    peer_grads = {r: all_grads[r] for r in range(world) if r != rank} if all_grads else None
+    calls = {"replicated": 0, "mean": 0}
+
+    def reduce_fn(dst, sources):
+        calls["mean"] += 1
+        for i, d in enumerate(dst):
+            acc = sources[0][i].clone()
+            for src in sources[1:]:
+                acc += src[i]
+            d.copy_(acc / len(sources))
 
     def step_fn(ps, gs, ms, replicas):
         calls["replicated"] += 1
@@ -135,32 +147,43 @@ def _worker_peer(rank, world, port, out_dir, all_params):
             for rep in replicas:
                 rep[k].copy_(torch.from_numpy(w_new))
 
-    opt = DistributedMuonAdamW(params, [], step_fn=step_fn, peer_params=peers)
+    opt = DistributedMuonAdamW(params, [], step_fn=step_fn, peer_params=peers, peer_grads=peer_grads,
+                               reduce_fn=reduce_fn)
     for step in range(2):
-        for p, g in zip(params, _grads(rank, step)):
-            p.grad = g
+        for k, (p, g) in enumerate(zip(params, _grads(rank, step))):
+            if all_grads:
+                all_grads[rank][k].copy_(g)      # the rank's gradient buffer, seen by its peers
+                p.grad = all_grads[rank][k]
+            else:
+                p.grad = g
         opt.step()
-    out = {"params": [p.numpy().tolist() for p in params], "calls": calls["replicated"]}
+    out = {"params": [p.numpy().tolist() for p in params], "calls": calls["replicated"],
+           "mean_calls": calls["mean"]}
     with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
         json.dump(out, f)
     dist.barrier()
     dist.destroy_process_group()
 
 
-def test_owner_writes_peer_replicas_equals_single_process(tmp_path):
+@pytest.mark.parametrize("peer_grads", [False, True])
+def test_owner_writes_peer_replicas_equals_single_process(tmp_path, peer_grads):
     world, port = 2, _free_port()
-    all_params = []
+    all_params, all_grads = [], []
     for r in range(world):
         ps = [p.clone() for p in _params()]
-        for p in ps:
-            p.share_memory_()
+        gs = [torch.zeros_like(p) for p in ps]
+        for t in ps + gs:
+            t.share_memory_()
         all_params.append(ps)
-    mp.start_processes(_worker_peer, args=(world, port, str(tmp_path), all_params), nprocs=world,
-                       join=True, start_method="spawn")
+        all_grads.append(gs)
+    mp.start_processes(_worker_peer, args=(world, port, str(tmp_path), all_params,
+                                           all_grads if peer_grads else None),
+                       nprocs=world, join=True, start_method="spawn")
     res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
     ref_params, _ = _reference()
     for r in range(world):
         assert res[r]["calls"] == 2
+        assert res[r]["mean_calls"] == (2 if peer_grads else 0)
         for got, want in zip(res[r]["params"], ref_params):
             np.testing.assert_allclose(np.array(got), want, rtol=0, atol=1e-15)
 

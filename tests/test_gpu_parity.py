@@ -405,6 +405,33 @@ def test_optimizer_replicas_follow_construction_order(dev):
             assert torch.equal(rep[k], ps[k]), k
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_reduce_mean_bitwise(dev, dtype):
+    """muon_reduce_mean equals the same fp32 sum in rank order times the fp32
+    reciprocal, rounded to the tensors' dtype: bit for bit, for vector
+    bodies and scalar tails, several tensors per launch, in place too."""
+    shapes = [(256, 1024), (1001,), (7,), (130, 198), (1,)]
+    for nsrc in (1, 2, 3, 8):
+        srcs = [[torch.randn(s, device=dev).to(dtype) for s in shapes] for _ in range(nsrc)]
+        dst = [torch.empty(s, device=dev, dtype=dtype) for s in shapes]
+        api.muon_reduce_mean(dst, srcs)
+        inv = torch.tensor(1.0, dtype=torch.float32, device=dev) / nsrc
+        for i in range(len(shapes)):
+            acc = srcs[0][i].float()
+            for r in range(1, nsrc):
+                acc = acc + srcs[r][i].float()
+            want = (acc * inv).to(dtype)
+            assert torch.equal(dst[i], want), (nsrc, shapes[i])
+        # in place: the destination is source 0
+        keep = [t.clone() for t in srcs[0]]
+        api.muon_reduce_mean(srcs[0], srcs)
+        for i in range(len(shapes)):
+            acc = keep[i].float()
+            for r in range(1, nsrc):
+                acc = acc + srcs[r][i].float()
+            assert torch.equal(srcs[0][i], (acc * inv).to(dtype))
+
+
 def test_replicated_step_multi_wave(dev):
     """A workspace that holds one matrix at a time: copies still complete."""
     shapes = [(256, 512), (512, 256)]

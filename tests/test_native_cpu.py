@@ -128,6 +128,25 @@ def test_replicated_step_validation(L):
     assert "replicas[1]" in N.last_error()
 
 
+def test_reduce_mean_validation(L):
+    dst = (ctypes.c_void_p * 1)(0x10000)
+    src = (ctypes.c_void_p * 1)(0x20000)
+    n = (ctypes.c_int64 * 1)(100)
+    T = ctypes.POINTER(ctypes.c_void_p) * 9
+    tab = T(*[ctypes.cast(src, ctypes.POINTER(ctypes.c_void_p))] * 9)
+    assert L.muon_reduce_mean(dst, tab, 0, n, 1, 0, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_reduce_mean(dst, tab, 9, n, 1, 0, None) == N.MUON_ERR_INVALID_ARG
+    assert L.muon_reduce_mean(dst, tab, 2, n, 1, 7, None) == N.MUON_ERR_INVALID_ARG
+    bad = (ctypes.c_void_p * 1)(0x10004)
+    assert L.muon_reduce_mean(bad, tab, 2, n, 1, 0, None) == N.MUON_ERR_INVALID_ARG
+    misal = (ctypes.c_void_p * 1)(0x20008)
+    tab2 = T(ctypes.cast(src, ctypes.POINTER(ctypes.c_void_p)), ctypes.cast(misal, ctypes.POINTER(ctypes.c_void_p)))
+    assert L.muon_reduce_mean(dst, tab2, 2, n, 1, 0, None) == N.MUON_ERR_INVALID_ARG
+    assert "sources[1][0]" in N.last_error()
+    neg = (ctypes.c_int64 * 1)(-1)
+    assert L.muon_reduce_mean(dst, tab, 2, neg, 1, 0, None) == N.MUON_ERR_INVALID_ARG
+
+
 def test_adamw_validation(L):
     p = (ctypes.c_void_p * 1)(0x10000)
     n = (ctypes.c_int64 * 1)(16)
