@@ -307,7 +307,8 @@ def run_gpu(args):
     D = DeviceWorkload(wl, dev, e2e_host=not args.no_e2e, pinned=e2e_pinned)
     flags = (N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
              | (N.MUON_NORMUON if args.normuon else 0)
-             | (N.MUON_ROW_EQUILIBRATE if args.row_equilibrate else 0))
+             | (N.MUON_ROW_EQUILIBRATE if args.row_equilibrate else 0)
+             | (N.MUON_TC_NARROW_TILES if args.narrow_tiles else 0))
     ws_bytes = api.muon_workspace_size(D.groups, flags)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     coeffs = W.NS_COEFFS_FIXED
@@ -500,6 +501,7 @@ def run_gpu(args):
                        "ns_steps": K, "grads": "bf16", "params_state": "fp32",
                        "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
                        "gemm_tiles": "128x256 single-CTA" if args.single_cta else
+                       "CTA pairs: 256x256" if args.narrow_tiles else
                        "CTA pairs: 256x512 (Gram, B'X), 256x256 (A*A, fused update)",
                        "normuon": bool(args.normuon), "row_equilibrate": bool(args.row_equilibrate)},
             "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
@@ -609,6 +611,8 @@ def main():
                     help="row-normalise the orthogonalised update (NorMuon)")
     ap.add_argument("--row-equilibrate", action="store_true",
                     help="MuonEq row equilibration of the momentum-smoothed matrix before Newton-Schulz")
+    ap.add_argument("--narrow-tiles", action="store_true",
+                    help="Gram and B'X on 256x256 CTA-pair tiles instead of 256x512")
     ap.add_argument("--single-cta", action="store_true",
                     help="Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of CTA pairs")
     args = ap.parse_args()
