@@ -514,9 +514,10 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
                              static_cast<uint32_t>(acc * C::BN);
       // Active chunks form one range [c_lo, c_hi): a symmetric tile skips the
       // chunks of strictly lower 128-blocks (a prefix) and a ragged tile stops
-      // at N.  The bf16 operand of chunk c+1 is loaded while chunk c is
-      // combined and stored, so one L2 round trip is in flight at all times.
-      // The fused update loads X and W (prefetched to L2 above) with each chunk.
+      // at N.  For A*A the A operand of chunk c+1 is loaded while chunk c is
+      // combined and stored, so one L2 round trip is in flight at all times;
+      // the fused update loads W (prefetched to L2 above) with each chunk; the
+      // Gram and B'X epilogues load nothing.
       const int ib = row0 / 128;   // 128-row block of this CTA's rows
       int c_hi = 0;
       if (jslice < q.N) c_hi = min(kChunks, (q.N - jslice + 31) / 32);
@@ -533,13 +534,11 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         sm100::tmem_ld32(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), v);
         epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, mirror, in, win, v);
       };
-      if constexpr (EPI == EPI_AXPY_UPDATE) {
-        // no room for a second operand buffer next to W: one chunk at a time
+      if constexpr (EPI != EPI_POLY) {
 #pragma unroll 1
         for (int cc = c_lo; cc < c_hi; ++cc) {
-          EpiIn in;
-          epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc), chunk_j0(cc) + 32 <= q.N, in);
-          process(cc, in);
+          const EpiIn none{};
+          process(cc, none);
         }
       } else {
         EpiIn in0, in1;
