@@ -35,10 +35,20 @@ enum EpiKind : int { EPI_GRAM = 0, EPI_POLY = 1, EPI_AXPY = 2, EPI_AXPY_UPDATE =
 // One problem = `batch` same-shape matrices laid out at a fixed batch stride.
 //   C[i][j] = sum_k Aop(i,k) * Bop(j,k)
 //   Aop(i,k) = a[i*lda + k] (K-major) or a[k*lda + i] (MN-major), same for Bop.
+// Symmetric m x m matrices (A, B') are stored by the tensor-core path in
+// "upper" form: element (i, j) is written only where j/256 >= i/256 (the
+// 256x256 blocks on and above the diagonal, diagonal blocks in full).  A
+// product that reads such an operand takes a K block that lies left of the
+// operand rows' diagonal block from the stored block above the diagonal,
+// transposed (an MN-major load of rows k, columns i: the value at (k, i) is
+// the one (i, k) would hold).
+constexpr int kSymBlock = 256;
+
 struct GemmProblem {
   int M, N, K, batch;
   int a_mn, b_mn;
-  int sym;                  // output symmetric: upper tiles computed and mirrored
+  int sym;                  // output symmetric: upper tiles computed, upper form stored
+  int a_sym, b_sym;         // operand stored in upper form (tensor-core path)
   int tiles_m, tiles_n, tiles_per_mat, tile_begin;
   // operands (SIMT path reads these directly; the tensor-core path uses tensor maps)
   const void* a; long long a_bs; int a_ld;
@@ -57,6 +67,8 @@ struct GemmProblem {
 struct alignas(64) TcGemmParams {
   CUtensorMap tmA[kMaxProblems];
   CUtensorMap tmB[kMaxProblems];
+  CUtensorMap tmA2[kMaxProblems];   // MN-major boxes of an upper-form A operand (its K blocks left of the diagonal)
+  CUtensorMap tmB2[kMaxProblems];   // likewise for B
   GemmProblem prob[kMaxProblems];
   float* wptr[kMaxUpdMats];
   int wcols[kMaxUpdMats];   // param row pitch (= cols)

@@ -4,16 +4,19 @@
 // Newton-Schulz Orthogonalization; "3.9 Optimizers", Muon: Orthogonalizing
 // the Update) is three products:
 //   gram  A = s^2 X X^T          symmetric: only tiles touching the upper
-//                                triangle run; off-diagonal blocks are also
-//                                stored transposed (mirrored)
+//                                triangle run, and A is stored in upper form
+//                                (256x256 blocks on and above the diagonal)
 //   poly  B' = a I + b A + c A A symmetric likewise; A A = A A^T since A is
 //                                symmetric, so both operands are rows of A;
+//                                K blocks left of a row block's diagonal are
+//                                read transposed from the stored upper form;
 //                                the epilogue reads the A tile for b*A and
 //                                adds a on the diagonal
 //   axpy  X' = s B' X            = s (a X + B X); wide matrices; tall ones
 //                                (iterated as X^T) compute X' = s X B' in
-//                                parameter layout.  The epilogue only scales
-//                                and converts: a X rides in the product
+//                                parameter layout; B' is read like A above.
+//                                The epilogue only scales and converts: a X
+//                                rides in the product
 //   axpy_update                  last iteration: U = bf16(X') feeds the
 //                                cautious-decay update of W directly
 // s is the Frobenius scale 1/(||m~||+1e-7), applied on the first iteration
@@ -231,7 +234,7 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&e)[4], float (&a)[3
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const GemmProblem& q, int mat,
-                                               int i, int j0, bool full, bool wvec, bool mirror,
+                                               int i, int j0, bool full, bool wvec,
                                                const EpiIn& in, const EpiW& win, float (&v)[32]) {
   if (i >= q.M) return;
   float f = 1.f;
@@ -301,13 +304,6 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         if (j0 + c < q.N) row[c] = __float2bfloat16_rn(v[c]);
-    }
-    if (mirror) {
-      // out[j][i] for this thread's 32 columns; lanes hold consecutive i, so
-      // each of these stores is one coalesced 64-byte run across the warp.
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        if (j0 + c < q.N) out[static_cast<long long>(j0 + c) * q.out_ld + i] = __float2bfloat16_rn(v[c]);
     }
   }
 }
@@ -393,21 +389,27 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
             if (PAIR) sm100::tma_load_3d_pair(dst, m, leader_full, x, y, tc.mat);
             else sm100::tma_load_3d(dst, m, &full_bar[stage], x, y, tc.mat);
           };
-          if (!q.a_mn) {
+          // an upper-form operand's K block left of its rows' diagonal block
+          // comes transposed from the block above the diagonal (MN-major)
+          const bool a_t = q.a_sym && (k0 / kSymBlock) < (arow / kSymBlock);
+          if (!q.a_mn && !a_t) {
             load(sa, &p.tmA[tc.prob], k0, arow);
           } else {
+            const CUtensorMap* ma = a_t ? &p.tmA2[tc.prob] : &p.tmA[tc.prob];
 #pragma unroll
-            for (int h = 0; h < C::A_ROWS / 64; ++h) load(sa + h * 8192, &p.tmA[tc.prob], arow + h * 64, k0);
+            for (int h = 0; h < C::A_ROWS / 64; ++h) load(sa + h * 8192, ma, arow + h * 64, k0);
           }
 #pragma unroll
           for (int n = 0; n < NSUB; ++n) {
             uint8_t* sbn = sb + n * C::SUB_B_BYTES;
             const int brow_n = brow + n * TC_BN;
-            if (!q.b_mn) {
+            const bool b_t = q.b_sym && (k0 / kSymBlock) < (brow_n / kSymBlock);
+            if (!q.b_mn && !b_t) {
               load(sbn, &p.tmB[tc.prob], k0, brow_n);
             } else {
+              const CUtensorMap* mb = b_t ? &p.tmB2[tc.prob] : &p.tmB[tc.prob];
 #pragma unroll
-              for (int h = 0; h < C::SUB_B_ROWS / 64; ++h) load(sbn + h * 8192, &p.tmB[tc.prob], brow_n + h * 64, k0);
+              for (int h = 0; h < C::SUB_B_ROWS / 64; ++h) load(sbn + h * 8192, mb, brow_n + h * 64, k0);
             }
           }
           if (++stage == C::STAGES) {
@@ -439,7 +441,9 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         const TileCoord tc = decode_tile<C::BM, C::BN>(p, t);
         const GemmProblem& q = p.prob[tc.prob];
         const int kblocks = (q.K + C::BK - 1) / C::BK;
-        const uint32_t idesc = sm100::make_idesc_bf16(C::BM, TC_BN, q.a_mn, q.b_mn);
+        // 256-row blocks of the operand rows (the same for both CTAs of a pair)
+        const int ablk = (tc.tm * C::BM) / kSymBlock;
+        const int bblk0 = (tc.tn * C::BN) / kSymBlock;
         if (!sm100::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) {
           record_timeout(p.status, abort_flag);
           break;
@@ -453,20 +457,35 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
             break;
           }
           sm100::tc_fence_after();
+          // descriptors of this K block, built once: the single issuing thread
+          // must keep up with MMAs of ~128 cycles, so the inner loop only adds
+          // the K16 offset to the start-address field ((address >> 4) in 14
+          // bits; stage offsets never carry out of it)
           const uint32_t sa = sm100::smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
+          const int kblk = (kb * C::BK) / kSymBlock;
+          const bool a_mn = q.a_mn || (q.a_sym && kblk < ablk);
+          const uint64_t ad0 = a_mn ? sm100::make_sdesc(sa, 8192, 1024) : sm100::make_sdesc(sa, 16, 1024);
+          const uint64_t a_inc = a_mn ? (2048 >> 4) : (32 >> 4);
+          uint64_t bd0[NSUB], b_inc[NSUB];
+          uint32_t idn[NSUB];
+#pragma unroll
+          for (int n = 0; n < NSUB; ++n) {
+            const bool b_mn = q.b_mn || (q.b_sym && kblk < bblk0 + (n * TC_BN) / kSymBlock);
+            const uint32_t sbn = sb + n * C::SUB_B_BYTES;
+            bd0[n] = b_mn ? sm100::make_sdesc(sbn, 8192, 1024) : sm100::make_sdesc(sbn, 16, 1024);
+            b_inc[n] = b_mn ? (2048 >> 4) : (32 >> 4);
+            idn[n] = sm100::make_idesc_bf16(C::BM, TC_BN, a_mn ? 1 : 0, b_mn ? 1 : 0);
+          }
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
-            const uint64_t ad = q.a_mn ? sm100::make_sdesc(sa + kk * 2048, 8192, 1024)
-                                       : sm100::make_sdesc(sa + kk * 32, 16, 1024);
 #pragma unroll
             for (int n = 0; n < NSUB; ++n) {
-              const uint32_t sbn = sb + n * C::SUB_B_BYTES;
-              const uint64_t bd = q.b_mn ? sm100::make_sdesc(sbn + kk * 2048, 8192, 1024)
-                                         : sm100::make_sdesc(sbn + kk * 32, 16, 1024);
+              const uint64_t ad = ad0 + static_cast<uint64_t>(kk) * a_inc;
+              const uint64_t bd = bd0[n] + static_cast<uint64_t>(kk) * b_inc[n];
               const uint32_t dn = d_tmem + static_cast<uint32_t>(n * TC_BN);
-              if (PAIR) sm100::umma_bf16_pair(dn, ad, bd, idesc, (kb | kk) ? 1u : 0u);
-              else sm100::umma_bf16(dn, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+              if (PAIR) sm100::umma_bf16_pair(dn, ad, bd, idn[n], (kb | kk) ? 1u : 0u);
+              else sm100::umma_bf16(dn, ad, bd, idn[n], (kb | kk) ? 1u : 0u);
             }
           }
           if (PAIR) sm100::umma_commit_pair_both(&empty_bar[stage]);
@@ -518,21 +537,21 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       // combined and stored, so one L2 round trip is in flight at all times;
       // the fused update loads W (prefetched to L2 above) with each chunk; the
       // Gram and B'X epilogues load nothing.
-      const int ib = row0 / 128;   // 128-row block of this CTA's rows
+      // symmetric output in upper form: chunks left of the rows' 256-block are not stored
+      const int rblk = row0 / kSymBlock;
       int c_hi = 0;
       if (jslice < q.N) c_hi = min(kChunks, (q.N - jslice + 31) / 32);
       int c_lo = 0;
-      if (q.sym) c_lo = max(0, (128 * ib - jslice) / 32);
+      if (q.sym) c_lo = max(0, (kSymBlock * rblk - jslice) / 32);
       auto chunk_j0 = [&](int cc) { return jslice + cc * 32; };
       auto process = [&](int cc, const EpiIn& in) {
         const int j0 = chunk_j0(cc);
-        const bool mirror = q.sym && (j0 / 128) > ib;
         const bool full = (j0 + 32 <= q.N);
         EpiW win;
         epilogue_load_w<EPI>(p, q, tc.mat, i, j0, full, wvec, win);
         float v[32];
         sm100::tmem_ld32(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), v);
-        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, mirror, in, win, v);
+        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, in, win, v);
       };
       if constexpr (EPI != EPI_POLY) {
 #pragma unroll 1

@@ -663,7 +663,13 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldc;
       P.scale_mode = (k == 0) ? 2 : 0;
     }
-    if (f32) P.sym = 0;  // the fp32 scaffold computes full outputs
+    // the tensor-core path stores A and B' in upper form and reads them so;
+    // the fp32 scaffold computes and reads full matrices
+    if (!f32) {
+      if (epi == EPI_POLY) P.a_sym = P.b_sym = 1;
+      else if (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) (q.tall ? P.b_sym : P.a_sym) = 1;
+    }
+    if (f32) P.sym = 0;
     P.tiles_m = (P.M + BM - 1) / BM;
     P.tiles_n = (P.N + BN - 1) / BN;
     if (P.sym) {
@@ -689,14 +695,21 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
         st = map_for(&TP.tmA[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, 128);
         if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, b_rows);
       } else if (epi == EPI_POLY) {
+        // A in upper form: K-major boxes, plus MN-major boxes for its transposed K blocks
         st = map_for(&TP.tmA[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, 128);
         if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, b_rows);
+        if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
+        if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
       } else if (!q.tall) {
+        // B' in upper form (A operand here)
         st = map_for(&TP.tmA[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, 128);
         if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, 1, q.c, q.r, q.ldc, q.xstride, b_rows);
+        if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
       } else {
+        // B' in upper form (B operand here)
         st = map_for(&TP.tmA[nprob], xcur, 0, q.c, q.r, q.ldc, q.xstride, 128);
         if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, b_rows);
+        if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
       }
       if (st != MUON_OK) return st;
       TP.prob[nprob] = P;
