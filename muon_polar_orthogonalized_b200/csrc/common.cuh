@@ -69,6 +69,7 @@ struct alignas(64) TcGemmParams {
   CUtensorMap tmB[kMaxProblems];
   CUtensorMap tmA2[kMaxProblems];   // MN-major boxes of an upper-form A operand (its K blocks left of the diagonal)
   CUtensorMap tmB2[kMaxProblems];   // likewise for B
+  CUtensorMap tmOut[kMaxProblems];  // output rows of Gram and B'X: 32x32 boxes, 64-byte swizzle
   GemmProblem prob[kMaxProblems];
   float* wptr[kMaxUpdMats];
   int wcols[kMaxUpdMats];   // param row pitch (= cols)

@@ -61,6 +61,19 @@ namespace muon {
 #define MUON_TC_RASTER_GN 8
 #endif
 
+#ifndef MUON_TC_EPI_WARPS
+#define MUON_TC_EPI_WARPS 8
+#endif
+// Epilogue warps: a multiple of 4, since warp w may only read TMEM lanes
+// 32*(w%4) .. +31; with 8, two warps share each lane quadrant and split the
+// tile's 256 columns between them.
+constexpr int TC_EPI_WARPS = MUON_TC_EPI_WARPS;
+constexpr int TC_EPI_SPLIT = TC_EPI_WARPS / 4;          // column slices per lane quadrant
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;       // producer + MMA + epilogue warps
+// Output staging for the TMA row stores: per epilogue warp two 2 KB buffers of
+// 32 rows x 32 bf16 (64-byte swizzle), used alternately.
+constexpr int TC_STAGE_TILE_BYTES = 32 * 32 * 2;
+constexpr int TC_STAGING_BYTES = TC_EPI_WARPS * 2 * TC_STAGE_TILE_BYTES;
 template <bool PAIR, int NSUB>
 struct TcCfg {
   static_assert(NSUB == 1 || (PAIR && NSUB == 2), "512-column tiles need CTA pairs");
@@ -76,18 +89,12 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = NSUB == 2 ? MUON_TC_WIDE_STAGES : PAIR ? MUON_TC_PAIR_STAGES : 4;
   static constexpr int ACC_BUFS = NSUB == 1 ? 2 : 1;   // TMEM accumulators (512 columns in all)
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;          // barriers, TMEM slot, abort flag
+  static constexpr int STAGING_OFF = BAR_OFF + 1024;            // output staging (TC_STAGING_BYTES)
+  static constexpr int SMEM_BYTES = STAGING_OFF + TC_STAGING_BYTES + 1024 /*align slack*/;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 };
 constexpr int TC_BN = 256;   // columns of one MMA (N) and of a narrow tile
-#ifndef MUON_TC_EPI_WARPS
-#define MUON_TC_EPI_WARPS 8
-#endif
-// Epilogue warps: a multiple of 4, since warp w may only read TMEM lanes
-// 32*(w%4) .. +31; with 8, two warps share each lane quadrant and split the
-// tile's 256 columns between them.
-constexpr int TC_EPI_WARPS = MUON_TC_EPI_WARPS;
-constexpr int TC_EPI_SPLIT = TC_EPI_WARPS / 4;          // column slices per lane quadrant
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;       // producer + MMA + epilogue warps
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_RASTER_GN = MUON_TC_RASTER_GN;   // tile-column band width of the non-symmetric raster
 
@@ -133,6 +140,8 @@ __device__ __forceinline__ void record_timeout(unsigned int* status, volatile in
   atomicOr(status, kDevTimeout);
 }
 
+// Row store of one chunk straight from registers (A*A products): 4 x 16 bytes
+// per lane.
 __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -144,6 +153,39 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
       w[h] = *reinterpret_cast<uint32_t*>(&b);
     }
     d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// The Gram and B'X epilogues instead stage their rows for a TMA store (their
+// epilogues load nothing else, and the staged store measured faster there;
+// for A*A, whose epilogue also reads A, the direct store was faster).
+// One warp's 32 rows x 32 columns of output, lane = row: packed to bf16 into a
+// 2 KB staging buffer in the 64-byte-swizzle layout (16-byte unit u of row r
+// at unit u ^ ((r >> 1) & 3), four shared-memory wavefronts per store), then
+// written by one TMA store at (j0, y, mat).  The buffer used two chunks ago
+// is reused once its store has finished reading it.  Rows >= M and columns
+// >= N of the box are clipped by the tensor map; a box that starts at or
+// beyond row M is not issued.  Warp-uniform; every lane calls it.
+__device__ __forceinline__ void stage_row_store(const CUtensorMap* tmap, uint8_t* buf, int lane,
+                                                const float (&v)[32], int j0, int y, int M, int mat) {
+  if (lane == 0) sm100::bulk_wait_group_read<1>();
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(v[u * 8 + h * 2], v[u * 8 + h * 2 + 1]);
+      w[h] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    const int su = u ^ ((lane >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + lane * 64 + su * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  sm100::fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && y < M) {
+    sm100::tma_store_3d(tmap, buf, j0, y, mat);
+    sm100::bulk_commit_group();
   }
 }
 
@@ -295,9 +337,8 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
           for (int r = 0; r < p.nrep; ++r) p.rptr[r][wi][roff + c] = nv;
         }
     }
-  } else {
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(q.out) + mat * q.out_bs;
-    __nv_bfloat16* row = out + static_cast<long long>(i) * q.out_ld + j0;
+  } else if constexpr (EPI == EPI_POLY) {
+    __nv_bfloat16* row = static_cast<__nv_bfloat16*>(q.out) + mat * q.out_bs + static_cast<long long>(i) * q.out_ld + j0;
     if (full) {
       st_bf16x32(row, v);
     } else {
@@ -306,6 +347,7 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
         if (j0 + c < q.N) row[c] = __float2bfloat16_rn(v[c]);
     }
   }
+  // Gram and B'X: the row goes out through stage_row_store
 }
 
 template <int EPI, bool PAIR, int NSUB>
@@ -314,12 +356,13 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   using C = TcCfg<PAIR, NSUB>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty_bar = full_bar + C::STAGES;
   uint64_t* tfull_bar = empty_bar + C::STAGES;   // [2]
   uint64_t* tempty_bar = tfull_bar + 2;          // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* staging = smem + C::STAGING_OFF;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -510,6 +553,8 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     const int slice = (warp - 2) / 4;                   // which column slice of the tile
     constexpr int kChunks = C::BN / 32 / TC_EPI_SPLIT;  // 32-column chunks per warp
     const int row_in_cta = quad * 32 + lane;
+    uint8_t* my_staging = staging + (warp - 2) * 2 * TC_STAGE_TILE_BYTES;
+    int stage_ctr = 0;   // staging buffer in use: stage_ctr & 1
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = unit; t < p.total_tiles; t += nunits) {
@@ -552,6 +597,11 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         float v[32];
         sm100::tmem_ld32(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), v);
         epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, in, win, v);
+        if constexpr (EPI == EPI_GRAM || EPI == EPI_AXPY) {
+          stage_row_store(&p.tmOut[tc.prob], my_staging + (stage_ctr & 1) * TC_STAGE_TILE_BYTES, lane, v, j0,
+                          row0 + quad * 32, q.M, tc.mat);
+          ++stage_ctr;
+        }
       };
       if constexpr (EPI != EPI_POLY) {
 #pragma unroll 1
@@ -583,6 +633,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) sm100::bulk_wait_group<0>();   // every staged store written
   }
 
   sm100::tc_fence_before();

@@ -337,7 +337,8 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 
 // ------------------------------------------------------------ tensor maps
 muon_status make_map(CUtensorMap* map, void* base, int inner, int rows, int batch, size_t row_bytes,
-                     size_t batch_bytes, int box_inner, int box_rows) {
+                     size_t batch_bytes, int box_inner, int box_rows,
+                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   PFN_encodeTiled_t enc = get_encode();
   if (!enc) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
@@ -346,7 +347,7 @@ muon_status make_map(CUtensorMap* map, void* base, int inner, int rows, int batc
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %d x %d x %d", static_cast<int>(r),
@@ -710,6 +711,14 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
         st = map_for(&TP.tmA[nprob], xcur, 0, q.c, q.r, q.ldc, q.xstride, 128);
         if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, b_rows);
         if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
+      }
+      // Gram and B'X output rows are written by TMA stores of 32 x 32 boxes
+      // (64-byte swizzle); A*A and the fused update store directly
+      if (st == MUON_OK && (epi == EPI_GRAM || epi == EPI_AXPY)) {
+        const bool sq = (epi == EPI_GRAM);
+        const int out_inner = sq ? q.m : q.c, out_rows = sq ? q.m : q.r, out_ld = sq ? q.ldm : q.ldc;
+        st = make_map(&TP.tmOut[nprob], P.out, out_inner, out_rows, it.count,
+                      static_cast<size_t>(out_ld) * 2, q.xstride, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
       }
       if (st != MUON_OK) return st;
       TP.prob[nprob] = P;
