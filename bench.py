@@ -46,8 +46,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
 # set: same seven shapes, 1 layer instead of 32); see profiles/.
 TRAFFIC_CAPTURES = {
-    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "6136bb94a17f4425",
-                "bytes_per_launch": {"llama_8b_32l": 32 * 1214791808, "llama_8b_1layer": 1214791808},
+    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "42931f97979262fb",
+                "bytes_per_launch": {"llama_8b_32l": 32 * 1288274944, "llama_8b_1layer": 1288274944},
                 "profile": "profiles/tc_gemm_pair_llama_8b_1layer.md"},
 }
 
