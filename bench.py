@@ -46,20 +46,29 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
 # set: same seven shapes, 1 layer instead of 32); see profiles/.
 TRAFFIC_CAPTURES = {
-    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "42931f97979262fb",
+    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "71888fb0e1c511af",
                 "bytes_per_launch": {"llama_8b_32l": 32 * 1288274944, "llama_8b_1layer": 1288274944},
                 "profile": "profiles/tc_gemm_pair_llama_8b_1layer.md"},
 }
 
 
-def captured_traffic(kernel: str, workload: str):
+def source_fingerprint(files) -> str:
+    """sha256 prefix of the kernel sources with comments removed: changes
+    whenever the compiled code can, not when only a comment does."""
     import hashlib
+    import re
+    csrc = os.path.join(ROOT, "muon_polar_orthogonalized_b200", "csrc")
+    text = "".join(open(os.path.join(csrc, f)).read() for f in files)
+    return hashlib.sha256(re.sub(r"//[^\n]*|/\*.*?\*/", "", text, flags=re.S).encode()).hexdigest()[:16]
+
+
+def captured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture, or None once the
+    kernel's sources have changed since that capture."""
     cap = TRAFFIC_CAPTURES.get(kernel)
     if not cap or workload not in cap["bytes_per_launch"]:
         return None
-    csrc = os.path.join(ROOT, "muon_polar_orthogonalized_b200", "csrc")
-    h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in cap["sources"]))
-    if h.hexdigest()[:16] != cap["sha"]:
+    if source_fingerprint(cap["sources"]) != cap["sha"]:
         return None
     return cap["bytes_per_launch"][workload]
 

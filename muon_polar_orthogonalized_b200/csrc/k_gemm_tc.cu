@@ -577,7 +577,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * C::BN);
       // Active chunks form one range [c_lo, c_hi): a symmetric tile skips the
-      // chunks of strictly lower 128-blocks (a prefix) and a ragged tile stops
+      // chunks left of its rows' 256-block (a prefix) and a ragged tile stops
       // at N.  For A*A the A operand of chunk c+1 is loaded while chunk c is
       // combined and stored, so one L2 round trip is in flight at all times;
       // the fused update loads W (prefetched to L2 above) with each chunk; the
