@@ -40,7 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM traffic per launch of a kernel, from one ncu capture of the named
-# kernel sources (sha256 prefix of the files listed).  When the sources differ
+# kernel sources (their fingerprint: sha256 prefix of the files listed with
+# comments removed, source_fingerprint).  When the sources differ
 # from the captured ones the figure no longer describes the kernel and the
 # roofline reports traffic = null.  Captured on the one-layer slice of the 8B
 # shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
@@ -375,7 +376,6 @@ def run_gpu(args):
     prof = api.muon_profiler_read()
     ms_step = ms_total / args.steps
 
-    # ------------------------------------------------------- end to end
     # --------------------------------------------------------- end to end
     # Every step's gradients come from host memory.  They are copied on a copy
     # stream into one of two device gradient buffers while the previous step

@@ -3,6 +3,12 @@
 Argument marshalling only: every step of the optimizer runs in the CUDA
 library.  Tensors must already live on the current CUDA device; streams are
 torch streams (default: the current stream).
+
+The C ABI takes plain pointer arrays and cannot see their lengths or the
+tensors behind them, so the binding checks what it marshals: list lengths
+against the groups, and each tensor's device, dtype, contiguity and element
+count against the layout the library will read and write.  Raw integer
+pointers are passed through unchecked.
 """
 from __future__ import annotations
 
@@ -29,6 +35,47 @@ def _ptrs(tensors) -> ctypes.Array:
     return arr
 
 
+def _group_fields(s) -> Tuple[int, int, int, int, int]:
+    if isinstance(s, MuonGroup):
+        return s.rows, s.cols, s.count, s.first, s.grad_dtype
+    r, c, n, first, dt, _ = s
+    return int(r), int(c), int(n), int(first), int(dt)
+
+
+def _torch_dtype(code: int):
+    import torch
+    return torch.bfloat16 if code == N.MUON_BF16 else torch.float32
+
+
+def _check_tensor(t, what: str, numel: int, dtype) -> None:
+    if isinstance(t, int):
+        return
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous() and t.numel() == numel):
+        raise ValueError(f"{what}: expected a contiguous CUDA {dtype} tensor of {numel} elements, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}"
+                         + ("" if t.is_contiguous() else ", not contiguous"))
+
+
+def _check_group_lists(groups: Sequence, lists) -> None:
+    """lists: (name, tensors, dtype) with dtype None meaning the group's grad dtype."""
+    for s in groups:
+        r, c, n, first, dt = _group_fields(s)
+        if n <= 0 or first < 0:
+            continue   # the library rejects the group itself
+        for name, seq, dtype in lists:
+            if len(seq) < first + n:
+                raise ValueError(f"{name}: {len(seq)} entries, the groups index up to {first + n - 1}")
+            want = _torch_dtype(dt) if dtype is None else dtype
+            for j in range(first, first + n):
+                _check_tensor(seq[j], f"{name}[{j}]", r * c, want)
+
+
+def _check_step_args(groups, params, grads, momentum) -> None:
+    import torch
+    _check_group_lists(groups, (("params", params, torch.float32), ("grads", grads, None),
+                                ("momentum", momentum, torch.float32)))
+
+
 def make_groups(specs: Sequence) -> ctypes.Array:
     arr = (MuonGroup * max(len(specs), 1))()
     for i, s in enumerate(specs):
@@ -48,7 +95,12 @@ def _coeff_array(coeffs, ns_steps: int):
         flat = [float(x) for x in coeffs] * ns_steps
     else:
         for row in list(coeffs)[:ns_steps]:
-            flat.extend(float(x) for x in row)
+            vals = [float(x) for x in row]
+            if len(vals) != 3:
+                raise ValueError("coeffs: every row is one (a, b, c) triple")
+            flat.extend(vals)
+    if len(flat) != 3 * ns_steps:
+        raise ValueError(f"coeffs: {len(flat) // 3} rows of (a, b, c) for ns_steps = {ns_steps}")
     arr = (c_float * len(flat))(*flat)
     return arr
 
@@ -68,6 +120,7 @@ def muon_step(params, grads, momentum, groups: Sequence, lr: float, beta: float,
               stream=None) -> None:
     """One Muon step; see include/muon_b200.h.  params/grads/momentum are lists
     of tensors (or raw pointers) in pointer-array order."""
+    _check_step_args(groups, params, grads, momentum)
     g = make_groups(groups)
     ca = _coeff_array(coeffs, ns_steps)
     wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
@@ -84,6 +137,10 @@ def muon_step_replicated(params, grads, momentum, groups: Sequence, lr: float, b
     """muon_step that also writes each updated matrix into every replica list
     (replicas[r][i] is copy r of params[i]; tensors or raw device pointers,
     possibly in peer GPUs' memory)."""
+    import torch
+    _check_step_args(groups, params, grads, momentum)
+    for r, rep in enumerate(replicas):
+        _check_group_lists(groups, ((f"replicas[{r}]", rep, torch.float32),))
     g = make_groups(groups)
     ca = _coeff_array(coeffs, ns_steps)
     wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
@@ -103,10 +160,16 @@ def muon_reduce_mean(dst: Sequence, sources: Sequence[Sequence], stream=None) ->
     import torch
     if not dst:
         return
+    if dst[0].dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("muon_reduce_mean: tensors must be fp32 or bf16")
     dt = N.MUON_BF16 if dst[0].dtype == torch.bfloat16 else N.MUON_F32
-    for t in list(dst) + [x for src in sources for x in src]:
-        if t.dtype != dst[0].dtype or not t.is_contiguous():
-            raise ValueError("muon_reduce_mean: tensors must be contiguous and share one dtype")
+    for r, src in enumerate(sources):
+        if len(src) != len(dst):
+            raise ValueError(f"muon_reduce_mean: sources[{r}] has {len(src)} tensors, dst {len(dst)}")
+    for i, t in enumerate(dst):
+        _check_tensor(t, f"dst[{i}]", t.numel(), dst[0].dtype)
+        for r, src in enumerate(sources):
+            _check_tensor(src[i], f"sources[{r}][{i}]", t.numel(), dst[0].dtype)
     numel = (c_int64 * len(dst))(*[t.numel() for t in dst])
     rows = [_ptrs(src) for src in sources]
     table = (ctypes.POINTER(c_void_p) * max(len(rows), 1))(
@@ -122,6 +185,7 @@ def muon_step_scheduled(params, grads, momentum, groups: Sequence, lr: float, be
     """muon_step with the learning rate multiplied by the device schedule
     state's lr_mult (schedule_state: a 16-byte device tensor, see
     new_schedule_state)."""
+    _check_step_args(groups, params, grads, momentum)
     g = make_groups(groups)
     ca = _coeff_array(coeffs, ns_steps)
     wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
@@ -165,6 +229,8 @@ def muon_schedule_advance_cosine(schedule_state, total_steps: int, warmup_steps:
 
 def muon_orthogonalize(inputs, outputs, groups: Sequence, ns_steps: int, coeffs, flags: int,
                        workspace, workspace_bytes: Optional[int] = None, stream=None) -> None:
+    import torch
+    _check_group_lists(groups, (("inputs", inputs, None), ("outputs", outputs, torch.float32)))
     g = make_groups(groups)
     ca = _coeff_array(coeffs, ns_steps)
     wsb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
@@ -191,7 +257,18 @@ def _adamw_groups(groups: Sequence[AdamWSpec]):
     n = len(groups)
     arr = (AdamWGroup * max(n, 1))()
     keep = []
+    import torch
     for i, g in enumerate(groups):
+        n_t = len(g.params)
+        for name in ("grads", "exp_avg", "exp_avg_sq"):
+            if len(getattr(g, name)) != n_t:
+                raise ValueError(f"AdamW group {i}: {len(getattr(g, name))} {name} for {n_t} params")
+        for k, t in enumerate(g.params):
+            ne = t.numel()
+            _check_tensor(t, f"AdamW group {i} params[{k}]", ne, torch.float32)
+            _check_tensor(g.grads[k], f"AdamW group {i} grads[{k}]", ne, _torch_dtype(int(g.grad_dtype)))
+            _check_tensor(g.exp_avg[k], f"AdamW group {i} exp_avg[{k}]", ne, torch.float32)
+            _check_tensor(g.exp_avg_sq[k], f"AdamW group {i} exp_avg_sq[{k}]", ne, torch.float32)
         p, gr, m, v = _ptrs(g.params), _ptrs(g.grads), _ptrs(g.exp_avg), _ptrs(g.exp_avg_sq)
         numel = (c_int64 * max(len(g.params), 1))(*[t.numel() for t in g.params])
         keep.extend([p, gr, m, v, numel])

@@ -64,14 +64,26 @@ class MuonAdamW:
                 exp_avg=[torch.zeros_like(p) for p in ps],
                 exp_avg_sq=[torch.zeros_like(p) for p in ps]))
         self.step_count = 0
-        ws_need = api.muon_workspace_size(self._groups(torch.float32), self.flags) if self.muon_params else 0
+        ws_need = api.muon_workspace_size(self._groups([torch.float32] * len(self._shapes)), self.flags) \
+            if self.muon_params else 0
         nbytes = ws_need if workspace_bytes is None else max(int(workspace_bytes), 0)
         dev = self.muon_params[0].device if self.muon_params else torch.device("cuda")
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
 
-    def _groups(self, grad_dtype):
-        dt = N.MUON_BF16 if grad_dtype == torch.bfloat16 else N.MUON_F32
-        return [(r, c, n, first, dt, ls) for (r, c, n, first, ls) in self._shapes]
+    def _groups(self, grad_dtypes):
+        """Group descriptors, one gradient dtype per shape group."""
+        return [(r, c, n, first, N.MUON_BF16 if dt == torch.bfloat16 else N.MUON_F32, ls)
+                for (r, c, n, first, ls), dt in zip(self._shapes, grad_dtypes)]
+
+    def _grad_dtypes(self, grads):
+        """The gradient dtype of each shape group (fp32 or bf16, uniform within a group)."""
+        out = []
+        for (r, c, n, first, _) in self._shapes:
+            dts = {grads[k].dtype for k in range(first, first + n)}
+            if len(dts) != 1 or not dts <= {torch.float32, torch.bfloat16}:
+                raise ValueError(f"the grads of the {r}x{c} Muon matrices must all be fp32 or all bf16")
+            out.append(dts.pop())
+        return out
 
     @torch.no_grad()
     def step(self, stream=None, replicas: Optional[Sequence[Sequence[torch.Tensor]]] = None) -> None:
@@ -84,9 +96,7 @@ class MuonAdamW:
             grads = [p.grad for p in self.muon_params]
             if any(g is None for g in grads):
                 raise ValueError("every Muon parameter needs a .grad")
-            gd = grads[0].dtype
-            if any(g.dtype != gd for g in grads):
-                raise ValueError("Muon grads must share one dtype")
+            gd = self._grad_dtypes(grads)
             if replicas:
                 reps = [[rep[k] for k in self._order] for rep in replicas]
                 api.muon_step_replicated(self.muon_params, grads, self.momentum, self._groups(gd), self.lr,
@@ -107,14 +117,32 @@ class MuonAdamW:
             api.adamw_step(specs, self.step_count, stream=stream)
 
     def state_dict(self) -> dict:
+        """Step count and optimizer state; "momentum" follows the order in
+        which the Muon parameters were given, not the internal grouping."""
+        mom: List[Optional[torch.Tensor]] = [None] * len(self.momentum)
+        for k, pos in enumerate(self._order):
+            mom[pos] = self.momentum[k].clone()
         return {"step": self.step_count,
-                "momentum": [m.clone() for m in self.momentum],
+                "momentum": mom,
                 "exp_avg": [[t.clone() for t in g["exp_avg"]] for g in self.adamw_groups],
                 "exp_avg_sq": [[t.clone() for t in g["exp_avg_sq"]] for g in self.adamw_groups]}
 
     def load_state_dict(self, sd: dict) -> None:
+        """Restore a state_dict of an optimizer over parameters of the same
+        shapes, given in the same order; nothing is changed if it does not fit."""
+        def fits(dst: List[torch.Tensor], src, what: str) -> None:
+            if len(src) != len(dst) or any(tuple(a.shape) != tuple(b.shape) for a, b in zip(dst, src)):
+                raise ValueError(f"state_dict: {what} does not match this optimizer's parameters")
+        mom_internal = [sd["momentum"][pos] for pos in self._order] \
+            if len(sd["momentum"]) == len(self.momentum) else sd["momentum"]
+        fits(self.momentum, mom_internal, "momentum")
+        if len(sd["exp_avg"]) != len(self.adamw_groups) or len(sd["exp_avg_sq"]) != len(self.adamw_groups):
+            raise ValueError("state_dict: AdamW group count does not match")
+        for g, ea, es in zip(self.adamw_groups, sd["exp_avg"], sd["exp_avg_sq"]):
+            fits(g["exp_avg"], ea, "exp_avg")
+            fits(g["exp_avg_sq"], es, "exp_avg_sq")
         self.step_count = int(sd["step"])
-        for dst, src in zip(self.momentum, sd["momentum"]):
+        for dst, src in zip(self.momentum, mom_internal):
             dst.copy_(src)
         for g, ea, es in zip(self.adamw_groups, sd["exp_avg"], sd["exp_avg_sq"]):
             for dst, src in zip(g["exp_avg"], ea):

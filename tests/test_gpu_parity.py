@@ -866,3 +866,32 @@ def test_status_word_ok_after_step(dev):
     ws = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
     api.muon_step(W, G, M, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws)
     assert api.muon_query_status(ws) == N.MUON_OK
+
+
+def test_mixed_grad_dtypes_and_state_dict_order(dev):
+    """Shape groups may carry different gradient dtypes (each group is stepped
+    exactly as alone), and state_dict lists momentum in the order the
+    parameters were given, although the optimizer groups them by shape."""
+    torch.manual_seed(5)
+    shapes = [(128, 256), (256, 128), (128, 256)]   # internal order: 0, 2 | 1
+    mats = [torch.randn(s, device=dev) * 0.02 for s in shapes]
+    twins = [m.clone() for m in mats]
+    grads = [torch.randn(s, device=dev) for s in shapes]
+    grads[0], grads[2] = grads[0].to(torch.bfloat16), grads[2].to(torch.bfloat16)
+    opt = MuonAdamW(mats)
+    for m, g in zip(mats, grads):
+        m.grad = g
+    opt.step()
+    alone_a, alone_b = MuonAdamW([twins[0], twins[2]]), MuonAdamW([twins[1]])
+    for m, g in zip(twins, grads):
+        m.grad = g
+    alone_a.step()
+    alone_b.step()
+    for x, y in zip(mats, twins):
+        assert torch.equal(x, y)
+    sd = opt.state_dict()
+    for k in range(3):   # one step from zero momentum: m = G
+        assert torch.equal(sd["momentum"][k], grads[k].float())
+    with pytest.raises(ValueError, match="momentum"):
+        opt.load_state_dict(dict(sd, momentum=sd["momentum"][:2]))
+    opt.load_state_dict(sd)

@@ -205,3 +205,43 @@ def test_schedule_validation(L):
     n = (ctypes.c_int64 * 1)(16)
     g = N.AdamWGroup(p, p, p, p, n, 1, 0, 1e-3, 0.9, 0.95, 1e-8, 0.0)
     assert L.adamw_step_scheduled(ctypes.byref(g), 1, None, None) == N.MUON_ERR_INVALID_ARG
+
+
+# ------------------------------------------------ binding-side validation
+# The C ABI receives bare pointer arrays; the Python binding checks list
+# lengths, coefficient rows and tensor layouts before the call, so that a
+# short list or a wrong dtype never reaches the library.  Raw integer
+# pointers pass through unchecked (fake addresses here: nothing is launched).
+
+GROUPS = [(4, 8, 2, 0, N.MUON_F32, 1.0)]
+FAKE = [0x100000, 0x200000]
+
+
+def test_binding_rejects_short_coefficient_table():
+    with pytest.raises(ValueError, match="coeffs"):
+        api.muon_step(FAKE, FAKE, FAKE, GROUPS, 0.02, 0.95, 0.0, 3,
+                      [(3.4445, -4.7750, 2.0315)] * 2, 0, 0x300000, workspace_bytes=1 << 20)
+    with pytest.raises(ValueError, match="triple"):
+        api.muon_step(FAKE, FAKE, FAKE, GROUPS, 0.02, 0.95, 0.0, 1, [(1.0, 2.0)], 0, 0x300000,
+                      workspace_bytes=1 << 20)
+
+
+def test_binding_rejects_short_pointer_lists():
+    with pytest.raises(ValueError, match="grads: 1 entries"):
+        api.muon_step(FAKE, FAKE[:1], FAKE, GROUPS, 0.02, 0.95, 0.0, 0, None, 0, 0x300000,
+                      workspace_bytes=1 << 20)
+    with pytest.raises(ValueError, match=r"replicas\[0\]"):
+        api.muon_step_replicated(FAKE, FAKE, FAKE, GROUPS, 0.02, 0.95, 0.0, 0, None, 0, 0x300000,
+                                 [FAKE[:1]], workspace_bytes=1 << 20)
+
+
+def test_binding_rejects_tensors_the_library_would_misread():
+    import torch
+    cpu = [torch.zeros(4, 8), torch.zeros(4, 8)]
+    with pytest.raises(ValueError, match=r"params\[0\].*CUDA"):
+        api.muon_step(cpu, FAKE, FAKE, GROUPS, 0.02, 0.95, 0.0, 0, None, 0, 0x300000,
+                      workspace_bytes=1 << 20)
+    spec = api.AdamWSpec([torch.zeros(8)], [torch.zeros(8)], [torch.zeros(8)], [], 1e-3, 0.9, 0.95,
+                         1e-8, 0.0)
+    with pytest.raises(ValueError, match="exp_avg_sq"):
+        api.adamw_step([spec], 1)
