@@ -84,6 +84,7 @@ enum {
 /*
  * One shape group: `count` matrices of rows x cols (parameter orientation),
  * the pointers params[first .. first+count-1] (same for grads, momentum).
+ * The groups of one call index disjoint ranges (else MUON_ERR_INVALID_ARG).
  * A group with rows > cols is iterated as its transpose ("Polar Express"
  * orientation); no physical transpose is made: the kernels read it
  * MN-major.

@@ -262,6 +262,20 @@ muon_status validate_groups(const muon_group* groups, int n_groups) {
     if (g.grad_dtype != MUON_F32 && g.grad_dtype != MUON_BF16)
       return fail(MUON_ERR_INVALID_ARG, "group %d: grad_dtype %d unknown", i, g.grad_dtype);
     if (!std::isfinite(g.lr_scale)) return fail(MUON_ERR_INVALID_ARG, "group %d: lr_scale not finite", i);
+    if (static_cast<long long>(g.first) + g.count > (1ll << 30))
+      return fail(MUON_ERR_INVALID_ARG, "group %d: first + count too large", i);
+  }
+  // the groups' pointer ranges [first, first + count) must not overlap: one
+  // matrix in two groups would be updated twice by concurrent kernels
+  std::vector<std::pair<int, int>> ranges;
+  for (int i = 0; i < n_groups; ++i)
+    if (groups[i].count > 0) ranges.emplace_back(groups[i].first, i);
+  std::sort(ranges.begin(), ranges.end());
+  for (size_t k = 1; k < ranges.size(); ++k) {
+    const muon_group& prev = groups[ranges[k - 1].second];
+    if (prev.first + prev.count > ranges[k].first)
+      return fail(MUON_ERR_INVALID_ARG, "groups %d and %d index overlapping pointer ranges", ranges[k - 1].second,
+                  ranges[k].second);
   }
   return MUON_OK;
 }

@@ -75,6 +75,7 @@ def _call_step(L, groups, ptr_count, ns=5, coeffs=True, flags=3, ws=0x1000, wsb=
     (dict(groups=[(4, 4, 1, 0, 7, 1.0)]), N.MUON_ERR_INVALID_ARG),          # dtype
     (dict(groups=[(4, 4, 1, 0, 0, float("nan"))]), N.MUON_ERR_INVALID_ARG),  # lr_scale
     (dict(groups=[(70000, 4, 1, 0, 0, 1.0)]), N.MUON_ERR_INVALID_ARG),      # too large
+    (dict(groups=[(4, 8, 2, 0, 0, 1.0), (8, 8, 1, 1, 0, 1.0)]), N.MUON_ERR_INVALID_ARG),  # overlap
     (dict(ns=17), N.MUON_ERR_INVALID_ARG),
     (dict(ns=-1), N.MUON_ERR_INVALID_ARG),
     (dict(coeffs=False), N.MUON_ERR_INVALID_ARG),
