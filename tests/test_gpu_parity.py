@@ -878,13 +878,16 @@ def test_mixed_grad_dtypes_and_state_dict_order(dev):
     twins = [m.clone() for m in mats]
     grads = [torch.randn(s, device=dev) for s in shapes]
     grads[0], grads[2] = grads[0].to(torch.bfloat16), grads[2].to(torch.bfloat16)
+    def set_grads(ps):
+        for m, g in zip(ps, grads):
+            m.grad_dtype = g.dtype   # a bf16 .grad on an fp32 parameter must be declared
+            m.grad = g
+
     opt = MuonAdamW(mats)
-    for m, g in zip(mats, grads):
-        m.grad = g
+    set_grads(mats)
     opt.step()
     alone_a, alone_b = MuonAdamW([twins[0], twins[2]]), MuonAdamW([twins[1]])
-    for m, g in zip(twins, grads):
-        m.grad = g
+    set_grads(twins)
     alone_a.step()
     alone_b.step()
     for x, y in zip(mats, twins):
