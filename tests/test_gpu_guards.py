@@ -78,3 +78,37 @@ def test_step_never_reads_unwritten_workspace(dev, extra):
         results.append([t.clone() for t in W + M])
     for a, b in zip(*results):
         assert torch.equal(a, b)
+
+
+def test_orthogonalize_and_adamw_write_nothing_outside(dev):
+    """The orthogonaliser on the edge shapes (including 1-row and 1-column
+    matrices) and AdamW on tensors whose lengths are not multiples of 4."""
+    from tests.test_gpu_parity import EDGE_SHAPES
+    bands = []
+
+    def guard(t):
+        buf, view = guarded_copy(t)
+        bands.append((buf, t.numel() * t.element_size()))
+        return view
+
+    groups = [(r, c, 1, k, N.MUON_BF16, 1.0) for k, (r, c) in enumerate(EDGE_SHAPES)]
+    inputs = [guard(torch.randn(r, c, device=dev).to(torch.bfloat16)) for r, c in EDGE_SHAPES]
+    outs = [guard(torch.zeros(r, c, device=dev)) for r, c in EDGE_SHAPES]
+    need = api.muon_workspace_size(groups, 0)
+    wbuf = torch.full((2 * GUARD_BYTES + need,), CANARY, dtype=torch.uint8, device=dev)
+    ws = wbuf[GUARD_BYTES:GUARD_BYTES + need]
+    api.muon_orthogonalize(inputs, outs, groups, 5, FIXED, 0, ws)
+
+    numels = [17, 1000, 4099, 65539]
+    P = [guard(torch.randn(n, device=dev) * 0.02) for n in numels]
+    Gr = [guard(torch.randn(n, device=dev).to(torch.bfloat16)) for n in numels]
+    Ma = [guard(torch.zeros(n, device=dev)) for n in numels]
+    Va = [guard(torch.zeros(n, device=dev)) for n in numels]
+    spec = api.AdamWSpec(P, Gr, Ma, Va, 3e-4, 0.9, 0.95, 1e-8, 0.1)
+    for t in (1, 2):
+        api.adamw_step([spec], t)
+    torch.cuda.synchronize()
+    assert api.muon_query_status(ws) == N.MUON_OK
+    assert all(bool(torch.isfinite(o).all()) for o in outs)
+    for k, (buf, nbytes) in enumerate(bands + [(wbuf, need)]):
+        assert canaries_intact(buf, nbytes), f"guard band {k} overwritten"
