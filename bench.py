@@ -47,20 +47,24 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
 # set: same seven shapes, 1 layer instead of 32); see profiles/.
 TRAFFIC_CAPTURES = {
-    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "71888fb0e1c511af",
+    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "2e92259ec58a2537",
                 "bytes_per_launch": {"llama_8b_32l": 32 * 1288274944, "llama_8b_1layer": 1288274944},
                 "profile": "profiles/tc_gemm_pair_llama_8b_1layer.md"},
 }
 
 
 def source_fingerprint(files) -> str:
-    """sha256 prefix of the kernel sources with comments removed: changes
-    whenever the compiled code can, not when only a comment does."""
+    """sha256 prefix of the kernel sources with comments, blank lines and
+    trailing blanks removed: changes whenever the compiled code can, not when
+    only a comment does."""
     import hashlib
     import re
     csrc = os.path.join(ROOT, "muon_polar_orthogonalized_b200", "csrc")
     text = "".join(open(os.path.join(csrc, f)).read() for f in files)
-    return hashlib.sha256(re.sub(r"//[^\n]*|/\*.*?\*/", "", text, flags=re.S).encode()).hexdigest()[:16]
+    text = re.sub(r"//[^\n]*|/\*.*?\*/", "", text, flags=re.S)
+    # what is left of comment-only lines, and trailing blanks, do not count
+    code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def captured_traffic(kernel: str, workload: str):

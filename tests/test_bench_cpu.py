@@ -1,0 +1,69 @@
+"""Host-side checks of the benchmark's bookkeeping (no GPU).
+
+  * the algorithmic work it divides by, against totals written out by hand
+    for the 8B-shaped set (parameter counts, nominal Newton-Schulz FLOPs,
+    bytes per parameter of each HBM-bound kernel);
+  * the one-layer slice is exactly 1/32 of the 32-layer set, which the
+    scaled DRAM-traffic figure relies on;
+  * the source fingerprint that guards the captured DRAM traffic ignores
+    comments and changes with code.
+"""
+import os
+import shutil
+
+import bench
+from muon_polar_orthogonalized_b200 import workloads as wl
+
+# 8B shapes, written out: per layer Wq, Wo 4096x4096; Wk, Wv 1024x4096;
+# gate, up 14336x4096; down 4096x14336; 32 layers; AdamW on two 128256x4096
+# tables; bf16 gradients everywhere.
+PER_LAYER = [(4096, 4096)] * 2 + [(1024, 4096)] * 2 + [(14336, 4096)] * 2 + [(4096, 14336)]
+
+
+def test_algorithmic_work_of_the_8b_set():
+    w = wl.get("llama_8b_32l")
+    work = bench.algorithmic_work(w)
+    params = 32 * sum(r * c for r, c in PER_LAYER)
+    assert params == 6_979_321_856 == w.muon_params()
+    flops = 0
+    for r, c in PER_LAYER:
+        m, n = min(r, c), max(r, c)
+        flops += 32 * (4 * m * m * n + 2 * m ** 3)   # one quintic iteration, nominal
+    nominal = 5 * flops
+    assert abs(nominal - 665.9e12) < 0.05e12
+    got = 5 * (work["gram_flops"] + work["poly_flops"] + work["axpy_flops"])
+    assert got == nominal == w.ns_flops_nominal()
+    # momentum: bf16 G in (2), fp32 m in and out (8), bf16 X0 out (2)
+    assert work["momentum_bytes"] == 12 * params
+    # unfused update: bf16 U in (2), fp32 W in and out (8)
+    assert work["update_bytes"] == 10 * params
+    # AdamW: bf16 g in (2); fp32 p, m, v in and out (24)
+    adam_params = 2 * 128256 * 4096
+    assert work["adamw_bytes"] == 26 * adam_params
+
+
+def test_one_layer_slice_is_a_thirty_second_of_the_set():
+    full, one = wl.get("llama_8b_32l"), wl.get("llama_8b_1layer")
+    a, b = bench.algorithmic_work(full), bench.algorithmic_work(one)
+    for k in ("gram_flops", "poly_flops", "axpy_flops", "momentum_bytes", "update_bytes"):
+        assert a[k] == 32 * b[k], k
+    cap = bench.TRAFFIC_CAPTURES["ns_axpy"]["bytes_per_launch"]
+    assert cap["llama_8b_32l"] == 32 * cap["llama_8b_1layer"]
+
+
+def test_source_fingerprint_ignores_comments_only(tmp_path, monkeypatch):
+    src = os.path.join(bench.ROOT, "muon_polar_orthogonalized_b200", "csrc")
+    dst = tmp_path / "muon_polar_orthogonalized_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    files = bench.TRAFFIC_CAPTURES["ns_axpy"]["sources"]
+    base = bench.source_fingerprint(files)
+    assert base == bench.TRAFFIC_CAPTURES["ns_axpy"]["sha"]
+    assert bench.captured_traffic("ns_axpy", "llama_8b_32l") is not None
+    f = dst / files[0]
+    text = f.read_text()
+    f.write_text("// a comment line\n/* and a\n   block comment */\n" + text)
+    assert bench.source_fingerprint(files) == base
+    f.write_text(text.replace("namespace muon {", "namespace muon {\nconstexpr int kProbe = 1;", 1))
+    assert bench.source_fingerprint(files) != base
+    assert bench.captured_traffic("ns_axpy", "llama_8b_32l") is None
