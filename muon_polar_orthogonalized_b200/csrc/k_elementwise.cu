@@ -24,6 +24,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "elt_params.cuh"
 
@@ -942,16 +944,17 @@ static cudaError_t launch_rowq(const EltParams& p, int cls, int sms, cudaStream_
     return cudaGetLastError();
   }
   auto k = momentum_rowq_kernel<GBF16>;
-  static bool attr_set[64] = {};  // per device (the attribute is per device)
+  // the attribute is set once per device; concurrent callers may both set it
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowEqSmemCols * 4)) !=
         cudaSuccess)
       return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   int cols = 0;
   for (int i = 0; i < p.nmats; ++i)
