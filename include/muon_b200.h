@@ -317,10 +317,21 @@ const char* muon_status_string(muon_status s);
 const char* muon_last_error(void);
 
 /*
- * Optional per-kernel timing.  When enabled, every launch is bracketed by
- * CUDA events on its own stream.  muon_profiler_read synchronises on those
- * events and writes, per kernel kind, the summed device milliseconds and the
- * launch count since the last reset; it returns the number of kinds.
+ * Optional per-kernel timing (no counterpart on the optimizer pages; it
+ * feeds the benchmark's per-kernel rooflines).  Process-wide state, guarded
+ * by a lock.  While enabled, every launch of the library is bracketed by
+ * CUDA events on its own stream (the events come from a pool the library
+ * owns; enabling adds two event records per launch and nothing else).
+ *   muon_profiler_enable   on != 0 enables; returns the previous setting.
+ *   muon_profiler_reset    waits for the recorded events, then clears.
+ *   muon_profiler_read     waits for the recorded events and writes, for
+ *                          kinds 0 .. min(max_kinds, kind count) - 1, the summed
+ *                          device milliseconds and launch counts since the
+ *                          last reset into the caller's host arrays (either
+ *                          may be NULL); returns the kind count.
+ *   muon_kernel_kind_count / muon_kernel_kind_name   the kinds' names ("" for
+ *                          an index out of range); static strings.
+ * Do not enable it while a stream is being captured into a CUDA graph.
  */
 int muon_profiler_enable(int on);
 void muon_profiler_reset(void);
