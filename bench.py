@@ -103,16 +103,21 @@ class ClockSampler:
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
+        out = open(self.path, "w")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                stdout=out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        finally:
+            out.close()   # the sampler process holds its own descriptor
 
     def stop(self):
         if self.proc is None:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         try:

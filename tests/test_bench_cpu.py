@@ -67,3 +67,46 @@ def test_source_fingerprint_ignores_comments_only(tmp_path, monkeypatch):
     f.write_text(text.replace("namespace muon {", "namespace muon {\nconstexpr int kProbe = 1;", 1))
     assert bench.source_fingerprint(files) != base
     assert bench.captured_traffic("ns_axpy", "llama_8b_32l") is None
+
+
+def test_clock_sampler_reads_clocks_and_throttle_reasons(monkeypatch):
+    """Median SM clock over the samples that parse, the highest max clock,
+    and every throttle reason seen active (nvidia-smi faked)."""
+    lines = ["0, 1241, 1965, 985.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+             "0, 1300, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+             "0, [N/A], 1965, 990.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+             "0, 1100, 1965, 700.0, 0x0000000000000040, Not Active, Active, Not Active, Not Active",
+             "truncated line"]
+
+    class FakeSmi:
+        def __init__(self, args, stdout=None, stderr=None):
+            assert "--query-gpu=" + bench.ClockSampler.FIELDS in args
+            stdout.write("\n".join(lines) + "\n")
+            stdout.flush()
+
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+        def kill(self):
+            pass
+
+    monkeypatch.setattr(bench.subprocess, "Popen", FakeSmi)
+    sampler = bench.ClockSampler(0)
+    sampler.start()
+    got = sampler.stop()
+    assert got["sm_mhz"] == 1241.0 and got["sm_max_mhz"] == 1965.0 and got["samples"] == 3
+    assert got["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi(monkeypatch):
+    def no_smi(*a, **k):
+        raise FileNotFoundError("nvidia-smi")
+
+    monkeypatch.setattr(bench.subprocess, "Popen", no_smi)
+    sampler = bench.ClockSampler(0)
+    sampler.start()
+    got = sampler.stop()
+    assert got["sm_mhz"] is None and got["reasons"] == ["nvidia-smi unavailable"]
