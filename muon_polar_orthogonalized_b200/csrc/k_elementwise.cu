@@ -35,9 +35,10 @@ namespace muon {
 // the momentum / update kernels stream 2-3 arrays and run best at full
 // occupancy (8 x 256 threads per SM) with 2 vec4 units per thread; AdamW
 // streams 4 arrays and runs best with 4 units per thread at 4 blocks per SM.
-// At that budget (64 registers) ptxas keeps about 200 bytes per AdamW thread
-// in local memory; the 2-block shape (128 registers, no spill) measured
-// slower.  The untried next step is 3 blocks.
+// At that budget (64 registers for 1024 threads per SM) ptxas keeps about 200
+// bytes per AdamW thread in local memory; 2 blocks of 512 threads (the same
+// budget) measured alike.  A budget without the spill (fewer threads per SM)
+// has not been measured yet.
 #ifndef MUON_ELT_UNROLL
 #define MUON_ELT_UNROLL 2
 #endif
