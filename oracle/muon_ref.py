@@ -307,7 +307,8 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 
 
 def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: int = 5,
-                                eps: float = NS_EPS, fold_a: bool = False) -> np.ndarray:
+                                eps: float = NS_EPS, fold_a: bool = False, exact_diag: bool = False,
+                                rounding=None) -> np.ndarray:
     """The iteration with bf16 rounding wherever a bf16 matrix is stored.
 
     [MAC] casts to bf16 before iterating and keeps X, A, B in bf16.  Storage
@@ -318,25 +319,39 @@ def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: in
 
     fold_a: the stored B holds a on its diagonal, B' = bf16(a I + b A + c A A),
     and X' = bf16(B' X): the same algebra, a*X + B X = (a I + B) X, with the
-    rounding moved, as a kernel that folds a into B stores it.
+    rounding moved.
+    exact_diag (with fold_a): the part of B''s diagonal that bf16 cannot hold,
+    lo_i = d_i - bf16(d_i), is kept unrounded beside the stored B' and added
+    back as lo_i * X_ij, so X' = bf16(B' X + lo * X): B' keeps its diagonal
+    exactly and only its off-diagonal entries are rounded.
+    rounding: the function applied at every storage point (round_bf16 by
+    default); the identity turns every mode into the exact iteration.
     """
+    rnd = round_bf16 if rounding is None else rounding
+    if exact_diag and not fold_a:
+        raise ValueError("exact_diag applies to the folded B'")
     g = np.asarray(g, dtype=np.float64)
     s = 1.0 / (np.sqrt(np.sum(g * g)) + eps)
-    x = round_bf16(g)
+    x = rnd(g)
     transposed = x.shape[0] > x.shape[1]
     if transposed:
         x = x.T
     for k, (a, b, c) in enumerate(_coeff_list(coeffs, steps)):
         sk = s if k == 0 else 1.0
-        A = round_bf16(sk * sk * (x @ x.T))
+        A = rnd(sk * sk * (x @ x.T))
         if fold_a:
-            B = round_bf16(a * np.eye(A.shape[0]) + b * A + c * (A @ A))
-            x = round_bf16(sk * (B @ x))
+            Bfull = a * np.eye(A.shape[0]) + b * A + c * (A @ A)
+            B = rnd(Bfull)
+            if exact_diag:
+                lo = np.diag(Bfull) - np.diag(B)
+                x = rnd(sk * (B @ x + lo[:, None] * x))
+            else:
+                x = rnd(sk * (B @ x))
         else:
-            B = round_bf16(b * A + c * (A @ A))
-            x = round_bf16(sk * (a * x + B @ x))
+            B = rnd(b * A + c * (A @ A))
+            x = rnd(sk * (a * x + B @ x))
     if steps == 0:
-        x = round_bf16(s * x)
+        x = rnd(s * x)
     if transposed:
         x = x.T
     return np.ascontiguousarray(x)

@@ -233,13 +233,69 @@ def test_torch_muon_cross_check(pages):
     assert abs(np.linalg.norm(upd_t) / np.linalg.norm(u) - 1) < 0.05
 
 
-def test_bf16_emulation_close_to_fp64():
+EMUL_MODES = {"pages": {}, "fold_a": {"fold_a": True},
+              "fold_a_exact_diag": {"fold_a": True, "exact_diag": True}}
+
+
+@pytest.mark.parametrize("mode", list(EMUL_MODES))
+def test_bf16_emulation_close_to_fp64(mode):
     """Diagnostic mode stays within the bf16 tolerance of the fp64 oracle."""
+    kw = EMUL_MODES[mode]
     g = wl.iid_normal((64, 256), 1.0, 3)
-    e = _rel(oracle.newton_schulz_bf16_emulated(g), oracle.newton_schulz(g))
+    e = _rel(oracle.newton_schulz_bf16_emulated(g, **kw), oracle.newton_schulz(g))
     assert 1e-4 < e < 2e-2
     gt = g.T.copy()
-    assert _rel(oracle.newton_schulz_bf16_emulated(gt), oracle.newton_schulz(gt)) < 2e-2
+    assert _rel(oracle.newton_schulz_bf16_emulated(gt, **kw), oracle.newton_schulz(gt)) < 2e-2
+
+
+@pytest.mark.parametrize("mode", list(EMUL_MODES))
+def test_bf16_emulation_algebra_is_exact(mode):
+    """With rounding switched off, each storage layout is an exact rewriting
+    of the pages' iteration (deferred scale; a*X + B X = (a I + B) X; the
+    diagonal split B' = bf16(B') + diag(lo)), so it must reproduce the fp64
+    oracle -- itself pinned to the SVD closed form -- on wide, tall and
+    ragged inputs, for several step counts and a per-step table."""
+    kw = EMUL_MODES[mode]
+    table = np.array([[3.0, -3.2, 1.2], [2.5, -2.0, 0.6], [1.875, -1.25, 0.375]])
+    for shape, seed in [((24, 80), 1), ((80, 24), 2), ((33, 33), 3)]:
+        g = wl.iid_normal(shape, 1.0, seed)
+        for steps, coeffs in [(0, oracle.NS_COEFFS_FIXED), (1, oracle.NS_COEFFS_FIXED),
+                              (5, oracle.NS_COEFFS_FIXED), (3, table)]:
+            got = oracle.newton_schulz_bf16_emulated(g, coeffs, steps, rounding=lambda x: x, **kw)
+            assert _rel(got, oracle.newton_schulz(g, coeffs, steps)) < 1e-12, (mode, shape, steps)
+
+
+def test_bf16_emulation_first_order_bound_on_diagonal_input():
+    """One step on a diagonal input with bf16-exact entries: every matrix
+    stays diagonal and each stored value carries a relative rounding error of
+    at most u = 2^-8, so with t = s*sigma, q = b t^2 + c t^4 the first-order
+    error of the new diagonal against p(t) = t (a + q) is at most
+      pages:      t u (|a + q| + |b| t^2 + 2|c| t^4 + |q|)     (A, B, X' rounded)
+      fold_a:     t u (2|a + q| + |b| t^2 + 2|c| t^4)          (A, B', X' rounded)
+      exact_diag: t u (|a + q| + |b| t^2 + 2|c| t^4)           (A, X' rounded)
+    (times 1 + 4u for the second-order terms).  Each mode must stay inside its
+    own bound; folding without the exact diagonal must leave the exact-diagonal
+    bound somewhere (the diagonal of B' is then rounded)."""
+    u = 2.0 ** -8
+    a, b, c = oracle.NS_COEFFS_FIXED
+    sig = oracle.round_bf16(np.geomspace(1.0, 1e-2, 256) * (1.0 + np.arange(256) % 7 / 64.0))
+    assert np.array_equal(oracle.round_bf16(sig), sig)
+    G = np.diag(sig)
+    s = 1.0 / (np.sqrt(np.sum(sig * sig)) + oracle.NS_EPS)
+    t = s * sig
+    q = b * t ** 2 + c * t ** 4
+    common = abs(b) * t ** 2 + 2 * abs(c) * t ** 4
+    bound = {"pages": t * u * (np.abs(a + q) + common + np.abs(q)) * (1 + 4 * u),
+             "fold_a": t * u * (2 * np.abs(a + q) + common) * (1 + 4 * u),
+             "fold_a_exact_diag": t * u * (np.abs(a + q) + common) * (1 + 4 * u)}
+    err = {}
+    for mode, kw in EMUL_MODES.items():
+        x = oracle.newton_schulz_bf16_emulated(G, steps=1, **kw)
+        assert np.count_nonzero(x - np.diag(np.diag(x))) == 0
+        err[mode] = np.abs(np.diag(x) - t * (a + q))
+        assert np.all(err[mode] <= bound[mode]), mode
+        assert err[mode].max() > 0.05 * bound[mode].max(), mode   # it does round
+    assert np.any(err["fold_a"] > bound["fold_a_exact_diag"])
 
 
 def test_round_bf16_rne():
