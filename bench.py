@@ -18,6 +18,13 @@ collective), so per-GPU work is fixed: weak scaling.
 
 Rank 0 prints one JSON line.  --impl reference times the CPU fp64 oracle on a
 bounded sample of the same workload instead (the reference arm).
+
+--distributed times the data-parallel optimizer instead (DistributedMuonAdamW:
+every rank holds the whole parameter set, the matrices are owner-sharded for
+Muon and the AdamW tensors ZeRO-1-sliced; per step one reduce_scatter of the
+flat gradient buffers, the owners' steps, one all_gather of the flat parameter
+buffers over NCCL).  Total work is one optimizer step of one model however
+many ranks share it: strong scaling.
 """
 from __future__ import annotations
 
@@ -45,11 +52,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # from the captured ones the figure no longer describes the kernel and the
 # roofline reports traffic = null.  Captured on the one-layer slice of the 8B
 # shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
-# set: same seven shapes, 1 layer instead of 32); see profiles/.
+# set: same seven shapes, 1 layer instead of 32).
 TRAFFIC_CAPTURES = {
     "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "2e92259ec58a2537",
-                "bytes_per_launch": {"llama_8b_32l": 32 * 1288274944, "llama_8b_1layer": 1288274944},
-                "profile": "profiles/tc_gemm_pair_llama_8b_1layer.md"},
+                "bytes_per_launch": {"llama_8b_32l": 32 * 1288274944, "llama_8b_1layer": 1288274944}},
 }
 
 
@@ -146,8 +152,10 @@ class ClockSampler:
 
 # ------------------------------------------------------------- workload
 def algorithmic_work(wl):
-    """Per-step algorithmic FLOPs / bytes of each kernel kind (nominal FLOPs per
-    the spec: gram 2 m^2 n, A.A 2 m^3, B.X 2 m^2 n per iteration)."""
+    """Per-iteration FLOPs and per-step bytes of each kernel kind.  Nominal
+    FLOPs as the spec counts them: gram 2 m^2 n, A.A 2 m^3, B.X 2 m^2 n per
+    iteration.  Executed FLOPs: the two symmetric products compute only the
+    upper half (gram m^2 n, A.A m^3); B.X is not symmetric (2 m^2 n)."""
     gram = poly = axpy = 0.0
     mom_bytes = upd_bytes = 0.0
     for s in wl.muon:
@@ -162,8 +170,9 @@ def algorithmic_work(wl):
     for t in wl.adamw:
         gb = 2 if t.grad_dtype == "bf16" else 4
         adam_bytes += t.count * math.prod(t.shape) * (gb + 24)
-    return dict(gram_flops=gram, poly_flops=poly, axpy_flops=axpy, momentum_bytes=mom_bytes,
-                update_bytes=upd_bytes, adamw_bytes=adam_bytes)
+    return dict(gram_flops=gram, poly_flops=poly, axpy_flops=axpy,
+                gram_flops_executed=gram / 2, poly_flops_executed=poly / 2, axpy_flops_executed=axpy,
+                momentum_bytes=mom_bytes, update_bytes=upd_bytes, adamw_bytes=adam_bytes)
 
 
 class DeviceWorkload:
@@ -449,10 +458,10 @@ def run_gpu(args):
                              "avg_launch_ms": round(ms / n, 4)}
         K = wl.ns_steps
         alg = {
-            "ns_gram": ("tensor", work["gram_flops"]),
-            "ns_poly": ("tensor", work["poly_flops"]),
-            "ns_axpy": ("tensor", work["axpy_flops"]),
-            "ns_axpy_update": ("tensor", work["axpy_flops"]),
+            "ns_gram": ("tensor", work["gram_flops_executed"]),
+            "ns_poly": ("tensor", work["poly_flops_executed"]),
+            "ns_axpy": ("tensor", work["axpy_flops_executed"]),
+            "ns_axpy_update": ("tensor", work["axpy_flops_executed"]),
             "momentum_norm": ("hbm", work["momentum_bytes"]),
             "momentum_rowq": ("hbm", work["momentum_bytes"]),
             "update": ("hbm", work["update_bytes"]),
@@ -460,11 +469,18 @@ def run_gpu(args):
             "adamw": ("hbm", work["adamw_bytes"]),
         }
         # per-step algorithmic work of each kernel kind: GEMM kinds run once per
-        # NS iteration (the last B.X is the fused-update kind), elementwise once
-        per_step_work = {
+        # NS iteration (the last B.X is the fused-update kind), elementwise
+        # once.  GEMMs count executed FLOPs (the roofline must not credit the
+        # symmetric products with tiles they skip); nominal FLOPs are kept
+        # per kernel beside them.
+        n_axpy = K - 1 if "ns_axpy_update" in kinds else K
+        nominal_step_work = {
             "ns_gram": work["gram_flops"] * K, "ns_poly": work["poly_flops"] * K,
-            "ns_axpy": work["axpy_flops"] * (K - 1 if "ns_axpy_update" in kinds else K),
-            "ns_axpy_update": work["axpy_flops"],
+            "ns_axpy": work["axpy_flops"] * n_axpy, "ns_axpy_update": work["axpy_flops"]}
+        per_step_work = {
+            "ns_gram": work["gram_flops_executed"] * K, "ns_poly": work["poly_flops_executed"] * K,
+            "ns_axpy": work["axpy_flops_executed"] * n_axpy,
+            "ns_axpy_update": work["axpy_flops_executed"],
             "momentum_norm": work["momentum_bytes"], "momentum_rowq": work["momentum_bytes"],
             "update": work["update_bytes"],
             "normuon_update": work["update_bytes"],
@@ -483,7 +499,7 @@ def run_gpu(args):
                         "unit": "TFLOP/s", "frac": round(ach / peak, 4),
                         "traffic": captured_traffic(dom, wl.name), "traffic_unit": "bytes per launch",
                         "peak_source": f"{peak_src} (sustained bf16 cuBLAS)",
-                        "work_per_launch": per_launch, "work_unit": "nominal FLOP"}
+                        "work_per_launch": per_launch, "work_unit": "executed FLOP"}
             else:
                 ach = per_launch / avg_s / 1e9
                 peak = peaks["hbm_gbs"]
@@ -496,10 +512,13 @@ def run_gpu(args):
         for k in ("momentum_norm", "momentum_rowq", "update", "normuon_update", "adamw"):
             if k in kinds:
                 ew[k] = round(per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e9, 1)
+        sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         for k in ("ns_gram", "ns_poly", "ns_axpy", "ns_axpy_update"):
             if k in kinds:
-                per_kernel[k]["nominal_tflops"] = round(
-                    per_step_work[k] / (kinds[k][0] / args.steps / 1e3) / 1e12, 1)
+                sec = kinds[k][0] / args.steps / 1e3
+                per_kernel[k]["executed_tflops"] = round(per_step_work[k] / sec / 1e12, 1)
+                per_kernel[k]["executed_frac_of_sustained"] = round(per_step_work[k] / sec / 1e12 / sustained, 4)
+                per_kernel[k]["nominal_tflops"] = round(nominal_step_work[k] / sec / 1e12, 1)
         res = {
             "metric": METRIC,
             "value": round(ms_step, 3),
@@ -522,10 +541,14 @@ def run_gpu(args):
                        "CTA pairs: 256x256" if args.narrow_tiles else
                        "CTA pairs: 256x512 (Gram, B'X), 256x256 (A*A, fused update)",
                        "normuon": bool(args.normuon), "row_equilibrate": bool(args.row_equilibrate)},
-            "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
+            "ns_frac_of_peak_executed": round(ns_exe / (ns_ms / 1e3) / 1e12 / sustained, 4) if ns_ms else None,
             "ns_ms_per_step": round(ns_ms, 3),
-            "ns_frac_of_peak_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4) if ns_ms else None,
+            # nominal FLOPs (4 m^2 n + 2 m^3 per iteration) credit the symmetric
+            # products with the tiles they skip, so this can exceed 1
+            "ns_tflops_nominal": round(ns_nom / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
+            "ns_frac_of_peak_nominal_counting_skipped_tiles":
+                round(ns_nom / (ns_ms / 1e3) / 1e12 / sustained, 4) if ns_ms else None,
             "elementwise_gbs": ew,
             "roofline": roof,
             "per_kernel": per_kernel,
@@ -534,9 +557,97 @@ def run_gpu(args):
             "e2e": e2e,
         }
         if not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(wl, reps=1)
+            res["cpu_baseline"] = cpu_baseline(wl, samples=3, with_full_reference_step=True)
         print(json.dumps(res), flush=True)
     R.close()
+
+
+def run_distributed(args):
+    """One data-parallel optimizer step of the workload shared by all ranks."""
+    import torch
+    from muon_polar_orthogonalized_b200 import workloads as W
+    from muon_polar_orthogonalized_b200.build import build
+    from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
+
+    R = RankContext("nccl")
+    world, rank, local = R.world, R.rank, R.local
+    if rank == 0:
+        build()
+    R.barrier()
+    if rank != 0:
+        build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = W.get(args.workload)
+    if any(s.grad_dtype != "bf16" for s in wl.muon) or any(t.grad_dtype != "bf16" for t in wl.adamw):
+        raise SystemExit("--distributed takes a workload with bf16 gradients")
+    # placeholders of the right shapes (no storage): the optimizer moves every
+    # parameter into its flat buffers, which are then filled with the draws
+    zero = torch.zeros((), device=dev)
+    mats = [zero.expand(s.rows, s.cols) for s in wl.muon for _ in range(s.count)]
+    adam = [zero.expand(*t.shape) for t in wl.adamw for _ in range(t.count)]
+    groups = [dict(params=adam[i:i + 1], lr=W.ADAMW_LR, betas=W.ADAMW_BETAS, eps=W.ADAMW_EPS,
+                   weight_decay=0.0) for i in range(len(adam))]
+    opt = DistributedMuonAdamW(mats, groups, process_group=None, grad_dtype=torch.bfloat16,
+                               adamw_grad_dtype=torch.bfloat16, lr=W.MUON_LR, momentum=W.MUON_BETA,
+                               weight_decay=W.MUON_WD, ns_steps=wl.ns_steps)
+    gen = W.device_generator(dev, wl.name, "W", "flat")
+    opt.buf["muon_params"].normal_(0.0, 0.02, generator=gen)
+    opt.buf["adamw_params"].normal_(0.0, 0.02, generator=gen)
+    k = 0
+    for gi, s in enumerate(wl.muon):
+        for j in range(s.count):
+            opt.muon_grads[k].copy_(W.device_grad(wl, s.rows, s.cols, torch.bfloat16, dev, gi, j))
+            k += 1
+    for gl in opt.adamw_grads:
+        for g in gl:
+            g.copy_(torch.randn(g.shape, generator=gen, device=dev).mul_(wl.grad_std))
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        R.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        opt.step()
+    barrier()
+    ws = opt._local.workspace
+    if opt.owned and api_status(ws) != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        opt.step()
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = R.max(e0.elapsed_time(e1), device=dev) / args.steps
+    if rank == 0:
+        ns_exe = wl.ns_flops_executed()
+        res = {"metric": METRIC, "value": round(ms, 3), "unit": "ms", "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+               "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+               "data": "synthetic",
+               "config": {"workload": wl.name, "muon_params": wl.muon_params(),
+                          "adamw_params": wl.adamw_params(), "ns_steps": wl.ns_steps, "grads": "bf16",
+                          "params_state": "fp32", "l2": "inputs larger than L2 (no flush)",
+                          "parallelism": f"dp{world}: owner-sharded Muon, ZeRO-1 AdamW; one reduce_scatter "
+                                         "and one all_gather per flat buffer (NCCL)",
+                          "matrices_per_rank": [opt.owners.count(r) for r in range(world)]},
+               "ns_tflops_executed_per_gpu": round(ns_exe / world / (ms / 1e3) / 1e12, 1),
+               "clocks": clk, "e2e": None,
+               "e2e_note": "the distributed mode times the device step only"}
+        print(json.dumps(res), flush=True)
+    R.close()
+
+
+def api_status(ws) -> int:
+    from muon_polar_orthogonalized_b200 import api
+    return api.muon_query_status(ws)
 
 
 # --------------------------------------------------------- CPU (oracle)
@@ -551,49 +662,107 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(wl, reps: int = 1):
-    """The oracle, as it stands, on a bounded sample of the workload, scaled to
-    ms per full step: one Muon matrix of the cheapest shape group (timed
-    muon_step in fp64), extrapolated to every matrix by nominal NS FLOPs, plus
-    AdamW on a 4M-element slice extrapolated by element count."""
+def oracle_cores() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_muon_shape_seconds(rows: int, cols: int, ns_steps: int, grad_std: float, seed: int = 0) -> float:
+    """Wall seconds of the fp64 oracle's muon_step on one rows x cols matrix."""
     import numpy as np
 
     import oracle
     from muon_polar_orthogonalized_b200 import workloads as W
-    try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        cores = max([i.get("num_threads", 1) for i in info] or [1])
-    except Exception:
-        cores = os.cpu_count()
-    s = min(wl.muon, key=lambda s: min(s.rows, s.cols) ** 2 * max(s.rows, s.cols))
-    rng = np.random.default_rng(0)
-    Wm = rng.standard_normal((s.rows, s.cols)) * 0.02
-    G = rng.standard_normal((s.rows, s.cols)) * wl.grad_std
+    rng = np.random.default_rng(seed)
+    Wm = rng.standard_normal((rows, cols)) * 0.02
+    G = rng.standard_normal((rows, cols)) * grad_std
     M = np.zeros_like(G)
     t0 = time.perf_counter()
-    for _ in range(reps):
-        oracle.muon_step(Wm, G, M, W.MUON_LR, W.MUON_BETA, W.MUON_WD, wl.ns_steps, W.NS_COEFFS_FIXED)
-    t_mat = (time.perf_counter() - t0) / reps
-    m, n = min(s.rows, s.cols), max(s.rows, s.cols)
-    f_mat = 4.0 * m * m * n + 2.0 * m ** 3
-    muon_ms = t_mat * (wl.ns_flops_nominal() / wl.ns_steps / f_mat) * 1e3
-    adam_ms = 0.0
+    oracle.muon_step(Wm, G, M, W.MUON_LR, W.MUON_BETA, W.MUON_WD, ns_steps, W.NS_COEFFS_FIXED)
+    return time.perf_counter() - t0
+
+
+def oracle_adamw_seconds(numel: int, grad_std: float, seed: int = 0) -> float:
+    import numpy as np
+
+    import oracle
+    from muon_polar_orthogonalized_b200 import workloads as W
+    rng = np.random.default_rng(seed)
+    p = rng.standard_normal(numel) * 0.02
+    g = rng.standard_normal(numel) * grad_std
+    z = np.zeros(numel)
+    t0 = time.perf_counter()
+    oracle.adamw_step(p, g, z, z.copy(), 1, W.ADAMW_LR, 0.9, 0.95, 1e-8, 0.0)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_ms(wl) -> float:
+    """One bounded sample of the oracle on the workload, scaled to ms per full
+    step: one matrix of every oriented shape (m x n, m <= n: a tall group runs
+    as its transpose, at the same cost) timed once, times the number of
+    matrices of that shape; plus AdamW on up to 4M elements scaled by element
+    count."""
+    by_shape = {}
+    for s in wl.muon:
+        key = (min(s.rows, s.cols), max(s.rows, s.cols))
+        by_shape[key] = by_shape.get(key, 0) + s.count
+    muon_s = sum(n * oracle_muon_shape_seconds(m, nn, wl.ns_steps, wl.grad_std)
+                 for (m, nn), n in by_shape.items())
+    adam_s = 0.0
     n_adam = wl.adamw_params()
     if n_adam:
         k = min(n_adam, 1 << 22)
-        p = rng.standard_normal(k) * 0.02
-        g = rng.standard_normal(k) * wl.grad_std
-        z = np.zeros(k)
-        t0 = time.perf_counter()
-        oracle.adamw_step(p, g, z, z, 1, W.ADAMW_LR, 0.9, 0.95, 1e-8, 0.0)
-        adam_ms = (time.perf_counter() - t0) * (n_adam / k) * 1e3
-    return {"value": round(muon_ms + adam_ms, 1), "unit": "ms", "cores": cores, "kind": "oracle",
-            "cpu_model": cpu_model(),
-            "sample": f"fp64 NumPy muon_step on one {s.rows}x{s.cols} matrix ({t_mat:.2f} s) scaled by "
-                      f"nominal NS FLOPs to all {sum(x.count for x in wl.muon)} matrices, plus AdamW on "
-                      f"{min(n_adam, 1 << 22)} elements scaled to {n_adam}",
-            "extrapolated": True}
+        adam_s = oracle_adamw_seconds(k, wl.grad_std) * (n_adam / k)
+    return (muon_s + adam_s) * 1e3
+
+
+def oracle_sample_description(wl) -> str:
+    shapes = sorted({(min(s.rows, s.cols), max(s.rows, s.cols)) for s in wl.muon})
+    n_adam = wl.adamw_params()
+    return (f"fp64 NumPy muon_step timed on one matrix of each oriented shape "
+            f"({', '.join(f'{m}x{n}' for m, n in shapes)}), scaled by the count of each to all "
+            f"{sum(x.count for x in wl.muon)} matrices, plus AdamW on {min(n_adam, 1 << 22)} "
+            f"elements scaled to {n_adam}")
+
+
+def oracle_full_step_ms(wl) -> float:
+    """The oracle's whole step on the workload, every matrix and every AdamW
+    tensor, unextrapolated (inputs drawn per matrix, not kept)."""
+    muon_s = 0.0
+    for s in wl.muon:
+        for j in range(s.count):
+            muon_s += oracle_muon_shape_seconds(s.rows, s.cols, wl.ns_steps, wl.grad_std, seed=j)
+    adam_s = sum(oracle_adamw_seconds(math.prod(t.shape), wl.grad_std, seed=j)
+                 for t in wl.adamw for j in range(t.count))
+    return (muon_s + adam_s) * 1e3
+
+
+def cpu_baseline(wl, samples: int = 3, with_full_reference_step: bool = False):
+    """The oracle, as it stands, on the host cores: the median of `samples`
+    bounded samples (oracle_sample_ms) with their spread; a sample is
+    extrapolated to the full step unless it already is the full step.  With
+    with_full_reference_step, the d=768 transformer set's whole step is also
+    timed unextrapolated beside it."""
+    from muon_polar_orthogonalized_b200 import workloads as W
+    vals = [oracle_sample_ms(wl) for _ in range(samples)]
+    extrapolated = any(s.count > 1 for s in wl.muon) or any(t.count > 1 for t in wl.adamw) or \
+        wl.adamw_params() > (1 << 22)
+    out = {"value": round(statistics.median(vals), 1), "unit": "ms", "cores": oracle_cores(),
+           "kind": "oracle", "cpu_model": cpu_model(),
+           "sample": oracle_sample_description(wl) + f"; median of {samples} samples",
+           "samples_ms": [round(v, 1) for v in vals],
+           "spread_ms": [round(min(vals), 1), round(max(vals), 1)],
+           "extrapolated": extrapolated}
+    if with_full_reference_step and wl.name != "gpt_d768_12l":
+        ref = W.get("gpt_d768_12l")
+        out["full_step_unextrapolated"] = {
+            "workload": ref.name, "ms": round(oracle_full_step_ms(ref), 1),
+            "sample_estimate_ms": round(oracle_sample_ms(ref), 1)}
+    return out
 
 
 def run_reference(args):
@@ -602,11 +771,13 @@ def run_reference(args):
     from muon_polar_orthogonalized_b200 import workloads as W
     wl = W.get(args.workload)
     for _ in range(args.warmup):
-        cpu_baseline(wl)
-    vals = [cpu_baseline(wl)["value"] for _ in range(args.steps)]
-    cb = cpu_baseline(wl)
-    v = statistics.median(vals)
-    cb["value"] = v
+        oracle_sample_ms(wl)
+    vals = [oracle_sample_ms(wl) for _ in range(args.steps)]
+    v = round(statistics.median(vals), 1)
+    cb = {"value": v, "unit": "ms", "cores": oracle_cores(), "kind": "oracle", "cpu_model": cpu_model(),
+          "sample": oracle_sample_description(wl) + f"; one sample per step, median of {args.steps}",
+          "samples_ms": [round(x, 1) for x in vals], "spread_ms": [round(min(vals), 1), round(max(vals), 1)],
+          "extrapolated": True}
     res = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms", "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -633,11 +804,15 @@ def main():
                     help="Gram and B'X on 256x256 CTA-pair tiles instead of 256x512")
     ap.add_argument("--single-cta", action="store_true",
                     help="Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of CTA pairs")
+    ap.add_argument("--distributed", action="store_true",
+                    help="time the data-parallel optimizer (owner-sharded Muon, ZeRO-1 AdamW) over the ranks")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.distributed:
+        run_distributed(args)
     else:
         run_gpu(args)
 

@@ -8,6 +8,7 @@
   * the source fingerprint that guards the captured DRAM traffic ignores
     comments and changes with code.
 """
+import argparse
 import os
 import shutil
 
@@ -58,12 +59,13 @@ def test_source_fingerprint_ignores_comments_only(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     files = bench.TRAFFIC_CAPTURES["ns_axpy"]["sources"]
     base = bench.source_fingerprint(files)
-    assert base == bench.TRAFFIC_CAPTURES["ns_axpy"]["sha"]
-    assert bench.captured_traffic("ns_axpy", "llama_8b_32l") is not None
+    current = base == bench.TRAFFIC_CAPTURES["ns_axpy"]["sha"]
+    assert (bench.captured_traffic("ns_axpy", "llama_8b_32l") is not None) == current
     f = dst / files[0]
     text = f.read_text()
     f.write_text("// a comment line\n/* and a\n   block comment */\n" + text)
     assert bench.source_fingerprint(files) == base
+    assert (bench.captured_traffic("ns_axpy", "llama_8b_32l") is not None) == current
     f.write_text(text.replace("namespace muon {", "namespace muon {\nconstexpr int kProbe = 1;", 1))
     assert bench.source_fingerprint(files) != base
     assert bench.captured_traffic("ns_axpy", "llama_8b_32l") is None
@@ -110,3 +112,27 @@ def test_clock_sampler_without_nvidia_smi(monkeypatch):
     sampler.start()
     got = sampler.stop()
     assert got["sm_mhz"] is None and got["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_reference_arm_line_on_small_workload(capsys, monkeypatch):
+    """The oracle arm prints one JSON line whose value is the median of its
+    per-step samples, with their spread, on the arm's own workload."""
+    import json
+    import statistics
+    monkeypatch.delenv("RANK", raising=False)
+    args = argparse.Namespace(workload="single_256x1024", steps=3, warmup=1)
+    bench.run_reference(args)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["workload"] == "single_256x1024"
+    cb = line["cpu_baseline"]
+    assert len(cb["samples_ms"]) == 3
+    assert line["value"] == cb["value"] == round(statistics.median(cb["samples_ms"]), 1)
+    assert cb["spread_ms"][0] <= line["value"] <= cb["spread_ms"][1]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["higher_is_better"] is False
+
+
+def test_cpu_baseline_median_and_spread():
+    cb = bench.cpu_baseline(wl.get("single_256x1024"), samples=3)
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1
+    assert cb["spread_ms"][0] <= cb["value"] <= cb["spread_ms"][1]
+    assert cb["extrapolated"] is False   # one matrix and one AdamW tensor: the sample is the step
