@@ -86,14 +86,24 @@ class MuonAdamW:
         return out
 
     @torch.no_grad()
-    def step(self, stream=None, replicas: Optional[Sequence[Sequence[torch.Tensor]]] = None) -> None:
+    def step(self, stream=None, replicas: Optional[Sequence[Sequence[torch.Tensor]]] = None,
+             muon_grads: Optional[Sequence[torch.Tensor]] = None,
+             adamw_grads: Optional[Sequence[Sequence[torch.Tensor]]] = None) -> None:
         """One MuonAdamW step.  replicas: optional copies of the Muon
         parameters (replicas[r][k] is copy r of the k-th tensor given at
         construction, e.g. another data-parallel rank's replica in peer
-        memory); each receives the updated values (muon_step_replicated)."""
+        memory); each receives the updated values (muon_step_replicated).
+        muon_grads / adamw_grads: the gradients to use instead of each
+        parameter's .grad (muon_grads[k] for the k-th Muon tensor given at
+        construction, adamw_grads[g][j] for tensor j of AdamW group g)."""
         self.step_count += 1
         if self.muon_params:
-            grads = [p.grad for p in self.muon_params]
+            if muon_grads is not None:
+                if len(muon_grads) != len(self.muon_params):
+                    raise ValueError("muon_grads must hold one gradient per Muon parameter")
+                grads = [muon_grads[k] for k in self._order]
+            else:
+                grads = [p.grad for p in self.muon_params]
             if any(g is None for g in grads):
                 raise ValueError("every Muon parameter needs a .grad")
             gd = self._grad_dtypes(grads)
@@ -107,8 +117,10 @@ class MuonAdamW:
                               self.beta, self.wd, self.ns_steps, self.coeffs, self.flags,
                               self.workspace, stream=stream)
         specs = []
-        for g in self.adamw_groups:
-            grads = [p.grad for p in g["params"]]
+        if adamw_grads is not None and len(adamw_grads) != len(self.adamw_groups):
+            raise ValueError("adamw_grads must hold one list per AdamW group")
+        for gi, g in enumerate(self.adamw_groups):
+            grads = list(adamw_grads[gi]) if adamw_grads is not None else [p.grad for p in g["params"]]
             if any(x is None for x in grads):
                 raise ValueError("every AdamW parameter needs a .grad")
             specs.append(api.AdamWSpec(g["params"], grads, g["exp_avg"], g["exp_avg_sq"], g["lr"],

@@ -1,13 +1,20 @@
-"""Owner-sharded Muon across data-parallel ranks, on CPU with gloo (world 2).
+"""Owner-sharded Muon and ZeRO-1 AdamW across data-parallel ranks, on CPU
+with gloo (world 2).
 
-The protocol of muon_polar_orthogonalized_b200.distributed (reduce each
-matrix's gradient to its owner, owner steps, owner broadcasts) runs on two
-gloo ranks with the per-rank compute taken from the fp64 oracle; the result
-must equal one process stepping every matrix on the data-parallel mean
-gradient.  Also checks the owner assignment and that momentum lives only on
-owners.
+The protocol of muon_polar_orthogonalized_b200.distributed -- one
+reduce_scatter of each flat gradient buffer, every rank steps what it owns
+(its Muon matrices, its slice of the AdamW tensors), one in-place all_gather
+of each flat parameter buffer -- runs on two gloo ranks with the per-rank
+compute taken from the fp64 oracle; the result must equal one process
+stepping every matrix and every AdamW tensor on the data-parallel mean
+gradient.  The peer-buffer variant (every rank's buffers in shared memory
+standing in for peer GPU memory: owners average the gradients from every
+rank themselves and write every rank's copy of what they update) must give
+the same.  Also checks the flat layout, the owner assignment, and that
+momentum and AdamW state live only where owned.
 """
 import json
+import math
 import os
 import socket
 import sys
@@ -19,6 +26,8 @@ import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SHAPES = [(64, 128), (128, 64), (96, 96), (32, 256), (256, 32), (48, 80)]
+ADAM_SHAPES = [(10, 4), (7,)]          # 40 elements straddle the two ranks' slices
+ADAM_LR = [1e-3, 5e-3]
 LR, BETA, WD = 0.02, 0.95, 0.01
 
 
@@ -33,12 +42,54 @@ def _params():
     return [torch.from_numpy(rng.standard_normal(s) * 0.02) for s in SHAPES]
 
 
+def _adam_params():
+    rng = np.random.default_rng(5)
+    return [torch.from_numpy(rng.standard_normal(s) * 0.02) for s in ADAM_SHAPES]
+
+
 def _grads(rank, step):
     rng = np.random.default_rng(1000 + 10 * step + rank)
     return [torch.from_numpy(rng.standard_normal(s)) for s in SHAPES]
 
 
-def _worker(rank, world, port, out_dir):
+def _adam_grads(rank, step):
+    rng = np.random.default_rng(2000 + 10 * step + rank)
+    return [torch.from_numpy(rng.standard_normal(s)) for s in ADAM_SHAPES]
+
+
+def _oracle_fns(oracle, calls):
+    def step_fn(ps, gs, ms, replicas=None):
+        calls["muon"] += 1
+        for k, (p, g, m) in enumerate(zip(ps, gs, ms)):
+            w_new, m_new, _ = oracle.muon_step(p.numpy(), g.numpy(), m.numpy(), LR, BETA, WD)
+            p.copy_(torch.from_numpy(w_new))
+            m.copy_(torch.from_numpy(m_new))
+            for rep in replicas or []:
+                rep[k].copy_(torch.from_numpy(w_new))
+
+    def adamw_fn(pieces, step):
+        calls["adamw"] += 1
+        for pc in pieces:
+            b1, b2 = pc["betas"]
+            for p, g, m, v in zip(pc["params"], pc["grads"], pc["exp_avg"], pc["exp_avg_sq"]):
+                pn, mn, vn = oracle.adamw_step(p.numpy(), g.numpy(), m.numpy(), v.numpy(), step, pc["lr"],
+                                               b1, b2, pc["eps"], pc["weight_decay"])
+                p.copy_(torch.from_numpy(pn))
+                m.copy_(torch.from_numpy(mn))
+                v.copy_(torch.from_numpy(vn))
+    return step_fn, adamw_fn
+
+
+def _run_steps(opt, rank):
+    for step in range(2):
+        for k, g in enumerate(_grads(rank, step)):
+            opt.muon_grads[k].copy_(g)
+        for gi, g in enumerate(_adam_grads(rank, step)):
+            opt.adamw_grads[gi][0].copy_(g)
+        opt.step()
+
+
+def _worker(rank, world, port, out_dir, shared):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -46,31 +97,37 @@ def _worker(rank, world, port, out_dir):
     import oracle
     from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
     dist.init_process_group("gloo", rank=rank, world_size=world)
-    params = _params()
-    emb = torch.from_numpy(np.random.default_rng(5).standard_normal((10, 4)) * 0.02)
-    state = {"m": torch.zeros_like(emb), "v": torch.zeros_like(emb), "t": 0}
+    params, adam = _params(), _adam_params()
+    groups = [dict(params=[a], lr=lr) for a, lr in zip(adam, ADAM_LR)]
+    calls = {"muon": 0, "adamw": 0, "mean": 0}
+    step_fn, adamw_fn = _oracle_fns(oracle, calls)
+    kw = {}
+    if shared is not None:
+        peer_grads = shared.get("peer_grads")
 
-    def step_fn(ps, gs, ms):
-        for p, g, m in zip(ps, gs, ms):
-            w_new, m_new, _ = oracle.muon_step(p.numpy(), g.numpy(), m.numpy(), LR, BETA, WD)
-            p.copy_(torch.from_numpy(w_new))
-            m.copy_(torch.from_numpy(m_new))
-
-    def adamw_fn(groups):
-        state["t"] += 1
-        p = groups[0]["params"][0]
-        pn, mn, vn = oracle.adamw_step(p.numpy(), p.grad.numpy(), state["m"].numpy(), state["v"].numpy(),
-                                       state["t"], 1e-3, 0.9, 0.95, 1e-8, 0.0)
-        p.copy_(torch.from_numpy(pn)); state["m"].copy_(torch.from_numpy(mn)); state["v"].copy_(torch.from_numpy(vn))
-
-    opt = DistributedMuonAdamW(params, [dict(params=[emb])], step_fn=step_fn, adamw_fn=adamw_fn)
-    for step in range(2):
-        for p, g in zip(params, _grads(rank, step)):
-            p.grad = g
-        emb.grad = torch.from_numpy(np.random.default_rng(2000 + 10 * step + rank).standard_normal((10, 4)))
-        opt.step()
-    out = {"params": [p.numpy().tolist() for p in params], "emb": emb.numpy().tolist(),
-           "owners": opt.owners, "owned": opt.owned, "momentum_keys": sorted(opt.momentum)}
+        def reduce_fn(dst, sources):
+            calls["mean"] += 1
+            for i, d in enumerate(dst):
+                acc = sources[0][i].clone()
+                for src in sources[1:]:
+                    acc += src[i]
+                d.copy_(acc / len(sources))
+        bufs = shared["bufs"]
+        kw = dict(buffers=bufs[rank],
+                  peer_params={q: (bufs[q]["muon_params"], bufs[q]["adamw_params"])
+                               for q in range(world) if q != rank},
+                  reduce_fn=reduce_fn)
+        if peer_grads:
+            kw["peer_grads"] = {q: (bufs[q]["muon_grads"], bufs[q]["adamw_grads"])
+                                for q in range(world) if q != rank}
+    opt = DistributedMuonAdamW(params, groups, step_fn=step_fn, adamw_fn=adamw_fn, **kw)
+    # parameters now live in the flat buffers; gradients are written into them
+    assert all(p.grad is g for p, g in zip(params, opt.muon_grads))
+    _run_steps(opt, rank)
+    state_numel = sum(t.numel() for pc in opt._pieces for t in pc["exp_avg"])
+    out = {"params": [p.numpy().tolist() for p in params], "adam": [a.numpy().tolist() for a in adam],
+           "owners": opt.owners, "owned": opt.owned, "momentum_keys": sorted(opt.momentum),
+           "adam_state_numel": state_numel, "calls": calls}
     with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
         json.dump(out, f)
     dist.barrier()
@@ -82,124 +139,103 @@ def _reference():
     import oracle
     params = [p.numpy() for p in _params()]
     moms = [np.zeros_like(p) for p in params]
-    emb = np.random.default_rng(5).standard_normal((10, 4)) * 0.02
-    m = v = np.zeros_like(emb)
+    adam = [a.numpy() for a in _adam_params()]
+    ms = [np.zeros_like(a) for a in adam]
+    vs = [np.zeros_like(a) for a in adam]
     for step in range(2):
         g_mean = [(a.numpy() + b.numpy()) / 2 for a, b in zip(_grads(0, step), _grads(1, step))]
         for i in range(len(params)):
             params[i], moms[i], _ = oracle.muon_step(params[i], g_mean[i], moms[i], LR, BETA, WD)
-        ge = (np.random.default_rng(2000 + 10 * step).standard_normal((10, 4)) +
-              np.random.default_rng(2000 + 10 * step + 1).standard_normal((10, 4))) / 2
-        emb, m, v = oracle.adamw_step(emb, ge, m, v, step + 1, 1e-3, 0.9, 0.95, 1e-8, 0.0)
-    return params, emb
+        ga = [(a.numpy() + b.numpy()) / 2 for a, b in zip(_adam_grads(0, step), _adam_grads(1, step))]
+        for t in range(len(adam)):
+            adam[t], ms[t], vs[t] = oracle.adamw_step(adam[t], ga[t], ms[t], vs[t], step + 1, ADAM_LR[t],
+                                                      0.9, 0.95, 1e-8, 0.0)
+    return params, adam
 
 
-def test_owner_sharded_step_equals_single_process(tmp_path):
-    world, port = 2, _free_port()
-    mp.start_processes(_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True,
-                       start_method="spawn")
-    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
-    ref_params, ref_emb = _reference()
+def _check(res, world):
+    ref_params, ref_adam = _reference()
     for r in range(world):
         for got, want in zip(res[r]["params"], ref_params):
             np.testing.assert_allclose(np.array(got), want, rtol=0, atol=1e-15)
-        np.testing.assert_allclose(np.array(res[r]["emb"]), ref_emb, rtol=0, atol=1e-15)
+        for got, want in zip(res[r]["adam"], ref_adam):
+            np.testing.assert_allclose(np.array(got), want, rtol=0, atol=1e-15)
+
+
+def test_sharded_step_equals_single_process(tmp_path):
+    world, port = 2, _free_port()
+    mp.start_processes(_worker, args=(world, port, str(tmp_path), None), nprocs=world, join=True,
+                       start_method="spawn")
+    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
+    _check(res, world)
     # every matrix owned by exactly one rank; momentum only where owned
     assert res[0]["owners"] == res[1]["owners"]
-    owned = sorted(res[0]["owned"] + res[1]["owned"])
-    assert owned == list(range(len(SHAPES)))
+    assert sorted(res[0]["owned"] + res[1]["owned"]) == list(range(len(SHAPES)))
     for r in range(world):
         assert res[r]["momentum_keys"] == res[r]["owned"]
-
-
-def _worker_peer(rank, world, port, out_dir, all_params, all_grads):
-    """As _worker, with every rank's Muon parameters (and, if given, gradients)
-    in shared memory standing in for peer GPU memory: owners write the other
-    rank's copies in their step (peer_params) instead of broadcasting, and
-    average the gradients from every rank themselves (peer_grads) instead of
-    the reduces."""
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
-                      WORLD_SIZE=str(world))
-    sys.path.insert(0, ROOT)
-    import torch.distributed as dist
-    import oracle
-    from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
-    dist.init_process_group("gloo", rank=rank, world_size=world)
-    params = all_params[rank]
-    peers = {r: all_params[r] for r in range(world) if r != rank}
-    peer_grads = {r: all_grads[r] for r in range(world) if r != rank} if all_grads else None
-    calls = {"replicated": 0, "mean": 0}
-
-    def reduce_fn(dst, sources):
-        calls["mean"] += 1
-        for i, d in enumerate(dst):
-            acc = sources[0][i].clone()
-            for src in sources[1:]:
-                acc += src[i]
-            d.copy_(acc / len(sources))
-
-    def step_fn(ps, gs, ms, replicas):
-        calls["replicated"] += 1
-        for k, (p, g, m) in enumerate(zip(ps, gs, ms)):
-            w_new, m_new, _ = oracle.muon_step(p.numpy(), g.numpy(), m.numpy(), LR, BETA, WD)
-            p.copy_(torch.from_numpy(w_new))
-            m.copy_(torch.from_numpy(m_new))
-            for rep in replicas:
-                rep[k].copy_(torch.from_numpy(w_new))
-
-    opt = DistributedMuonAdamW(params, [], step_fn=step_fn, peer_params=peers, peer_grads=peer_grads,
-                               reduce_fn=reduce_fn)
-    for step in range(2):
-        for k, (p, g) in enumerate(zip(params, _grads(rank, step))):
-            if all_grads:
-                all_grads[rank][k].copy_(g)      # the rank's gradient buffer, seen by its peers
-                p.grad = all_grads[rank][k]
-            else:
-                p.grad = g
-        opt.step()
-    out = {"params": [p.numpy().tolist() for p in params], "calls": calls["replicated"],
-           "mean_calls": calls["mean"]}
-    with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
-        json.dump(out, f)
-    dist.barrier()
-    dist.destroy_process_group()
+    # ZeRO-1: the AdamW state is split, not replicated
+    total = sum(math.prod(s) for s in ADAM_SHAPES)
+    assert res[0]["adam_state_numel"] + res[1]["adam_state_numel"] == total
+    assert 0 < res[0]["adam_state_numel"] < total
 
 
 @pytest.mark.parametrize("peer_grads", [False, True])
-def test_owner_writes_peer_replicas_equals_single_process(tmp_path, peer_grads):
+def test_peer_buffers_equal_single_process(tmp_path, peer_grads):
+    sys.path.insert(0, ROOT)
+    from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
     world, port = 2, _free_port()
-    all_params, all_grads = [], []
+    sizes = DistributedMuonAdamW.buffer_numels(SHAPES, [math.prod(s) for s in ADAM_SHAPES], world)
+    bufs = []
     for r in range(world):
-        ps = [p.clone() for p in _params()]
-        gs = [torch.zeros_like(p) for p in ps]
-        for t in ps + gs:
+        b = {k: torch.zeros(n, dtype=torch.float64) for k, n in sizes.items()}
+        for t in b.values():
             t.share_memory_()
-        all_params.append(ps)
-        all_grads.append(gs)
-    mp.start_processes(_worker_peer, args=(world, port, str(tmp_path), all_params,
-                                           all_grads if peer_grads else None),
-                       nprocs=world, join=True, start_method="spawn")
+        bufs.append(b)
+    shared = {"bufs": bufs, "peer_grads": peer_grads}
+    mp.start_processes(_worker, args=(world, port, str(tmp_path), shared), nprocs=world, join=True,
+                       start_method="spawn")
     res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
-    ref_params, _ = _reference()
+    _check(res, world)
     for r in range(world):
-        assert res[r]["calls"] == 2
-        assert res[r]["mean_calls"] == (2 if peer_grads else 0)
-        for got, want in zip(res[r]["params"], ref_params):
-            np.testing.assert_allclose(np.array(got), want, rtol=0, atol=1e-15)
+        assert res[r]["calls"]["mean"] == (2 * 2 if peer_grads else 0)   # Muon region + AdamW slice
 
 
-def test_peer_params_must_cover_other_ranks():
+def test_flat_layout():
+    sys.path.insert(0, ROOT)
+    from muon_polar_orthogonalized_b200.distributed import ALIGN, FlatLayout
+    shapes = [(4096, 4096)] * 4 + [(1024, 4096)] * 4 + [(100, 37)] * 3
+    numels = [1000003, 17, 64, 5]
+    for world in (1, 2, 3, 8):
+        L = FlatLayout(shapes, numels, world)
+        assert L.muon_region % ALIGN == 0 and L.adamw_slice % ALIGN == 0
+        spans = sorted((o, o + math.prod(s)) for o, s in zip(L.muon_offset, shapes))
+        for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+            assert a1 <= b0                                   # disjoint
+        for i, (o, s) in enumerate(zip(L.muon_offset, shapes)):
+            assert o % ALIGN == 0
+            r = L.owners[i]
+            assert r * L.muon_region <= o and o + math.prod(s) <= (r + 1) * L.muon_region
+        covered = [0] * len(numels)
+        for r in range(world):
+            for t, start, n in L.owned_pieces(r):
+                assert (L.adamw_offset[t] + start) % ALIGN == 0
+                assert r * L.adamw_slice <= L.adamw_offset[t] + start
+                assert L.adamw_offset[t] + start + n <= (r + 1) * L.adamw_slice
+                covered[t] += n
+        assert covered == numels                              # every element owned once
+        assert L.adamw_offset[-1] + numels[-1] <= L.adamw_total
+
+
+def test_peers_must_cover_other_ranks():
     sys.path.insert(0, ROOT)
     from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
     ps = _params()
-    import pytest
     with pytest.raises(ValueError):
-        DistributedMuonAdamW(ps, [], step_fn=lambda *a: None, peer_params={1: ps})   # world 1: no peers
+        DistributedMuonAdamW(ps, [], step_fn=lambda *a: None,
+                             peer_params={1: (torch.zeros(1), torch.zeros(1))})   # world 1: no peers
     seen = []
-    opt = DistributedMuonAdamW(ps, [], step_fn=lambda p, g, m, reps: seen.append(len(reps)),
+    opt = DistributedMuonAdamW(_params(), [], step_fn=lambda p, g, m, reps: seen.append(len(reps)),
                                peer_params={})                                    # world 1: none needed
-    for p in ps:
-        p.grad = torch.zeros_like(p)
     opt.step()
     assert seen == [0]
 
