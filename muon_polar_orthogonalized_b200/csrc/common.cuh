@@ -50,12 +50,18 @@ struct GemmProblem {
   int sym;                  // output symmetric: upper tiles computed, upper form stored
   int a_sym, b_sym;         // operand stored in upper form (tensor-core path)
   int tiles_m, tiles_n, tiles_per_mat, tile_begin;
+  int col_major;            // tile order of a non-symmetric output: tile rows fastest
+                            // (else bands of tile columns, tile columns fastest)
   // operands (SIMT path reads these directly; the tensor-core path uses tensor maps)
   const void* a; long long a_bs; int a_ld;
   const void* b; long long b_bs; int b_ld;
   // epilogue
   void* out; long long out_bs; int out_ld;
   const void* ein; long long ein_bs; int ein_ld;   // A (poly) or X (axpy)
+  // exact diagonal of B' (tensor-core path): the A*A epilogue writes
+  // lo_i = B'_ii - bf16(B'_ii) for every row; the B'X epilogue adds lo * X,
+  // lo indexed by the output row (wide) or column (tall, dlo_col = 1)
+  float* dlo; long long dlo_bs; int dlo_col;
   int scale_mode;           // 0 none, 1: s^2 (first Gram), 2: s (first X update)
   int scale_base;           // index of matrix 0 of this problem in the scale array
   float ca, cb, cc;         // a_k, b_k, c_k

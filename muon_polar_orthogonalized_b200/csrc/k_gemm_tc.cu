@@ -10,13 +10,16 @@
 //                                symmetric, so both operands are rows of A;
 //                                K blocks left of a row block's diagonal are
 //                                read transposed from the stored upper form;
-//                                the epilogue reads the A tile for b*A and
-//                                adds a on the diagonal
-//   axpy  X' = s B' X            = s (a X + B X); wide matrices; tall ones
-//                                (iterated as X^T) compute X' = s X B' in
-//                                parameter layout; B' is read like A above.
-//                                The epilogue only scales and converts: a X
-//                                rides in the product
+//                                the epilogue reads the A tile for b*A, adds
+//                                a on the diagonal and keeps, per row, the
+//                                part of the diagonal that bf16 drops:
+//                                lo_i = B'_ii - bf16(B'_ii), in fp32
+//   axpy  X' = s (B' X + lo X)   = s (a X + B X) with B''s diagonal exact;
+//                                wide matrices; tall ones (iterated as X^T)
+//                                compute X' = s (X B' + X lo) in parameter
+//                                layout; B' is read like A above.  a X rides
+//                                in the product; the epilogue adds lo_i X_ij
+//                                (X read at the output's position) and scales
 //   axpy_update                  last iteration: U = bf16(X') feeds the
 //                                cautious-decay update of W directly
 // s is the Frobenius scale 1/(||m~||+1e-7), applied on the first iteration
@@ -34,7 +37,8 @@
 //   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
 //   warps 2-9: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31; two warps
 //              per lane quadrant split the tile's columns)
-// No multicast is used anywhere.
+// No TMA or bulk load uses multicast; the only multicast is the
+// tcgen05.commit that signals an mbarrier in both CTAs of a pair.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -104,7 +108,11 @@ struct TileCoord {
 
 // Linear tile index -> (problem, matrix, tile row, tile column).  Symmetric
 // problems enumerate, per tile row I, only the tile columns that reach the
-// upper triangle: J >= I*BM/BN.
+// upper triangle: J >= I*BM/BN.  A column-major problem walks every tile row
+// of one tile column before the next column (B'X of a wide matrix: the
+// concurrent tiles share few X panels and all of B', which stays in L2, so
+// each operand is read from DRAM about once); the others walk bands of
+// TC_RASTER_GN tile columns row by row.
 template <int BM, int BN>
 __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
   int pi = 0;
@@ -124,6 +132,9 @@ __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
     }
     tm = I;
     tn = (I * BM) / BN + r;
+  } else if (q.col_major) {
+    tn = r / q.tiles_m;
+    tm = r - tn * q.tiles_m;
   } else {
     const int band_tiles = q.tiles_m * TC_RASTER_GN;
     const int band = r / band_tiles;
@@ -156,9 +167,8 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
   }
 }
 
-// The Gram and B'X epilogues instead stage their rows for a TMA store (their
-// epilogues load nothing else, and the staged store measured faster there;
-// for A*A, whose epilogue also reads A, the direct store was faster).
+// The Gram and B'X epilogues instead stage their rows for a TMA store (the
+// staged store measured faster there; for A*A the direct store was faster).
 // One warp's 32 rows x 32 columns of output, lane = row: packed to bf16 into a
 // 2 KB staging buffer in the 64-byte-swizzle layout (16-byte unit u of row r
 // at unit u ^ ((r >> 1) & 3), four shared-memory wavefronts per store), then
@@ -214,9 +224,9 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
 template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const GemmProblem& q,
                                                   int mat, int i, int jt, int width) {
-  if (EPI == EPI_GRAM || EPI == EPI_AXPY || i >= q.M) return;
+  if (EPI == EPI_GRAM || i >= q.M) return;
   const int ncols = min(width, q.N - jt);  // jt < N
-  if (EPI == EPI_POLY) {
+  if (EPI == EPI_POLY || ((EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) && q.dlo)) {
     const char* ein = reinterpret_cast<const char*>(
         static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
     for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
@@ -229,18 +239,19 @@ __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const G
 }
 
 struct EpiIn {
-  uint4 e[4];     // 32 bf16 of the epilogue operand A (A*A products)
+  uint4 e[4];     // 32 bf16 of the epilogue operand: A (A*A) or X (B'X)
 };
 struct EpiW {
   float4 w[8];    // 32 fp32 parameters (fused update)
 };
 
-// The bf16 operand A of one chunk (A*A products only).
+// The bf16 operand of one chunk: A for A*A, X for the exact-diagonal term of
+// B'X (nothing for the Gram).
 template <int EPI>
 __device__ __forceinline__ void epilogue_load(const TcGemmParams& p, const GemmProblem& q, int mat,
                                               int i, int j0, bool full, EpiIn& in) {
   if (i >= q.M) return;
-  if (EPI == EPI_POLY && full) {
+  if ((EPI == EPI_POLY || ((EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) && q.dlo)) && full) {
     const uint4* e4 = reinterpret_cast<const uint4*>(
         static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0);
 #pragma unroll
@@ -296,7 +307,64 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
     }
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]) + ((j0 + c == i) ? q.ca : 0.f);
+    if (q.dlo && i >= j0 && i < j0 + 32) {
+      // this row's diagonal element: keep what its bf16 rounding drops (exact
+      // in fp32, the two values being within a factor of two of each other)
+      float lo = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (j0 + c == i) lo = v[c] - __bfloat162float(__float2bfloat16_rn(v[c]));
+      q.dlo[mat * q.dlo_bs + i] = lo;
+    }
   } else {
+    if constexpr (EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) {
+      if (q.dlo) {
+        // B''s exact diagonal: add lo * X at the output's own position
+        const float* lo = q.dlo + mat * q.dlo_bs;
+        if (!q.dlo_col && full) {
+          const float l = lo[i];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t w[4] = {in.e[u].x, in.e[u].y, in.e[u].z, in.e[u].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
+              v[u * 8 + h * 2] = fmaf(l, f.x, v[u * 8 + h * 2]);
+              v[u * 8 + h * 2 + 1] = fmaf(l, f.y, v[u * 8 + h * 2 + 1]);
+            }
+          }
+        } else {
+        float x[32];
+        if (full) {
+          unpack_bf16x32(in.e, x);
+        } else {
+          const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs +
+                                    static_cast<long long>(i) * q.ein_ld + j0;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = (j0 + c < q.N) ? __bfloat162float(xr[c]) : 0.f;
+        }
+        if (!q.dlo_col) {
+          const float l = lo[i];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] = fmaf(l, x[c], v[c]);
+        } else if (full) {
+          const float4* l4 = reinterpret_cast<const float4*>(lo + j0);   // ldm pitch: 32-byte rows
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 l = l4[c4];
+            v[c4 * 4 + 0] = fmaf(l.x, x[c4 * 4 + 0], v[c4 * 4 + 0]);
+            v[c4 * 4 + 1] = fmaf(l.y, x[c4 * 4 + 1], v[c4 * 4 + 1]);
+            v[c4 * 4 + 2] = fmaf(l.z, x[c4 * 4 + 2], v[c4 * 4 + 2]);
+            v[c4 * 4 + 3] = fmaf(l.w, x[c4 * 4 + 3], v[c4 * 4 + 3]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (j0 + c < q.N) v[c] = fmaf(lo[j0 + c], x[c], v[c]);
+        }
+        }
+      }
+    }
     // Gram: s^2 on the first iteration; axpy: s on the first iteration
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] *= f;
@@ -569,19 +637,15 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         const int wi = q.w_first + tc.mat;
         wvec = ((reinterpret_cast<uintptr_t>(p.wptr[wi]) | (static_cast<uintptr_t>(p.wcols[wi]) << 2)) & 15u) == 0;
       }
-      if (!sm100::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
-        record_timeout(p.status, abort_flag);
-        break;
-      }
-      sm100::tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                             static_cast<uint32_t>(acc * C::BN);
       // Active chunks form one range [c_lo, c_hi): a symmetric tile skips the
       // chunks left of its rows' 256-block (a prefix) and a ragged tile stops
-      // at N.  For A*A the A operand of chunk c+1 is loaded while chunk c is
-      // combined and stored, so one L2 round trip is in flight at all times;
-      // the fused update loads W (prefetched to L2 above) with each chunk; the
-      // Gram and B'X epilogues load nothing.
+      // at N.  B'X keeps kXAhead chunks of X in flight: the first ones are
+      // loaded before the accumulator is ready (the epilogue warps are idle
+      // while the tile's MMAs run), each later one when a buffer frees up.
+      // For A*A the A operand of chunk c+1 is loaded while chunk c is
+      // combined and stored; the fused update loads X and W (both
+      // prefetched to L2 above) with each chunk; the Gram epilogue loads
+      // nothing.
       // symmetric output in upper form: chunks left of the rows' 256-block are not stored
       const int rblk = row0 / kSymBlock;
       int c_hi = 0;
@@ -589,11 +653,32 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       int c_lo = 0;
       if (q.sym) c_lo = max(0, (kSymBlock * rblk - jslice) / 32);
       auto chunk_j0 = [&](int cc) { return jslice + cc * 32; };
-      auto process = [&](int cc, const EpiIn& in) {
+      constexpr int kXAhead = 2;
+      EpiIn xb[kXAhead];
+      if constexpr (EPI == EPI_AXPY) {
+        if (q.dlo) {
+#pragma unroll
+          for (int k = 0; k < kXAhead; ++k)
+            if (k < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(k), chunk_j0(k) + 32 <= q.N, xb[k]);
+        }
+      }
+      if (!sm100::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
+        record_timeout(p.status, abort_flag);
+        break;
+      }
+      sm100::tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(acc * C::BN);
+      auto process = [&](int cc, const EpiIn& in_prev) {
         const int j0 = chunk_j0(cc);
         const bool full = (j0 + 32 <= q.N);
         EpiW win;
         epilogue_load_w<EPI>(p, q, tc.mat, i, j0, full, wvec, win);
+        // the fused update loads its X chunk with W (no register room for a
+        // second chunk in flight); the other epilogues got theirs one chunk ahead
+        EpiIn in_now;
+        if constexpr (EPI == EPI_AXPY_UPDATE) epilogue_load<EPI>(p, q, tc.mat, i, j0, full, in_now);
+        const EpiIn& in = (EPI == EPI_AXPY_UPDATE) ? in_now : in_prev;
         float v[32];
         sm100::tmem_ld32(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), v);
         epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, in, win, v);
@@ -603,11 +688,28 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           ++stage_ctr;
         }
       };
-      if constexpr (EPI != EPI_POLY) {
+      if constexpr (EPI == EPI_GRAM || EPI == EPI_AXPY_UPDATE) {
 #pragma unroll 1
         for (int cc = c_lo; cc < c_hi; ++cc) {
           const EpiIn none{};
           process(cc, none);
+        }
+      } else if constexpr (EPI == EPI_AXPY) {
+        // c_lo = 0 (not symmetric); the inner loop is unrolled so that xb[]
+        // stays in registers
+        static_assert(kChunks % kXAhead == 0, "whole rounds of X buffers");
+#pragma unroll 1
+        for (int c0 = 0; c0 < kChunks; c0 += kXAhead) {
+#pragma unroll
+          for (int k = 0; k < kXAhead; ++k) {
+            const int cc = c0 + k;
+            if (cc < c_hi) {
+              process(cc, xb[k]);
+              if (q.dlo && cc + kXAhead < c_hi)
+                epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc + kXAhead), chunk_j0(cc + kXAhead) + 32 <= q.N,
+                                   xb[k]);
+            }
+          }
         }
       } else {
         EpiIn in0, in1;

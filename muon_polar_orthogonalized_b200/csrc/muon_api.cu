@@ -212,6 +212,7 @@ struct WaveItem {
   size_t x0, x1, b;     // byte offsets in the workspace
   int sbase;            // index of the item's first matrix in the wave's scale array
   long long pbase;      // first partial sum of the item's first matrix (wave-relative)
+  size_t lo = 0;        // byte offset of the item's diagonal residuals (ldm floats per matrix)
 };
 
 struct Wave {
@@ -244,6 +245,8 @@ size_t layout_wave(Wave& w, const std::vector<GroupGeom>& geo) {
     off = align_up(off + q.xstride * it.count, 1024);
     it.b = off;
     off = align_up(off + q.bstride * it.count, 1024);
+    it.lo = off;
+    off = align_up(off + 4ull * q.ldm * it.count, 1024);
   }
   w.total = off;
   return off;
@@ -663,6 +666,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       P.sym = 1;
       P.out = bbuf; P.out_bs = bs_el; P.out_ld = q.ldm;   // B' = a I + b A + c A A
       P.ein = xoth; P.ein_bs = xs_el; P.ein_ld = q.ldm;
+      if (!f32) { P.dlo = reinterpret_cast<float*>(a.ws + it.lo); P.dlo_bs = q.ldm; }
     } else {
       P.M = q.r;
       P.N = q.c;
@@ -677,6 +681,12 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       }
       P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldc;
       P.scale_mode = (k == 0) ? 2 : 0;
+      if (!f32) {
+        // the part of B''s diagonal that bf16 drops comes back as lo * X,
+        // X read at the output's own position
+        P.dlo = reinterpret_cast<float*>(a.ws + it.lo); P.dlo_bs = q.ldm; P.dlo_col = q.tall;
+        P.ein = xcur; P.ein_bs = xs_el; P.ein_ld = q.ldc;
+      }
     }
     // the tensor-core path stores A and B' in upper form and reads them so;
     // the fp32 scaffold computes and reads full matrices
@@ -685,6 +695,9 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       else if (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) (q.tall ? P.b_sym : P.a_sym) = 1;
     }
     if (f32) P.sym = 0;
+    // B'X of a wide matrix: tile rows fastest, so that B' (m x m, indexed by
+    // the tile row) stays in L2 while each X panel streams through once
+    P.col_major = (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) && !q.tall;
     P.tiles_m = (P.M + BM - 1) / BM;
     P.tiles_n = (P.N + BN - 1) / BN;
     if (P.sym) {
@@ -1073,7 +1086,7 @@ static muon_status adamw_impl(const adamw_group* groups, int n_groups, int64_t s
         T.b2 = g.beta2;
         T.omb2 = static_cast<float>(1.0 - b2);
         T.step_size = static_cast<float>(g.lr / bc1);
-        T.sqrt_bc2 = static_cast<float>(std::sqrt(bc2));
+        T.rsqrt_bc2 = static_cast<float>(1.0 / std::sqrt(bc2));
         T.eps = g.eps;
         T.lr = g.lr;
         T.wd = g.wd;

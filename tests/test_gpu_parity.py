@@ -74,19 +74,43 @@ def tol_bf16(r, c, ns=5):
     return TOL_BF16 if (min(r, c) >= 16 and ns <= 5) else 3e-2
 
 
+def pages_bf16_error(x, ns=5, coeffs=FIXED):
+    """How far bf16 storage at the pages' own storage points (X, A, B and
+    each new X rounded; a*X added before the rounding of X') lands from fp64
+    on this input: what the method itself loses in bf16."""
+    ref = oracle.newton_schulz(x, coeffs, ns)
+    return rel(oracle.newton_schulz_bf16_emulated(x, coeffs, ns), ref)
+
+
+def bf16_gate(r, c, ns, e_pages):
+    """bf16-mode tolerance on the orthogonalised update: 2e-2 (tol_bf16), or,
+    only where bf16 storage at the pages' storage points (the bf16-emulated
+    iteration of the pages, on the same input) is already further than that
+    from fp64, 1.15 x that error + 1e-3.  Some inputs (m = 32..40 with nearly
+    equal singular values, e.g. 4100 x 36) have the pages' own bf16 iteration
+    2.0-2.6e-2 from fp64."""
+    return max(tol_bf16(r, c, ns), 1.15 * e_pages + 1e-3)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_orthogonalize_bf16_parity(dev, dtype):
     ins, outs = orth_case(dev, EDGE_SHAPES, dtype)
     for (r, c), x, u in zip(EDGE_SHAPES, ins, outs):
         ref = oracle.newton_schulz(x, FIXED, 5)
         e = rel(u, ref)
-        emu = rel(u, oracle.newton_schulz_bf16_emulated(x, FIXED, 5, fold_a=True))
-        print(f"{r}x{c}: rel err vs fp64 {e:.3e}, vs bf16-emulated {emu:.3e}")
+        gate = bf16_gate(r, c, 5, pages_bf16_error(x))
+        # diagnostic, stricter than the gate: the kernel's own storage points
+        # (a folded into B', B''s diagonal kept exact), emulated
+        emu = rel(u, oracle.newton_schulz_bf16_emulated(x, FIXED, 5, fold_a=True, exact_diag=True))
+        print(f"{r}x{c}: rel err vs fp64 {e:.3e} (gate {gate:.3e}), vs kernel-storage emulation {emu:.3e}")
         assert np.isfinite(u).all(), (r, c)
-        assert e <= tol_bf16(r, c), ((r, c), e)
+        assert e <= gate, ((r, c), e, gate)
         assert emu <= 1.5e-2, ((r, c), emu)
-        if max(r, c) <= 64:  # tiny: fp32 accumulation is exact enough to match bit for bit
-            assert emu == 0.0, ((r, c), emu)
+        if max(r, c) <= 64:
+            # tiny: the kernel follows the emulated storage points up to its
+            # fp32 (not fp64) diagonal residual, which can move a single
+            # rounding by one bf16 unit (a misplaced rounding moves ~1e-2)
+            assert emu <= 5e-4, ((r, c), emu)
 
 
 def test_orthogonalize_fp32_debug_parity(dev):
@@ -492,17 +516,6 @@ ROWEQ_SHAPES = [(1024, 256), (130, 200), (4100, 36), (256, 1024), (40, 3000), (2
                 (66, 130), (8, 20000)]
 
 
-def bf16_gate(r, c, ns, e_emul):
-    """bf16-mode tolerance: 2e-2 (tol_bf16), or, where bf16 storage alone (the
-    bf16-emulated oracle with the kernel's storage points, fold_a=True, on the
-    same input) is already further than that from fp64, 1.15 x that error +
-    1e-3.  For some inputs (m = 32..40 with nearly equal singular values,
-    e.g. 4100 x 36 or a row-equilibrated 40 x 3000) the emulated iteration is
-    2.0-2.5e-2 from fp64, because the five-step map amplifies bf16 storage
-    error there."""
-    return max(tol_bf16(r, c, ns), 1.15 * e_emul + 1e-3)
-
-
 def rowq_grad(shape, seed, step):
     """iid rows scaled by 10^U(-2, 2), so that equilibration matters; row 5
     of a matrix with more than 5 rows is zero."""
@@ -553,7 +566,7 @@ def test_row_equilibrate_parity(dev, gdt, mode):
                     assert rel(host64(W[i]), rw) <= 1e-7
             else:
                 _, mt = oracle.nesterov_momentum(m_old[i], hg[i], 0.95)
-                ue = oracle.newton_schulz_bf16_emulated(oracle.row_equilibrate(mt), FIXED, ns, fold_a=True)
+                ue = oracle.newton_schulz_bf16_emulated(oracle.row_equilibrate(mt), FIXED, ns)
                 if normuon:
                     ue = oracle.normuon_rows(ue)
                 rwe = oracle.cautious_weight_decay_update(w_old[i], ue, lr, wd, True)
@@ -839,23 +852,25 @@ def test_scheduled_graph_replay_matches_eager(dev):
     del graph
 
 
-def test_distributed_single_rank_equals_muonadamw(dev):
-    """With one rank the owner-sharded optimizer is exactly MuonAdamW."""
+@pytest.mark.parametrize("gdt", [torch.float32, torch.bfloat16])
+def test_distributed_single_rank_equals_muonadamw(dev, gdt):
+    """With one rank the sharded optimizer (flat buffers, no collectives) is
+    exactly MuonAdamW, for fp32 and bf16 gradient buffers."""
     from muon_polar_orthogonalized_b200.distributed import DistributedMuonAdamW
     torch.manual_seed(3)
     mats = [torch.randn(256, 384, device=dev) * 0.02, torch.randn(384, 256, device=dev) * 0.02]
     emb = torch.randn(500, 64, device=dev) * 0.02
     mats2, emb2 = [m.clone() for m in mats], emb.clone()
     a = MuonAdamW(mats, [dict(params=[emb])])
-    b = DistributedMuonAdamW(mats2, [dict(params=[emb2])])
+    b = DistributedMuonAdamW(mats2, [dict(params=[emb2])], grad_dtype=gdt, adamw_grad_dtype=gdt)
     assert b.owned == [0, 1]
     for step in range(3):
         g = torch.Generator(device=dev)
         g.manual_seed(step)
-        for x, y in zip(mats + [emb], mats2 + [emb2]):
-            x.grad = torch.randn(x.shape, generator=g, device=dev)
-            y.grad = x.grad.clone()
-        a.step()
+        grads = [torch.randn(x.shape, generator=g, device=dev).to(gdt) for x in mats + [emb]]
+        for k, gr in enumerate(grads):
+            (b.muon_grads[k] if k < 2 else b.adamw_grads[0][0]).copy_(gr)
+        a.step(muon_grads=grads[:2], adamw_grads=[[grads[2]]])
         b.step()
     for x, y in zip(mats + [emb], mats2 + [emb2]):
         assert torch.equal(x, y)
