@@ -187,22 +187,37 @@ muon_status muon_reduce_mean(void* const* dst, const void* const* const* sources
  * and allocates nothing.
  *
  * Same arguments and semantics as muon_step, minus the workspace.  Limit: the
- * largest single matrix must fit, i.e. muon_workspace_min_size(groups) <=
- * MUON_NOALLOC_SCRATCH_BYTES (32 MiB: e.g. up to 2048 x 2048 or 1024 x 4096);
- * larger sets are processed in waves; a matrix that does not fit returns
- * MUON_ERR_WORKSPACE with the sizes in muon_last_error().  Every GPU that
- * loads this library holds the array until the process exits.  The first
- * call on a device looks up the array's device address (make it before any
- * stream capture).  All calls on a device share the array: calls that overlap
- * on the GPU race and must be ordered by the caller (e.g. one stream).
- * muon_query_status(NULL, ...) cannot read its status word; a device-side
- * timeout is not reported for this entry point.
+ * largest single matrix must fit, i.e. muon_workspace_min_size(groups, flags)
+ * <= MUON_NOALLOC_SCRATCH_BYTES (32 MiB: with bf16 operands up to about
+ * 2048 x 2048 or 1024 x 7168; with MUON_FP32_DEBUG, whose buffers are twice
+ * as large, up to about 1600 x 1600 or 1024 x 3072); larger sets are
+ * processed in waves; a matrix that does not fit returns MUON_ERR_WORKSPACE
+ * with the sizes in muon_last_error().  Every GPU that loads this library
+ * holds the array until the process exits.  Each call looks up the array's
+ * device address in the current context; the first call on a device (or
+ * after a device reset) also loads the library's device code, so make it
+ * before any stream capture.  All calls on a device share the array: calls
+ * that overlap on the GPU race and must be ordered by the caller (e.g. one
+ * stream).  The status word of the last step is read with
+ * muon_query_status() on the address muon_noalloc_scratch() returns.
  */
 #define MUON_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 muon_status muon_step_noalloc(float* const* params, const void* const* grads,
                               float* const* momentum, const muon_group* groups, int n_groups,
                               float lr, float beta, float wd, int ns_steps, const float* coeffs,
                               uint32_t flags, muon_stream_t stream);
+
+/*
+ * The built-in scratch of muon_step_noalloc on the current device: its device
+ * address (*device_ptr) and size (*bytes, MUON_NOALLOC_SCRATCH_BYTES; bytes
+ * may be NULL).  Allocates nothing.  Its first 4 bytes are the status word of
+ * the last muon_step_noalloc on the device: muon_query_status(*device_ptr,
+ * stream) reports MUON_ERR_TIMEOUT if a device-side wait of that step ran
+ * out.  The rest of the array is the step's scratch; a caller writes nothing
+ * there.  Returns MUON_ERR_INVALID_ARG for a NULL device_ptr and MUON_ERR_CUDA
+ * if the address cannot be looked up (no device, or no context).
+ */
+muon_status muon_noalloc_scratch(void** device_ptr, size_t* bytes);
 
 /*
  * The orthogonaliser alone: outputs[i] <- NS(inputs[i]) as fp32, rows x cols,

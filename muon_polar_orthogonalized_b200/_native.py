@@ -58,6 +58,7 @@ SIGNATURES = {
     "muon_step_noalloc": (c_int, [POINTER(c_void_p), POINTER(c_void_p), POINTER(c_void_p),
                                   POINTER(MuonGroup), c_int, c_float, c_float, c_float, c_int,
                                   POINTER(c_float), c_uint32, c_void_p]),
+    "muon_noalloc_scratch": (c_int, [POINTER(c_void_p), POINTER(c_size_t)]),
     "muon_orthogonalize": (c_int, [POINTER(c_void_p), POINTER(c_void_p), POINTER(MuonGroup), c_int,
                                    c_int, POINTER(c_float), c_uint32, c_void_p, c_size_t, c_void_p]),
     "adamw_step": (c_int, [POINTER(AdamWGroup), c_int, c_int64, c_void_p]),

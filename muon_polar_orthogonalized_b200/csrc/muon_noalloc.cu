@@ -10,17 +10,20 @@
 //
 // The array lives in this library's device image, so every GPU that loads
 // the library holds it (MUON_NOALLOC_SCRATCH_BYTES) until the process exits.
-// Its device address is looked up once per device, on that device's first
-// call, with cudaGetSymbolAddress; make that first call before any stream
-// capture.  All calls on a device share the one array: calls that overlap on
-// the GPU (different streams, no ordering between them) race on it, so order
-// them (one stream, or events).  The array keeps the previous call's
-// contents; the step itself clears what must start at zero (the status word)
-// and overwrites the rest before reading it.
+// Host code cannot use the array's name as a device address; every call looks
+// the address up with cudaGetSymbolAddress on the current device (cheap once
+// the device code is loaded), so a device reset or another context on the
+// device never sees a stale address.  The first call on a device, or after a
+// reset, loads the device code: make it before any stream capture.  All calls
+// on a device share the one array: calls that overlap on the GPU (different
+// streams, no ordering between them) race on it, so order them (one stream,
+// or events).  The array keeps the previous call's contents; the step itself
+// clears what must start at zero (the status word) and overwrites the rest
+// before reading it.  muon_noalloc_scratch hands out the array's address so
+// that muon_query_status can read the status word of the last step.
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/muon_b200.h"
 
@@ -31,25 +34,20 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MUON_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (set up once per device).
+// Device address of g_noalloc_scratch in the current device's context.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return cudaSuccess;
+}
+
+muon_status lookup_failed(cudaError_t e) {
+  char msg[256];
+  snprintf(msg, sizeof(msg), "muon_step_noalloc scratch: address lookup failed: %s", cudaGetErrorString(e));
+  muon_set_last_error(msg);
+  return MUON_ERR_CUDA;
 }
 
 }  // namespace
@@ -76,13 +74,20 @@ extern "C" muon_status muon_step_noalloc(float* const* params, const void* const
   }
   void* ws = nullptr;
   const cudaError_t e = scratch_address(&ws);
-  if (e != cudaSuccess) {
-    char msg[256];
-    snprintf(msg, sizeof(msg), "muon_step_noalloc: scratch address lookup failed: %s",
-             cudaGetErrorString(e));
-    muon_set_last_error(msg);
-    return MUON_ERR_CUDA;
-  }
+  if (e != cudaSuccess) return lookup_failed(e);
   return muon_step(params, grads, momentum, groups, n_groups, lr, beta, wd, ns_steps, coeffs,
                    flags, ws, MUON_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" muon_status muon_noalloc_scratch(void** device_ptr, size_t* bytes) {
+  if (!device_ptr) {
+    muon_set_last_error("muon_noalloc_scratch: device_ptr is NULL");
+    return MUON_ERR_INVALID_ARG;
+  }
+  void* ws = nullptr;
+  const cudaError_t e = scratch_address(&ws);
+  if (e != cudaSuccess) return lookup_failed(e);
+  *device_ptr = ws;
+  if (bytes) *bytes = MUON_NOALLOC_SCRATCH_BYTES;
+  return MUON_OK;
 }
