@@ -52,7 +52,7 @@ struct AdamTensor {
   float b1, omb1;    // beta1, 1 - beta1
   float b2, omb2;
   float step_size;   // lr / (1 - beta1^t)
-  float sqrt_bc2;    // sqrt(1 - beta2^t)
+  float rsqrt_bc2;   // 1 / sqrt(1 - beta2^t)
   float eps;
   float lr, wd;      // base values (device schedule: the scalars above are recomputed)
 };

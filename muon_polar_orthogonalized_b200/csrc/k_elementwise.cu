@@ -31,14 +31,11 @@
 
 namespace muon {
 
-// Launch shapes, chosen by measurement on B200 (isolated, 1G elements):
-// the momentum / update kernels stream 2-3 arrays and run best at full
-// occupancy (8 x 256 threads per SM) with 2 vec4 units per thread; AdamW
-// streams 4 arrays and runs best with 4 units per thread at 4 blocks per SM.
-// At that budget (64 registers for 1024 threads per SM) ptxas keeps about 200
-// bytes per AdamW thread in local memory; 2 blocks of 512 threads (the same
-// budget) measured alike.  A budget without the spill (fewer threads per SM)
-// has not been measured yet.
+// Launch shapes: the momentum / update kernels stream 2-3 arrays and run
+// best at full occupancy (8 x 256 threads per SM) with 2 vec4 units per
+// thread (measured on B200, isolated, 1G elements).  AdamW streams 4 arrays;
+// with its approximate square root and division it needs 32 registers at 2
+// units per thread and full occupancy, with nothing in local memory.
 #ifndef MUON_ELT_UNROLL
 #define MUON_ELT_UNROLL 2
 #endif
@@ -46,10 +43,10 @@ namespace muon {
 #define MUON_ELT_MIN_BLOCKS 8
 #endif
 #ifndef MUON_ADAM_UNROLL
-#define MUON_ADAM_UNROLL 4
+#define MUON_ADAM_UNROLL 2
 #endif
 #ifndef MUON_ADAM_MIN_BLOCKS
-#define MUON_ADAM_MIN_BLOCKS 4
+#define MUON_ADAM_MIN_BLOCKS 8
 #endif
 constexpr int kEltThreads = 256;
 constexpr int kEltUnroll = MUON_ELT_UNROLL;                  // vec4 units per thread
@@ -663,13 +660,26 @@ __device__ __forceinline__ int find_tensor(const AdamTensor* t, int n, int blk) 
   return lo;
 }
 
+// The square root and the division of the step take the hardware's
+// approximate forms (sqrt.approx: a few units in the last place; __fdividef:
+// 2 ulp for the denominators that occur here, >= eps): each leaves a relative
+// error near 1e-7 in the step lr*m/denom, ~1e-9 of p, while the
+// correctly-rounded forms cost about four times the instructions, which
+// matter at the 1.0-1.3 GHz a power-capped step runs at.  m and v are
+// computed exactly as the page's update writes them.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float r;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 __device__ __forceinline__ void adam_elem(const AdamTensor& T, float g, float& p, float& m,
                                           float& v) {
   p = p * T.decay;
   m = fmaf(T.b1, m, T.omb1 * g);
   v = fmaf(T.b2, v, T.omb2 * (g * g));
-  const float denom = sqrtf(v) / T.sqrt_bc2 + T.eps;
-  p = fmaf(-T.step_size, m / denom, p);
+  const float denom = fmaf(sqrt_approx(v), T.rsqrt_bc2, T.eps);
+  p = fmaf(-T.step_size, __fdividef(m, denom), p);
 }
 
 template <bool GBF16>
@@ -726,7 +736,7 @@ __device__ __forceinline__ void sched_scalars(AdamTensor& T, const DevSched* s) 
   const double lr = static_cast<double>(T.lr) * static_cast<double>(s->lr_mult);
   T.decay = static_cast<float>(1.0 - lr * static_cast<double>(T.wd));
   T.step_size = static_cast<float>(lr / (1.0 - pow(static_cast<double>(T.b1), t)));
-  T.sqrt_bc2 = static_cast<float>(sqrt(1.0 - pow(static_cast<double>(T.b2), t)));
+  T.rsqrt_bc2 = static_cast<float>(1.0 / sqrt(1.0 - pow(static_cast<double>(T.b2), t)));
 }
 
 template <bool GBF16>
