@@ -308,7 +308,7 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 
 def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: int = 5,
                                 eps: float = NS_EPS, fold_a: bool = False, exact_diag: bool = False,
-                                rounding=None) -> np.ndarray:
+                                diag_scale: bool = False, rounding=None) -> np.ndarray:
     """The iteration with bf16 rounding wherever a bf16 matrix is stored.
 
     [MAC] casts to bf16 before iterating and keeps X, A, B in bf16.  Storage
@@ -324,12 +324,18 @@ def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: in
     lo_i = d_i - bf16(d_i), is kept unrounded beside the stored B' and added
     back as lo_i * X_ij, so X' = bf16(B' X + lo * X): B' keeps its diagonal
     exactly and only its off-diagonal entries are rounded.
+    diag_scale (with fold_a): row i of the product is multiplied by
+    r_i = d_i / bf16(d_i), so X' = bf16(r * (B' X)): the diagonal term
+    d_i X_i comes out exact and the off-diagonal terms of row i are scaled by
+    r_i = 1 + O(2^-9).
     rounding: the function applied at every storage point (round_bf16 by
     default); the identity turns every mode into the exact iteration.
     """
     rnd = round_bf16 if rounding is None else rounding
-    if exact_diag and not fold_a:
-        raise ValueError("exact_diag applies to the folded B'")
+    if (exact_diag or diag_scale) and not fold_a:
+        raise ValueError("exact_diag and diag_scale apply to the folded B'")
+    if exact_diag and diag_scale:
+        raise ValueError("exact_diag and diag_scale are alternatives")
     g = np.asarray(g, dtype=np.float64)
     s = 1.0 / (np.sqrt(np.sum(g * g)) + eps)
     x = rnd(g)
@@ -345,6 +351,10 @@ def newton_schulz_bf16_emulated(g: np.ndarray, coeffs=NS_COEFFS_FIXED, steps: in
             if exact_diag:
                 lo = np.diag(Bfull) - np.diag(B)
                 x = rnd(sk * (B @ x + lo[:, None] * x))
+            elif diag_scale:
+                d, h = np.diag(Bfull), np.diag(B)
+                r = np.where(h != 0, d / np.where(h != 0, h, 1.0), 1.0)
+                x = rnd(sk * (B @ x) * r[:, None])
             else:
                 x = rnd(sk * (B @ x))
         else:

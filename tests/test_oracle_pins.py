@@ -234,7 +234,8 @@ def test_torch_muon_cross_check(pages):
 
 
 EMUL_MODES = {"pages": {}, "fold_a": {"fold_a": True},
-              "fold_a_exact_diag": {"fold_a": True, "exact_diag": True}}
+              "fold_a_exact_diag": {"fold_a": True, "exact_diag": True},
+              "fold_a_diag_scale": {"fold_a": True, "diag_scale": True}}
 
 
 @pytest.mark.parametrize("mode", list(EMUL_MODES))
@@ -252,7 +253,8 @@ def test_bf16_emulation_close_to_fp64(mode):
 def test_bf16_emulation_algebra_is_exact(mode):
     """With rounding switched off, each storage layout is an exact rewriting
     of the pages' iteration (deferred scale; a*X + B X = (a I + B) X; the
-    diagonal split B' = bf16(B') + diag(lo)), so it must reproduce the fp64
+    diagonal split B' = bf16(B') + diag(lo); the row scale d/bf16(d) = 1
+    without rounding), so it must reproduce the fp64
     oracle -- itself pinned to the SVD closed form -- on wide, tall and
     ragged inputs, for several step counts and a per-step table."""
     kw = EMUL_MODES[mode]
@@ -273,6 +275,8 @@ def test_bf16_emulation_first_order_bound_on_diagonal_input():
       pages:      t u (|a + q| + |b| t^2 + 2|c| t^4 + |q|)     (A, B, X' rounded)
       fold_a:     t u (2|a + q| + |b| t^2 + 2|c| t^4)          (A, B', X' rounded)
       exact_diag: t u (|a + q| + |b| t^2 + 2|c| t^4)           (A, X' rounded)
+      diag_scale: the same as exact_diag (a diagonal B' has no off-diagonal
+                  terms for the row scale to touch)
     (times 1 + 4u for the second-order terms).  Each mode must stay inside its
     own bound; folding without the exact diagonal must leave the exact-diagonal
     bound somewhere (the diagonal of B' is then rounded)."""
@@ -288,6 +292,7 @@ def test_bf16_emulation_first_order_bound_on_diagonal_input():
     bound = {"pages": t * u * (np.abs(a + q) + common + np.abs(q)) * (1 + 4 * u),
              "fold_a": t * u * (2 * np.abs(a + q) + common) * (1 + 4 * u),
              "fold_a_exact_diag": t * u * (np.abs(a + q) + common) * (1 + 4 * u)}
+    bound["fold_a_diag_scale"] = bound["fold_a_exact_diag"]
     err = {}
     for mode, kw in EMUL_MODES.items():
         x = oracle.newton_schulz_bf16_emulated(G, steps=1, **kw)
