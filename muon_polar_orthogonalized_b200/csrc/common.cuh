@@ -58,10 +58,11 @@ struct GemmProblem {
   // epilogue
   void* out; long long out_bs; int out_ld;
   const void* ein; long long ein_bs; int ein_ld;   // A (poly) or X (axpy)
-  // exact diagonal of B' (tensor-core path): the A*A epilogue writes
-  // lo_i = B'_ii - bf16(B'_ii) for every row; the B'X epilogue adds lo * X,
-  // lo indexed by the output row (wide) or column (tall, dlo_col = 1)
-  float* dlo; long long dlo_bs; int dlo_col;
+  // exact diagonal of B' (tensor-core path): the A*A epilogue writes, per
+  // row, r_i = B'_ii / bf16(B'_ii) (fp32); the B'X epilogue multiplies the
+  // product's row i (wide) or column i (tall, dsc_col = 1) by r_i, which
+  // makes the diagonal term exact
+  float* dsc; long long dsc_bs; int dsc_col;
   int scale_mode;           // 0 none, 1: s^2 (first Gram), 2: s (first X update)
   int scale_base;           // index of matrix 0 of this problem in the scale array
   float ca, cb, cc;         // a_k, b_k, c_k

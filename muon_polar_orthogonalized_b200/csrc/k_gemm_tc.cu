@@ -12,14 +12,14 @@
 //                                read transposed from the stored upper form;
 //                                the epilogue reads the A tile for b*A, adds
 //                                a on the diagonal and keeps, per row, the
-//                                part of the diagonal that bf16 drops:
-//                                lo_i = B'_ii - bf16(B'_ii), in fp32
-//   axpy  X' = s (B' X + lo X)   = s (a X + B X) with B''s diagonal exact;
-//                                wide matrices; tall ones (iterated as X^T)
-//                                compute X' = s (X B' + X lo) in parameter
+//                                ratio r_i = B'_ii / bf16(B'_ii) in fp32
+//   axpy  X' = s r (B' X)        = s (a X + B X) with B''s diagonal exact:
+//                                row i of the product scaled by r_i makes
+//                                its diagonal term exact; wide matrices; tall
+//                                ones (iterated as X^T) compute
+//                                X' = s (X B') r (column scale) in parameter
 //                                layout; B' is read like A above.  a X rides
-//                                in the product; the epilogue adds lo_i X_ij
-//                                (X read at the output's position) and scales
+//                                in the product; the epilogue only scales
 //   axpy_update                  last iteration: U = bf16(X') feeds the
 //                                cautious-decay update of W directly
 // s is the Frobenius scale 1/(||m~||+1e-7), applied on the first iteration
@@ -151,10 +151,10 @@ __device__ __forceinline__ void record_timeout(unsigned int* status, volatile in
   atomicOr(status, kDevTimeout);
 }
 
-// Row store of one chunk straight from registers (A*A products): 4 x 16 bytes
-// per lane.
-__device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+// Row store of one chunk straight from registers (A*A products): 2 x 32
+// bytes per lane where the row is 32-byte aligned, else 4 x 16 bytes.
+__device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[32], bool v8) {
+  uint4 d[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t w[4];
@@ -163,7 +163,15 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
       __nv_bfloat162 b = __floats2bfloat162_rn(v[q * 8 + h * 2], v[q * 8 + h * 2 + 1]);
       w[h] = *reinterpret_cast<uint32_t*>(&b);
     }
-    d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    d[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (v8) {
+    sm100::st_global_v8(dst, d[0], d[1]);
+    sm100::st_global_v8(dst + 16, d[2], d[3]);
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d4[q] = d[q];
   }
 }
 
@@ -224,9 +232,9 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
 template <int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const GemmProblem& q,
                                                   int mat, int i, int jt, int width) {
-  if (EPI == EPI_GRAM || i >= q.M) return;
+  if (EPI == EPI_GRAM || EPI == EPI_AXPY || i >= q.M) return;
   const int ncols = min(width, q.N - jt);  // jt < N
-  if (EPI == EPI_POLY || ((EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) && q.dlo)) {
+  if (EPI == EPI_POLY) {
     const char* ein = reinterpret_cast<const char*>(
         static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + jt);
     for (int b = 0; b < ncols * 2; b += 128) prefetch_l2(ein + b);
@@ -239,23 +247,28 @@ __device__ __forceinline__ void epilogue_prefetch(const TcGemmParams& p, const G
 }
 
 struct EpiIn {
-  uint4 e[4];     // 32 bf16 of the epilogue operand: A (A*A) or X (B'X)
+  uint4 e[4];     // 32 bf16 of the epilogue operand A (A*A products)
 };
 struct EpiW {
   float4 w[8];    // 32 fp32 parameters (fused update)
 };
 
-// The bf16 operand of one chunk: A for A*A, X for the exact-diagonal term of
-// B'X (nothing for the Gram).
+// The bf16 operand A of one chunk (A*A products only).
 template <int EPI>
 __device__ __forceinline__ void epilogue_load(const TcGemmParams& p, const GemmProblem& q, int mat,
                                               int i, int j0, bool full, EpiIn& in) {
   if (i >= q.M) return;
-  if ((EPI == EPI_POLY || ((EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) && q.dlo)) && full) {
-    const uint4* e4 = reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0);
+  if (EPI == EPI_POLY && full) {
+    const __nv_bfloat16* src =
+        static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs + static_cast<long long>(i) * q.ein_ld + j0;
+    if (((q.ein_ld | q.ein_bs) & 15) == 0) {   // 32-byte rows (the buffers are 1024-byte aligned)
+      sm100::ld_global_v8(src, in.e[0], in.e[1]);
+      sm100::ld_global_v8(src + 16, in.e[2], in.e[3]);
+    } else {
+      const uint4* e4 = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) in.e[k] = e4[k];
+      for (int k = 0; k < 4; ++k) in.e[k] = e4[k];
+    }
   }
 }
 
@@ -266,9 +279,17 @@ __device__ __forceinline__ void epilogue_load_w(const TcGemmParams& p, const Gem
   if (i >= q.M) return;
   if (EPI == EPI_AXPY_UPDATE && full && wvec) {
     const int wi = q.w_first + mat;
-    const float4* w4 = reinterpret_cast<const float4*>(p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0);
+    const float* src = p.wptr[wi] + static_cast<long long>(i) * p.wcols[wi] + j0;
+    if ((reinterpret_cast<uintptr_t>(src) & 31u) == 0) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) in.w[k] = w4[k];
+      for (int k = 0; k < 4; ++k)
+        sm100::ld_global_v8(src + 8 * k, *reinterpret_cast<uint4*>(&in.w[2 * k]),
+                            *reinterpret_cast<uint4*>(&in.w[2 * k + 1]));
+    } else {
+      const float4* w4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) in.w[k] = w4[k];
+    }
   }
 }
 
@@ -285,16 +306,33 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&e)[4], float (&a)[3
   }
 }
 
+// Called by every lane of the warp (the tall B'X column scale is shuffled).
+// dsc: B'X's diagonal scale r of this thread's row (wide), or of column
+// j0 + lane (tall: lane c supplies column j0 + c's to every lane).
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const GemmProblem& q, int mat,
                                                int i, int j0, bool full, bool wvec,
-                                               const EpiIn& in, const EpiW& win, float (&v)[32]) {
-  if (i >= q.M) return;
+                                               const EpiIn& in, const EpiW& win, float dsc,
+                                               float (&v)[32]) {
   float f = 1.f;
   if (q.scale_mode) {
     const float s = p.scales[q.scale_base + mat];
     f = (q.scale_mode == 1) ? s * s : s;
   }
+  if constexpr (EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) {
+    // both orientations multiply the accumulator by the one product r * s,
+    // so that a matrix and its transpose give the same bits
+    if (q.dsc) {
+      if (q.dsc_col) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] *= __shfl_sync(0xffffffffu, dsc, c) * f;
+        f = 1.f;
+      } else {
+        f *= dsc;
+      }
+    }
+  }
+  if (i >= q.M) return;
   if constexpr (EPI == EPI_POLY) {
     float a[32];
     if (full) {
@@ -307,64 +345,17 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
     }
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] = fmaf(q.cb, a[c], q.cc * v[c]) + ((j0 + c == i) ? q.ca : 0.f);
-    if (q.dlo && i >= j0 && i < j0 + 32) {
-      // this row's diagonal element: keep what its bf16 rounding drops (exact
-      // in fp32, the two values being within a factor of two of each other)
-      float lo = 0.f;
+    if (q.dsc && i >= j0 && i < j0 + 32) {
+      // this row's diagonal element d: keep d / bf16(d), by which B'X scales
+      // the product's row i so that its diagonal term d X_i comes out exact
+      float d = 0.f;
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        if (j0 + c == i) lo = v[c] - __bfloat162float(__float2bfloat16_rn(v[c]));
-      q.dlo[mat * q.dlo_bs + i] = lo;
+        if (j0 + c == i) d = v[c];
+      const float h = __bfloat162float(__float2bfloat16_rn(d));
+      q.dsc[mat * q.dsc_bs + i] = (h != 0.f) ? d / h : 1.f;
     }
   } else {
-    if constexpr (EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) {
-      if (q.dlo) {
-        // B''s exact diagonal: add lo * X at the output's own position
-        const float* lo = q.dlo + mat * q.dlo_bs;
-        if (!q.dlo_col && full) {
-          const float l = lo[i];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t w[4] = {in.e[u].x, in.e[u].y, in.e[u].z, in.e[u].w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[h]));
-              v[u * 8 + h * 2] = fmaf(l, f.x, v[u * 8 + h * 2]);
-              v[u * 8 + h * 2 + 1] = fmaf(l, f.y, v[u * 8 + h * 2 + 1]);
-            }
-          }
-        } else {
-        float x[32];
-        if (full) {
-          unpack_bf16x32(in.e, x);
-        } else {
-          const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(q.ein) + mat * q.ein_bs +
-                                    static_cast<long long>(i) * q.ein_ld + j0;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) x[c] = (j0 + c < q.N) ? __bfloat162float(xr[c]) : 0.f;
-        }
-        if (!q.dlo_col) {
-          const float l = lo[i];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) v[c] = fmaf(l, x[c], v[c]);
-        } else if (full) {
-          const float4* l4 = reinterpret_cast<const float4*>(lo + j0);   // ldm pitch: 32-byte rows
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 l = l4[c4];
-            v[c4 * 4 + 0] = fmaf(l.x, x[c4 * 4 + 0], v[c4 * 4 + 0]);
-            v[c4 * 4 + 1] = fmaf(l.y, x[c4 * 4 + 1], v[c4 * 4 + 1]);
-            v[c4 * 4 + 2] = fmaf(l.z, x[c4 * 4 + 2], v[c4 * 4 + 2]);
-            v[c4 * 4 + 3] = fmaf(l.w, x[c4 * 4 + 3], v[c4 * 4 + 3]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (j0 + c < q.N) v[c] = fmaf(lo[j0 + c], x[c], v[c]);
-        }
-        }
-      }
-    }
     // Gram: s^2 on the first iteration; axpy: s on the first iteration
 #pragma unroll
     for (int c = 0; c < 32; ++c) v[c] *= f;
@@ -379,7 +370,6 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
     const bool cautious = p.cautious != 0;
     const float lr = p.sched ? q.lr * p.sched->lr_mult : q.lr;
     if (full && wvec) {
-      float4* w4 = reinterpret_cast<float4*>(w);
       float4 nw[8];
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
@@ -389,13 +379,22 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
         ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), lr, p.wd, cautious);
         ww.w = cautious_w(ww.w, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 3])), lr, p.wd, cautious);
         nw[c4] = ww;
-        w4[c4] = ww;
       }
-      for (int r = 0; r < p.nrep; ++r) {
-        float4* d4 = reinterpret_cast<float4*>(p.rptr[r][wi] + roff);
+      // W and each copy: 32-byte stores where the row segment is 32-byte aligned
+      auto store_row = [&](float* dst) {
+        if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) d4[c4] = nw[c4];
-      }
+          for (int k = 0; k < 4; ++k)
+            sm100::st_global_v8(dst + 8 * k, *reinterpret_cast<const uint4*>(&nw[2 * k]),
+                                *reinterpret_cast<const uint4*>(&nw[2 * k + 1]));
+        } else {
+          float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) d4[c4] = nw[c4];
+        }
+      };
+      store_row(w);
+      for (int r = 0; r < p.nrep; ++r) store_row(p.rptr[r][wi] + roff);
     } else {
 #pragma unroll
       for (int c = 0; c < 32; ++c)
@@ -408,7 +407,7 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
   } else if constexpr (EPI == EPI_POLY) {
     __nv_bfloat16* row = static_cast<__nv_bfloat16*>(q.out) + mat * q.out_bs + static_cast<long long>(i) * q.out_ld + j0;
     if (full) {
-      st_bf16x32(row, v);
+      st_bf16x32(row, v, ((q.out_ld | q.out_bs) & 15) == 0);
     } else {
 #pragma unroll
       for (int c = 0; c < 32; ++c)
@@ -639,13 +638,12 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       }
       // Active chunks form one range [c_lo, c_hi): a symmetric tile skips the
       // chunks left of its rows' 256-block (a prefix) and a ragged tile stops
-      // at N.  B'X keeps kXAhead chunks of X in flight: the first ones are
-      // loaded before the accumulator is ready (the epilogue warps are idle
-      // while the tile's MMAs run), each later one when a buffer frees up.
-      // For A*A the A operand of chunk c+1 is loaded while chunk c is
-      // combined and stored; the fused update loads X and W (both
-      // prefetched to L2 above) with each chunk; the Gram epilogue loads
-      // nothing.
+      // at N.  A*A loads its operand A one chunk ahead (the first one before
+      // the accumulator is ready); the fused update loads W (prefetched to L2
+      // above) with each chunk; the Gram and B'X epilogues load nothing but
+      // B'X's diagonal scales, once per tile.  (Requesting chunk c+1's
+      // accumulator columns from TMEM before storing chunk c measured no
+      // faster on the wide products.)
       // symmetric output in upper form: chunks left of the rows' 256-block are not stored
       const int rblk = row0 / kSymBlock;
       int c_hi = 0;
@@ -653,15 +651,42 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       int c_lo = 0;
       if (q.sym) c_lo = max(0, (kSymBlock * rblk - jslice) / 32);
       auto chunk_j0 = [&](int cc) { return jslice + cc * 32; };
-      constexpr int kXAhead = 2;
-      EpiIn xb[kXAhead];
-      if constexpr (EPI == EPI_AXPY) {
-        if (q.dlo) {
+      constexpr bool kOperand = (EPI == EPI_POLY);   // operand loaded one chunk ahead
+      auto load_operand = [&](int cc, EpiIn& in) {
+        if constexpr (kOperand) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc), chunk_j0(cc) + 32 <= q.N, in);
+      };
+      EpiIn ea, eb;   // operands of the even / odd chunk of a pair
+      if (c_lo < c_hi) load_operand(c_lo, ea);
+      // B'X: r_i of this thread's row (wide), or r_j of column jslice + 32 u
+      // + lane for each chunk u (tall; shuffled to every lane in the epilogue)
+      float dsc_row = 1.f;
+      float dsc_t[kChunks];
 #pragma unroll
-          for (int k = 0; k < kXAhead; ++k)
-            if (k < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(k), chunk_j0(k) + 32 <= q.N, xb[k]);
+      for (int u = 0; u < kChunks; ++u) dsc_t[u] = 1.f;
+      if constexpr (EPI == EPI_AXPY || EPI == EPI_AXPY_UPDATE) {
+        if (q.dsc) {
+          const float* d = q.dsc + tc.mat * q.dsc_bs;
+          if (!q.dsc_col) {
+            if (i < q.M) dsc_row = d[i];
+          } else {
+#pragma unroll
+            for (int u = 0; u < kChunks; ++u) {
+              const int jc = jslice + u * 32 + lane;
+              if (jc < q.N) dsc_t[u] = d[jc];
+            }
+          }
         }
       }
+      auto dsc_of = [&](int cc) {   // selects, no indexed register array
+        float r = dsc_row;
+        if (q.dsc_col) {
+          r = dsc_t[0];
+#pragma unroll
+          for (int u = 1; u < kChunks; ++u)
+            if (cc == u) r = dsc_t[u];
+        }
+        return r;
+      };
       if (!sm100::mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) {
         record_timeout(p.status, abort_flag);
         break;
@@ -669,60 +694,40 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       sm100::tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * C::BN);
-      auto process = [&](int cc, const EpiIn& in_prev) {
+      auto tmem_req = [&](int cc, uint32_t (&r)[32]) {
+        sm100::tmem_ld32_async(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), r);
+      };
+      auto process = [&](int cc, const EpiIn& in) {
         const int j0 = chunk_j0(cc);
         const bool full = (j0 + 32 <= q.N);
         EpiW win;
         epilogue_load_w<EPI>(p, q, tc.mat, i, j0, full, wvec, win);
-        // the fused update loads its X chunk with W (no register room for a
-        // second chunk in flight); the other epilogues got theirs one chunk ahead
-        EpiIn in_now;
-        if constexpr (EPI == EPI_AXPY_UPDATE) epilogue_load<EPI>(p, q, tc.mat, i, j0, full, in_now);
-        const EpiIn& in = (EPI == EPI_AXPY_UPDATE) ? in_now : in_prev;
+        uint32_t r[32];
+        tmem_req(cc, r);
+        sm100::tmem_wait_ld(r);
         float v[32];
-        sm100::tmem_ld32(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), v);
-        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, in, win, v);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r[k]);
+        epilogue_store<EPI>(p, q, tc.mat, i, j0, full, wvec, in, win, dsc_of(cc), v);
         if constexpr (EPI == EPI_GRAM || EPI == EPI_AXPY) {
           stage_row_store(&p.tmOut[tc.prob], my_staging + (stage_ctr & 1) * TC_STAGE_TILE_BYTES, lane, v, j0,
                           row0 + quad * 32, q.M, tc.mat);
           ++stage_ctr;
         }
       };
-      if constexpr (EPI == EPI_GRAM || EPI == EPI_AXPY_UPDATE) {
+      if constexpr (kOperand) {
 #pragma unroll 1
-        for (int cc = c_lo; cc < c_hi; ++cc) {
-          const EpiIn none{};
-          process(cc, none);
-        }
-      } else if constexpr (EPI == EPI_AXPY) {
-        // c_lo = 0 (not symmetric); the inner loop is unrolled so that xb[]
-        // stays in registers
-        static_assert(kChunks % kXAhead == 0, "whole rounds of X buffers");
-#pragma unroll 1
-        for (int c0 = 0; c0 < kChunks; c0 += kXAhead) {
-#pragma unroll
-          for (int k = 0; k < kXAhead; ++k) {
-            const int cc = c0 + k;
-            if (cc < c_hi) {
-              process(cc, xb[k]);
-              if (q.dlo && cc + kXAhead < c_hi)
-                epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc + kXAhead), chunk_j0(cc + kXAhead) + 32 <= q.N,
-                                   xb[k]);
-            }
+        for (int cc = c_lo; cc < c_hi; cc += 2) {
+          if (cc + 1 < c_hi) load_operand(cc + 1, eb);
+          process(cc, ea);
+          if (cc + 1 < c_hi) {
+            if (cc + 2 < c_hi) load_operand(cc + 2, ea);
+            process(cc + 1, eb);
           }
         }
       } else {
-        EpiIn in0, in1;
-        if (c_lo < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(c_lo), chunk_j0(c_lo) + 32 <= q.N, in0);
 #pragma unroll 1
-        for (int cc = c_lo; cc < c_hi; cc += 2) {
-          if (cc + 1 < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc + 1), chunk_j0(cc + 1) + 32 <= q.N, in1);
-          process(cc, in0);
-          if (cc + 1 < c_hi) {
-            if (cc + 2 < c_hi) epilogue_load<EPI>(p, q, tc.mat, i, chunk_j0(cc + 2), chunk_j0(cc + 2) + 32 <= q.N, in0);
-            process(cc + 1, in1);
-          }
-        }
+        for (int cc = c_lo; cc < c_hi; ++cc) process(cc, ea);
       }
       sm100::tc_fence_before();
       __syncwarp();

@@ -212,7 +212,7 @@ struct WaveItem {
   size_t x0, x1, b;     // byte offsets in the workspace
   int sbase;            // index of the item's first matrix in the wave's scale array
   long long pbase;      // first partial sum of the item's first matrix (wave-relative)
-  size_t lo = 0;        // byte offset of the item's diagonal residuals (ldm floats per matrix)
+  size_t dsc = 0;       // byte offset of the item's diagonal scales of B' (ldm floats per matrix)
 };
 
 struct Wave {
@@ -245,7 +245,7 @@ size_t layout_wave(Wave& w, const std::vector<GroupGeom>& geo) {
     off = align_up(off + q.xstride * it.count, 1024);
     it.b = off;
     off = align_up(off + q.bstride * it.count, 1024);
-    it.lo = off;
+    it.dsc = off;
     off = align_up(off + 4ull * q.ldm * it.count, 1024);
   }
   w.total = off;
@@ -666,7 +666,7 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       P.sym = 1;
       P.out = bbuf; P.out_bs = bs_el; P.out_ld = q.ldm;   // B' = a I + b A + c A A
       P.ein = xoth; P.ein_bs = xs_el; P.ein_ld = q.ldm;
-      if (!f32) { P.dlo = reinterpret_cast<float*>(a.ws + it.lo); P.dlo_bs = q.ldm; }
+      if (!f32) { P.dsc = reinterpret_cast<float*>(a.ws + it.dsc); P.dsc_bs = q.ldm; }
     } else {
       P.M = q.r;
       P.N = q.c;
@@ -682,10 +682,9 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldc;
       P.scale_mode = (k == 0) ? 2 : 0;
       if (!f32) {
-        // the part of B''s diagonal that bf16 drops comes back as lo * X,
-        // X read at the output's own position
-        P.dlo = reinterpret_cast<float*>(a.ws + it.lo); P.dlo_bs = q.ldm; P.dlo_col = q.tall;
-        P.ein = xcur; P.ein_bs = xs_el; P.ein_ld = q.ldc;
+        // row (wide) or column (tall) i of the product scaled by
+        // B'_ii / bf16(B'_ii): its diagonal term is then exact
+        P.dsc = reinterpret_cast<float*>(a.ws + it.dsc); P.dsc_bs = q.ldm; P.dsc_col = q.tall;
       }
     }
     // the tensor-core path stores A and B' in upper form and reads them so;

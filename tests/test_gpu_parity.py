@@ -100,16 +100,17 @@ def test_orthogonalize_bf16_parity(dev, dtype):
         e = rel(u, ref)
         gate = bf16_gate(r, c, 5, pages_bf16_error(x))
         # diagnostic, stricter than the gate: the kernel's own storage points
-        # (a folded into B', B''s diagonal kept exact), emulated
-        emu = rel(u, oracle.newton_schulz_bf16_emulated(x, FIXED, 5, fold_a=True, exact_diag=True))
+        # (a folded into B', the product's rows scaled so that B''s diagonal
+        # acts exactly), emulated
+        emu = rel(u, oracle.newton_schulz_bf16_emulated(x, FIXED, 5, fold_a=True, diag_scale=True))
         print(f"{r}x{c}: rel err vs fp64 {e:.3e} (gate {gate:.3e}), vs kernel-storage emulation {emu:.3e}")
         assert np.isfinite(u).all(), (r, c)
         assert e <= gate, ((r, c), e, gate)
         assert emu <= 1.5e-2, ((r, c), emu)
         if max(r, c) <= 64:
             # tiny: the kernel follows the emulated storage points up to its
-            # fp32 (not fp64) diagonal residual, which can move a single
-            # rounding by one bf16 unit (a misplaced rounding moves ~1e-2)
+            # fp32 (not fp64) diagonal scale, which can move a single rounding
+            # by one bf16 unit (a misplaced rounding moves ~1e-2)
             assert emu <= 5e-4, ((r, c), emu)
 
 
