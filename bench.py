@@ -54,8 +54,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
 # set: same seven shapes, 1 layer instead of 32).
 TRAFFIC_CAPTURES = {
-    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "2e92259ec58a2537",
-                "bytes_per_launch": {"llama_8b_32l": 32 * 1288274944, "llama_8b_1layer": 1288274944}},
+    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "bd71312e2e2d7932",
+                "bytes_per_launch": {"llama_8b_32l": 32 * 1037614336, "llama_8b_1layer": 1037614336}},
 }
 
 
