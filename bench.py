@@ -46,16 +46,17 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM traffic per launch of a kernel, from one ncu capture of the named
-# kernel sources (their fingerprint: sha256 prefix of the files listed with
-# comments removed, source_fingerprint).  When the sources differ
-# from the captured ones the figure no longer describes the kernel and the
-# roofline reports traffic = null.  Captured on the one-layer slice of the 8B
-# shapes and scaled x32 to a full launch (the slice is exactly 1/32 of the
-# set: same seven shapes, 1 layer instead of 32).
+# DRAM traffic of one pass of a product (its launches over every matrix of
+# the step), from one ncu capture of the named sources (the kernel and the
+# planner that composes its launches; their fingerprint: sha256 prefix of the
+# files listed with comments removed, source_fingerprint).  When the sources
+# differ from the captured ones the figure no longer describes the kernel and
+# the roofline reports traffic = null.  Captured on the one-layer slice of
+# the 8B shapes and scaled x32 (the slice is exactly 1/32 of the set: same
+# seven shapes, 1 layer instead of 32).
 TRAFFIC_CAPTURES = {
-    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh"], "sha": "bd71312e2e2d7932",
-                "bytes_per_launch": {"llama_8b_32l": 32 * 1037614336, "llama_8b_1layer": 1037614336}},
+    "ns_axpy": {"sources": ["k_gemm_tc.cu", "sm100.cuh", "common.cuh", "muon_api.cu"], "sha": "96e3b0633bb2ea27",
+                "bytes_per_pass": {"llama_8b_32l": 32 * 996114944, "llama_8b_1layer": 996114944}},
 }
 
 
@@ -74,14 +75,15 @@ def source_fingerprint(files) -> str:
 
 
 def captured_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu capture, or None once the
-    kernel's sources have changed since that capture."""
+    """DRAM bytes of one pass of the product from the committed ncu capture,
+    or None once the kernel's or the planner's sources have changed since that
+    capture."""
     cap = TRAFFIC_CAPTURES.get(kernel)
-    if not cap or workload not in cap["bytes_per_launch"]:
+    if not cap or workload not in cap["bytes_per_pass"]:
         return None
     if source_fingerprint(cap["sources"]) != cap["sha"]:
         return None
-    return cap["bytes_per_launch"][workload]
+    return cap["bytes_per_pass"][workload]
 
 
 def load_peaks():
@@ -336,7 +338,8 @@ def run_gpu(args):
     flags = (N.MUON_NESTEROV | N.MUON_CAUTIOUS_WD | (N.MUON_TC_SINGLE_CTA if args.single_cta else 0)
              | (N.MUON_NORMUON if args.normuon else 0)
              | (N.MUON_ROW_EQUILIBRATE if args.row_equilibrate else 0)
-             | (N.MUON_TC_NARROW_TILES if args.narrow_tiles else 0))
+             | (N.MUON_TC_NARROW_TILES if args.narrow_tiles else 0)
+             | (N.MUON_TC_WIDE_TILES if args.wide_tiles else 0))
     ws_bytes = api.muon_workspace_size(D.groups, flags)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     coeffs = W.NS_COEFFS_FIXED
@@ -492,12 +495,17 @@ def run_gpu(args):
             launches_per_step = n / args.steps
             per_launch = per_step_work[dom] / launches_per_step
             avg_s = ms / n / 1e3
+            # DRAM bytes of an average launch: the captured pass times the
+            # passes per step, over the launches per step
+            passes = {"ns_axpy": n_axpy, "ns_gram": K, "ns_poly": K, "ns_axpy_update": 1}.get(dom, 1)
+            cap_pass = captured_traffic(dom, wl.name)
+            traffic = round(cap_pass * passes / launches_per_step) if cap_pass else None
             if bound == "tensor":
                 ach = per_launch / avg_s / 1e12
                 peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
                 roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-                        "traffic": captured_traffic(dom, wl.name), "traffic_unit": "bytes per launch",
+                        "traffic": traffic, "traffic_unit": "bytes per launch",
                         "peak_source": f"{peak_src} (sustained bf16 cuBLAS)",
                         "work_per_launch": per_launch, "work_unit": "executed FLOP"}
             else:
@@ -505,7 +513,7 @@ def run_gpu(args):
                 peak = peaks["hbm_gbs"]
                 roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
                         "unit": "GB/s", "frac": round(ach / peak, 4),
-                        "traffic": captured_traffic(dom, wl.name), "traffic_unit": "bytes per launch",
+                        "traffic": traffic, "traffic_unit": "bytes per launch",
                         "peak_source": f"{peak_src} (HBM copy)",
                         "work_per_launch": per_launch, "work_unit": "algorithmic bytes"}
         ew = {}
@@ -539,7 +547,9 @@ def run_gpu(args):
                        "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
                        "gemm_tiles": "128x256 single-CTA" if args.single_cta else
                        "CTA pairs: 256x256" if args.narrow_tiles else
-                       "CTA pairs: 256x512 (Gram, B'X), 256x256 (A*A, fused update)",
+                       "CTA pairs: 256x512 (Gram, B'X), 256x256 (A*A, fused update)" if args.wide_tiles else
+                       "CTA pairs: Gram and B'X on 256x512 where the output width is a multiple of "
+                       "512 and K >= 2048, else 256x256; A*A and the fused update 256x256",
                        "normuon": bool(args.normuon), "row_equilibrate": bool(args.row_equilibrate)},
             "ns_tflops_executed": round(ns_exe / (ns_ms / 1e3) / 1e12, 1) if ns_ms else None,
             "ns_frac_of_peak_executed": round(ns_exe / (ns_ms / 1e3) / 1e12 / sustained, 4) if ns_ms else None,
@@ -801,7 +811,9 @@ def main():
     ap.add_argument("--row-equilibrate", action="store_true",
                     help="MuonEq row equilibration of the momentum-smoothed matrix before Newton-Schulz")
     ap.add_argument("--narrow-tiles", action="store_true",
-                    help="Gram and B'X on 256x256 CTA-pair tiles instead of 256x512")
+                    help="Gram and B'X on 256x256 CTA-pair tiles for every shape")
+    ap.add_argument("--wide-tiles", action="store_true",
+                    help="Gram and B'X on 256x512 CTA-pair tiles for every shape")
     ap.add_argument("--single-cta", action="store_true",
                     help="Newton-Schulz GEMMs on single-CTA 128x256 tiles instead of CTA pairs")
     ap.add_argument("--distributed", action="store_true",

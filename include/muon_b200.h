@@ -72,8 +72,13 @@ enum {
                                row of U (parameter orientation) by (||row||/sqrt(cols) + 1e-8) before
                                the decay and update, so each row's RMS is 1 and the step's is lr */
   MUON_TC_NARROW_TILES = 128u, /* run the Gram and B'X products on 256x256 CTA-pair tiles with two
-                               TMEM accumulators (as A*A and the fused update always are) instead of
-                               256x512 tiles with one; same results, for comparison */
+                               TMEM accumulators (as A*A and the fused update always are) for every
+                               shape; same results, for comparison.  By default a product runs on
+                               256x512 tiles with one accumulator only where its output width is a
+                               multiple of 512 and its K is at least 2048, where they are faster */
+  MUON_TC_WIDE_TILES = 256u, /* run the Gram and B'X products on 256x512 CTA-pair tiles for every
+                               shape; same results, for comparison (MUON_TC_NARROW_TILES wins if
+                               both are given) */
   MUON_ROW_EQUILIBRATE = 64u /* MuonEq row equilibration ("Stuck at the optimizer after figuring out
                                backward()", mira687's reply, names it without a formula): divide every
                                row of m~ (parameter orientation) by (||row|| + 1e-7) before the

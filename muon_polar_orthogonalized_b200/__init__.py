@@ -8,7 +8,8 @@ The optimizer classes live in `optimizer` (MuonAdamW) and `distributed`
 """
 from ._native import (MUON_BF16, MUON_CAUTIOUS_WD, MUON_F32, MUON_FP32_DEBUG,  # noqa: F401
                       MUON_NESTEROV, MUON_NORMUON, MUON_ROW_EQUILIBRATE, MUON_TC_NARROW_TILES,
-                      MUON_TC_SINGLE_CTA, MUON_UNFUSED_UPDATE, MuonError, MuonGroup)
+                      MUON_TC_SINGLE_CTA, MUON_TC_WIDE_TILES, MUON_UNFUSED_UPDATE, MuonError,
+                      MuonGroup)
 from .api import (AdamWSpec, adamw_step, adamw_step_scheduled, muon_orthogonalize,  # noqa: F401
                   muon_profiler_enable, muon_profiler_read, muon_profiler_reset,
                   muon_query_status, muon_reduce_mean, muon_schedule_advance,

@@ -33,6 +33,7 @@ MUON_TC_SINGLE_CTA = 16
 MUON_NORMUON = 32
 MUON_ROW_EQUILIBRATE = 64
 MUON_TC_NARROW_TILES = 128
+MUON_TC_WIDE_TILES = 256
 
 
 class MuonGroup(ctypes.Structure):

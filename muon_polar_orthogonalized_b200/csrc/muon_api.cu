@@ -565,18 +565,24 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
 }
 
 // Build and launch one NS product (epi) for every item of the wave.
-// Products that run on 512-column CTA-pair tiles (bit per EpiKind) unless
-// MUON_TC_NARROW_TILES or single-CTA mode is requested.  The wide tile reads
-// 25% fewer operand bytes from L2 per FLOP, so at the same SM cycles it draws
-// less power and runs at a higher clock under the 1 kW cap; its single
-// 512-column accumulator is drained without overlap.  Measured on 8 layers
-// of the 8B shapes: the Gram and B'X (whose epilogue only scales and stores)
-// take the same cycles on either tile and less time on the wide one; A*A
-// (epilogue reads A) and the fused-update B'X (reads and writes W) take
-// 25-35% more time on it.
+// Products that may run on 512-column CTA-pair tiles (bit per EpiKind).  The
+// wide tile reads 25% fewer operand bytes from L2 per FLOP, so at the same SM
+// cycles it draws less power and runs at a higher clock under the 1 kW cap;
+// its single 512-column accumulator is drained without overlap.  Measured on
+// 8 layers of the 8B shapes: the Gram and B'X (whose epilogue only scales and
+// stores) take the same cycles on either tile and less time on the wide one;
+// A*A (epilogue reads A) and the fused-update B'X (reads and writes W) take
+// 4-40% more time on it.  A problem of those products takes the wide tile
+// where its output width is a multiple of 512 (no partly empty tiles) and its
+// K at least kWideMinK (the undrained accumulator's epilogue is then a small
+// part of each tile); on the d=768 and d=1664 transformer sets, with K of 768
+// and 1664 and widths of 768 and 1664, the narrow tile was 13% and 5% faster
+// per step.  MUON_TC_NARROW_TILES / MUON_TC_WIDE_TILES force one tile for
+// every problem (same bits either way).
 #ifndef MUON_TC_WIDE_EPIS
 #define MUON_TC_WIDE_EPIS 0x5
 #endif
+constexpr int kWideMinK = 2048;
 
 muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
   const StepArgs& a = C.a;
@@ -584,10 +590,20 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
   const float ca = a.coeffs[3 * k], cb = a.coeffs[3 * k + 1], cc = a.coeffs[3 * k + 2];
   const float* scales = reinterpret_cast<const float*>(a.ws + w.scales_off);
   const bool pair = (a.flags & MUON_TC_SINGLE_CTA) == 0;
-  const bool wide = pair && !f32 && (a.flags & MUON_TC_NARROW_TILES) == 0 && ((MUON_TC_WIDE_EPIS >> epi) & 1);
+  const bool wide_ok = pair && !f32 && (a.flags & MUON_TC_NARROW_TILES) == 0 && ((MUON_TC_WIDE_EPIS >> epi) & 1);
+  const bool wide_all = wide_ok && (a.flags & MUON_TC_WIDE_TILES) != 0;
+  // the tile width of one item's problem (see above)
+  auto item_wide = [&](const GroupGeom& q) {
+    if (!wide_ok) return false;
+    if (wide_all) return true;
+    const int width = (epi == EPI_GRAM || epi == EPI_POLY) ? q.m : q.c;   // output columns
+    const int K = (epi == EPI_GRAM) ? q.n : q.m;
+    return width % 512 == 0 && K >= kWideMinK;
+  };
   const int BM = f32 ? simt_tile() : tc_tile_m(pair);
-  const int BN = f32 ? simt_tile() : tc_tile_n(wide);
   const int b_rows = tc_b_box_rows(pair);
+  bool wide = false;   // tile width of the launch being built
+  int BN = 0;
 
   static thread_local TcGemmParams TP;
   static thread_local SimtGemmParams SP;
@@ -626,149 +642,158 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
     return MUON_OK;
   };
 
-  for (const auto& it : w.items) {
-    if (nprob == kMaxProblems || nw + it.count > kMaxUpdMats) {
-      muon_status st = flush();
-      if (st != MUON_OK) return st;
-    }
-    const GroupGeom& q = C.geo[it.g];
-    const muon_group& g = a.groups[it.g];
-    char* xcur = a.ws + (x_in_0 ? it.x0 : it.x1);
-    char* xoth = a.ws + (x_in_0 ? it.x1 : it.x0);
-    char* bbuf = a.ws + it.b;
-    const long long xs_el = static_cast<long long>(q.xstride / q.esz);
-    const long long bs_el = static_cast<long long>(q.bstride / q.esz);
-    GemmProblem P;
-    std::memset(&P, 0, sizeof(P));
-    P.batch = it.count;
-    P.scale_base = it.sbase;
-    P.ca = ca;
-    P.cb = cb;
-    P.cc = cc;
-    P.lr = a.lr * g.lr_scale;
-    P.w_first = nw;
-    // operand / output roles
-    if (epi == EPI_GRAM) {
-      P.M = P.N = q.m;
-      P.K = q.n;
-      P.a_mn = P.b_mn = q.tall;
-      P.a = P.b = xcur;
-      P.a_bs = P.b_bs = xs_el;
-      P.a_ld = P.b_ld = q.ldc;
-      P.sym = 1;
-      P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldm;   // A lives in the other X buffer
-      P.scale_mode = (k == 0) ? 1 : 0;
-    } else if (epi == EPI_POLY) {
-      P.M = P.N = P.K = q.m;
-      P.a = P.b = xoth;
-      P.a_bs = P.b_bs = xs_el;
-      P.a_ld = P.b_ld = q.ldm;
-      P.sym = 1;
-      P.out = bbuf; P.out_bs = bs_el; P.out_ld = q.ldm;   // B' = a I + b A + c A A
-      P.ein = xoth; P.ein_bs = xs_el; P.ein_ld = q.ldm;
-      if (!f32) { P.dsc = reinterpret_cast<float*>(a.ws + it.dsc); P.dsc_bs = q.ldm; }
-    } else {
-      P.M = q.r;
-      P.N = q.c;
-      P.K = q.m;
-      // a X + B X = B' X with B' = a I + B from the A*A epilogue
-      if (!q.tall) {  // X' = B' X : Aop = B' (K-major), Bop = X (MN-major)
-        P.a = bbuf; P.a_bs = bs_el; P.a_ld = q.ldm; P.a_mn = 0;
-        P.b = xcur; P.b_bs = xs_el; P.b_ld = q.ldc; P.b_mn = 1;
-      } else {        // X' = X B' : Aop = X (K-major), Bop = B' (K-major, symmetric)
-        P.a = xcur; P.a_bs = xs_el; P.a_ld = q.ldc; P.a_mn = 0;
-        P.b = bbuf; P.b_bs = bs_el; P.b_ld = q.ldm; P.b_mn = 0;
+  // two passes: the problems on wide tiles, then those on narrow ones
+  for (int pass = 0; pass < 2; ++pass) {
+    wide = (pass == 0);
+    if (wide && !wide_ok) continue;
+    BN = f32 ? simt_tile() : tc_tile_n(wide);
+    for (const auto& it : w.items) {
+      if (item_wide(C.geo[it.g]) != wide) continue;
+      if (nprob == kMaxProblems || nw + it.count > kMaxUpdMats) {
+        muon_status st = flush();
+        if (st != MUON_OK) return st;
       }
-      P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldc;
-      P.scale_mode = (k == 0) ? 2 : 0;
-      if (!f32) {
-        // row (wide) or column (tall) i of the product scaled by
-        // B'_ii / bf16(B'_ii): its diagonal term is then exact
-        P.dsc = reinterpret_cast<float*>(a.ws + it.dsc); P.dsc_bs = q.ldm; P.dsc_col = q.tall;
-      }
-    }
-    // the tensor-core path stores A and B' in upper form and reads them so;
-    // the fp32 scaffold computes and reads full matrices
-    if (!f32) {
-      if (epi == EPI_POLY) P.a_sym = P.b_sym = 1;
-      else if (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) (q.tall ? P.b_sym : P.a_sym) = 1;
-    }
-    if (f32) P.sym = 0;
-    // B'X of a wide matrix: tile rows fastest, so that B' (m x m, indexed by
-    // the tile row) stays in L2 while each X panel streams through once
-    P.col_major = (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) && !q.tall;
-    P.tiles_m = (P.M + BM - 1) / BM;
-    P.tiles_n = (P.N + BN - 1) / BN;
-    if (P.sym) {
-      int t = 0;
-      for (int I = 0; I < P.tiles_m; ++I) t += P.tiles_n - (I * BM) / BN;
-      P.tiles_per_mat = t;
-    } else {
-      P.tiles_per_mat = P.tiles_m * P.tiles_n;
-    }
-    P.tile_begin = tiles;
-    const long long add = static_cast<long long>(P.tiles_per_mat) * it.count;
-    if (tiles + add > (1ll << 30)) return fail(MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
-    if (!f32) {
-      // tensor maps: the natural 3-D view (inner, rows, batch) of each buffer
-      auto map_for = [&](CUtensorMap* m, const void* base, int mn, int inner, int rows, int ld,
-                         size_t bstride, int box_rows) {
-        return make_map(m, const_cast<void*>(base), inner, rows, it.count, static_cast<size_t>(ld) * 2,
-                        bstride, 64, mn ? 64 : box_rows);
-      };
-      muon_status st;
-      // A boxes: 128 rows per CTA; B boxes: the rows of B this CTA stages
+      const GroupGeom& q = C.geo[it.g];
+      const muon_group& g = a.groups[it.g];
+      char* xcur = a.ws + (x_in_0 ? it.x0 : it.x1);
+      char* xoth = a.ws + (x_in_0 ? it.x1 : it.x0);
+      char* bbuf = a.ws + it.b;
+      const long long xs_el = static_cast<long long>(q.xstride / q.esz);
+      const long long bs_el = static_cast<long long>(q.bstride / q.esz);
+      GemmProblem P;
+      std::memset(&P, 0, sizeof(P));
+      P.batch = it.count;
+      P.scale_base = it.sbase;
+      P.ca = ca;
+      P.cb = cb;
+      P.cc = cc;
+      P.lr = a.lr * g.lr_scale;
+      P.w_first = nw;
+      // operand / output roles
       if (epi == EPI_GRAM) {
-        st = map_for(&TP.tmA[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, b_rows);
+        P.M = P.N = q.m;
+        P.K = q.n;
+        P.a_mn = P.b_mn = q.tall;
+        P.a = P.b = xcur;
+        P.a_bs = P.b_bs = xs_el;
+        P.a_ld = P.b_ld = q.ldc;
+        P.sym = 1;
+        P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldm;   // A lives in the other X buffer
+        P.scale_mode = (k == 0) ? 1 : 0;
       } else if (epi == EPI_POLY) {
-        // A in upper form: K-major boxes, plus MN-major boxes for its transposed K blocks
-        st = map_for(&TP.tmA[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, b_rows);
-        if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
-        if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
-      } else if (!q.tall) {
-        // B' in upper form (A operand here)
-        st = map_for(&TP.tmA[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, 1, q.c, q.r, q.ldc, q.xstride, b_rows);
-        if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
+        P.M = P.N = P.K = q.m;
+        P.a = P.b = xoth;
+        P.a_bs = P.b_bs = xs_el;
+        P.a_ld = P.b_ld = q.ldm;
+        P.sym = 1;
+        P.out = bbuf; P.out_bs = bs_el; P.out_ld = q.ldm;   // B' = a I + b A + c A A
+        P.ein = xoth; P.ein_bs = xs_el; P.ein_ld = q.ldm;
+        if (!f32) { P.dsc = reinterpret_cast<float*>(a.ws + it.dsc); P.dsc_bs = q.ldm; }
       } else {
-        // B' in upper form (B operand here)
-        st = map_for(&TP.tmA[nprob], xcur, 0, q.c, q.r, q.ldc, q.xstride, 128);
-        if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, b_rows);
-        if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
-      }
-      // Gram and B'X output rows are written by TMA stores of 32 x 32 boxes
-      // (64-byte swizzle); A*A and the fused update store directly
-      if (st == MUON_OK && (epi == EPI_GRAM || epi == EPI_AXPY)) {
-        const bool sq = (epi == EPI_GRAM);
-        const int out_inner = sq ? q.m : q.c, out_rows = sq ? q.m : q.r, out_ld = sq ? q.ldm : q.ldc;
-        st = make_map(&TP.tmOut[nprob], P.out, out_inner, out_rows, it.count,
-                      static_cast<size_t>(out_ld) * 2, q.xstride, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-      }
-      if (st != MUON_OK) return st;
-      TP.prob[nprob] = P;
-    } else {
-      SP.prob[nprob] = P;
-    }
-    if (epi == EPI_AXPY_UPDATE) {
-      for (int j = 0; j < it.count; ++j) {
-        const int pi = g.first + it.first + j;
-        if (f32) {
-          SP.wptr[nw + j] = a.params[pi];
-          SP.wcols[nw + j] = q.c;
-        } else {
-          TP.wptr[nw + j] = a.params[pi];
-          TP.wcols[nw + j] = q.c;
-          for (int r = 0; r < a.nrep; ++r) TP.rptr[r][nw + j] = a.replicas[r][pi];
+        P.M = q.r;
+        P.N = q.c;
+        P.K = q.m;
+        // a X + B X = B' X with B' = a I + B from the A*A epilogue
+        if (!q.tall) {  // X' = B' X : Aop = B' (K-major), Bop = X (MN-major)
+          P.a = bbuf; P.a_bs = bs_el; P.a_ld = q.ldm; P.a_mn = 0;
+          P.b = xcur; P.b_bs = xs_el; P.b_ld = q.ldc; P.b_mn = 1;
+        } else {        // X' = X B' : Aop = X (K-major), Bop = B' (K-major, symmetric)
+          P.a = xcur; P.a_bs = xs_el; P.a_ld = q.ldc; P.a_mn = 0;
+          P.b = bbuf; P.b_bs = bs_el; P.b_ld = q.ldm; P.b_mn = 0;
+        }
+        P.out = xoth; P.out_bs = xs_el; P.out_ld = q.ldc;
+        P.scale_mode = (k == 0) ? 2 : 0;
+        if (!f32) {
+          // row (wide) or column (tall) i of the product scaled by
+          // B'_ii / bf16(B'_ii): its diagonal term is then exact
+          P.dsc = reinterpret_cast<float*>(a.ws + it.dsc); P.dsc_bs = q.ldm; P.dsc_col = q.tall;
         }
       }
+      // the tensor-core path stores A and B' in upper form and reads them so;
+      // the fp32 scaffold computes and reads full matrices
+      if (!f32) {
+        if (epi == EPI_POLY) P.a_sym = P.b_sym = 1;
+        else if (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) (q.tall ? P.b_sym : P.a_sym) = 1;
+      }
+      if (f32) P.sym = 0;
+      // B'X of a wide matrix: tile rows fastest, so that B' (m x m, indexed by
+      // the tile row) stays in L2 while each X panel streams through once
+      P.col_major = (epi == EPI_AXPY || epi == EPI_AXPY_UPDATE) && !q.tall;
+      P.tiles_m = (P.M + BM - 1) / BM;
+      P.tiles_n = (P.N + BN - 1) / BN;
+      if (P.sym) {
+        int t = 0;
+        for (int I = 0; I < P.tiles_m; ++I) t += P.tiles_n - (I * BM) / BN;
+        P.tiles_per_mat = t;
+      } else {
+        P.tiles_per_mat = P.tiles_m * P.tiles_n;
+      }
+      P.tile_begin = tiles;
+      const long long add = static_cast<long long>(P.tiles_per_mat) * it.count;
+      if (tiles + add > (1ll << 30)) return fail(MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
+      if (!f32) {
+        // tensor maps: the natural 3-D view (inner, rows, batch) of each buffer
+        auto map_for = [&](CUtensorMap* m, const void* base, int mn, int inner, int rows, int ld,
+                           size_t bstride, int box_rows) {
+          return make_map(m, const_cast<void*>(base), inner, rows, it.count, static_cast<size_t>(ld) * 2,
+                          bstride, 64, mn ? 64 : box_rows);
+        };
+        muon_status st;
+        // A boxes: 128 rows per CTA; B boxes: the rows of B this CTA stages
+        if (epi == EPI_GRAM) {
+          st = map_for(&TP.tmA[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, 128);
+          if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, q.tall, q.c, q.r, q.ldc, q.xstride, b_rows);
+        } else if (epi == EPI_POLY) {
+          // A in upper form: K-major boxes, plus MN-major boxes for its transposed K blocks
+          st = map_for(&TP.tmA[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, 128);
+          if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, b_rows);
+          if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
+          if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
+        } else if (!q.tall) {
+          // B' in upper form (A operand here)
+          st = map_for(&TP.tmA[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, 128);
+          if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, 1, q.c, q.r, q.ldc, q.xstride, b_rows);
+          if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
+        } else {
+          // B' in upper form (B operand here)
+          st = map_for(&TP.tmA[nprob], xcur, 0, q.c, q.r, q.ldc, q.xstride, 128);
+          if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, b_rows);
+          if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
+        }
+        // Gram and B'X output rows are written by TMA stores of 32 x 32 boxes
+        // (64-byte swizzle); A*A and the fused update store directly
+        if (st == MUON_OK && (epi == EPI_GRAM || epi == EPI_AXPY)) {
+          const bool sq = (epi == EPI_GRAM);
+          const int out_inner = sq ? q.m : q.c, out_rows = sq ? q.m : q.r, out_ld = sq ? q.ldm : q.ldc;
+          st = make_map(&TP.tmOut[nprob], P.out, out_inner, out_rows, it.count,
+                        static_cast<size_t>(out_ld) * 2, q.xstride, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+        }
+        if (st != MUON_OK) return st;
+        TP.prob[nprob] = P;
+      } else {
+        SP.prob[nprob] = P;
+      }
+      if (epi == EPI_AXPY_UPDATE) {
+        for (int j = 0; j < it.count; ++j) {
+          const int pi = g.first + it.first + j;
+          if (f32) {
+            SP.wptr[nw + j] = a.params[pi];
+            SP.wcols[nw + j] = q.c;
+          } else {
+            TP.wptr[nw + j] = a.params[pi];
+            TP.wcols[nw + j] = q.c;
+            for (int r = 0; r < a.nrep; ++r) TP.rptr[r][nw + j] = a.replicas[r][pi];
+          }
+        }
+      }
+      nw += it.count;
+      tiles += static_cast<int>(add);
+      nprob += 1;
     }
-    nw += it.count;
-    tiles += static_cast<int>(add);
-    nprob += 1;
+    muon_status st = flush();
+    if (st != MUON_OK) return st;
   }
-  return flush();
+  return MUON_OK;
 }
 
 // dst[r][i] <- params[i] for every matrix of the wave (update paths that do
@@ -846,7 +871,8 @@ muon_status validate_common(const muon_group* groups, int n_groups, int ns_steps
   muon_status st = validate_groups(groups, n_groups);
   if (st != MUON_OK) return st;
   if (flags & ~(MUON_NESTEROV | MUON_CAUTIOUS_WD | MUON_FP32_DEBUG | MUON_UNFUSED_UPDATE |
-                MUON_TC_SINGLE_CTA | MUON_NORMUON | MUON_ROW_EQUILIBRATE | MUON_TC_NARROW_TILES))
+                MUON_TC_SINGLE_CTA | MUON_NORMUON | MUON_ROW_EQUILIBRATE | MUON_TC_NARROW_TILES |
+                MUON_TC_WIDE_TILES))
     return fail(MUON_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (ns_steps < 0 || ns_steps > kMaxNsSteps)
     return fail(MUON_ERR_INVALID_ARG, "ns_steps %d outside [0, %d]", ns_steps, kMaxNsSteps);

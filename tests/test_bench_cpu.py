@@ -48,7 +48,7 @@ def test_one_layer_slice_is_a_thirty_second_of_the_set():
     a, b = bench.algorithmic_work(full), bench.algorithmic_work(one)
     for k in ("gram_flops", "poly_flops", "axpy_flops", "momentum_bytes", "update_bytes"):
         assert a[k] == 32 * b[k], k
-    cap = bench.TRAFFIC_CAPTURES["ns_axpy"]["bytes_per_launch"]
+    cap = bench.TRAFFIC_CAPTURES["ns_axpy"]["bytes_per_pass"]
     assert cap["llama_8b_32l"] == 32 * cap["llama_8b_1layer"]
 
 

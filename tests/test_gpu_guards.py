@@ -25,7 +25,7 @@ GUARD_BYTES = 4096
 CANARY = 0xA5
 SHAPES = [(256, 1024), (1024, 256), (130, 200), (200, 130), (100, 300), (300, 100)]
 VARIANTS = [0, N.MUON_UNFUSED_UPDATE, N.MUON_NORMUON, N.MUON_ROW_EQUILIBRATE, N.MUON_FP32_DEBUG,
-            N.MUON_TC_NARROW_TILES]
+            N.MUON_TC_NARROW_TILES, N.MUON_TC_WIDE_TILES]
 
 
 def guarded_copy(t: torch.Tensor):

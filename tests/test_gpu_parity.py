@@ -221,22 +221,28 @@ def test_wide_and_narrow_tiles_agree(dev):
     """256x512 CTA-pair tiles (one 512-column accumulator, two N=256 MMAs per K
     step) and 256x256 tiles give identical bits for all three products, incl.
     shapes whose columns are not a multiple of 512 and several matrices per
-    launch; a full step with the fused update agrees too."""
-    shapes = [(256, 1024), (1024, 256), (384, 640), (640, 384), (129, 257), (700, 700), (512, 1800)]
-    a = orth_case(dev, shapes, "bf16", seed=23, counts=[2, 1, 1, 1, 3, 1, 1])[1]
-    b = orth_case(dev, shapes, "bf16", seed=23, counts=[2, 1, 1, 1, 3, 1, 1],
-                  flags=N.MUON_TC_NARROW_TILES)[1]
-    for x, y in zip(a, b):
-        assert np.array_equal(x, y)
+    launch, whether every problem takes one tile (forced either way) or each
+    takes its own (the default: wide only for widths that are multiples of
+    512 with K >= 2048, so that one product runs as two launches here); a
+    full step with the fused update agrees too."""
+    shapes = [(256, 1024), (1024, 256), (384, 640), (640, 384), (129, 257), (700, 700), (512, 1800),
+              (512, 2048), (2048, 512)]
+    counts = [2, 1, 1, 1, 3, 1, 1, 2, 1]
+    base = orth_case(dev, shapes, "bf16", seed=23, counts=counts)[1]
+    for flags in (N.MUON_TC_NARROW_TILES, N.MUON_TC_WIDE_TILES):
+        other = orth_case(dev, shapes, "bf16", seed=23, counts=counts, flags=flags)[1]
+        for x, y in zip(base, other):
+            assert np.array_equal(x, y), flags
     outs = []
-    for flags in (STEP_FLAGS, STEP_FLAGS | N.MUON_TC_NARROW_TILES):
+    for flags in (STEP_FLAGS, STEP_FLAGS | N.MUON_TC_NARROW_TILES, STEP_FLAGS | N.MUON_TC_WIDE_TILES):
         groups, W, G, M, _, _ = make_state(dev, [(384, 1536), (1536, 384)], "bf16", 24)
         ws = workspace(api.muon_workspace_size(groups, flags), dev)
         api.muon_step(W, G, M, groups, 0.02, 0.95, 0.01, 5, FIXED, flags, ws)
         torch.cuda.synchronize()
         outs.append([host64(w) for w in W])
-    for x, y in zip(*outs):
-        assert np.array_equal(x, y)
+    for other in outs[1:]:
+        for x, y in zip(outs[0], other):
+            assert np.array_equal(x, y)
 
 
 def test_batch_invariance_and_determinism(dev):

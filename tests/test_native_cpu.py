@@ -79,7 +79,7 @@ def _call_step(L, groups, ptr_count, ns=5, coeffs=True, flags=3, ws=0x1000, wsb=
     (dict(ns=17), N.MUON_ERR_INVALID_ARG),
     (dict(ns=-1), N.MUON_ERR_INVALID_ARG),
     (dict(coeffs=False), N.MUON_ERR_INVALID_ARG),
-    (dict(flags=256), N.MUON_ERR_INVALID_ARG),
+    (dict(flags=512), N.MUON_ERR_INVALID_ARG),
     (dict(ws=0), N.MUON_ERR_WORKSPACE),
     (dict(ws=0x1010), N.MUON_ERR_WORKSPACE),                                 # misaligned
     (dict(wsb=100), N.MUON_ERR_WORKSPACE),
