@@ -12,7 +12,8 @@ Inputs (~84 GB resident) are far larger than L2, so no flush is needed.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 cuda synchronize on both sides, CUDA events on the launching stream, max
-over ranks.  With N > 1 (torchrun), every rank runs its own replica of the
+over ranks; then K more steps with a CUDA-event pair around every launch for
+the per-kernel breakdown (kept out of the timed steps).  With N > 1 (torchrun), every rank runs its own replica of the
 workload on its GPU (matrices are independent problems; there is no data-path
 collective), so per-GPU work is fixed: weak scaling.
 
@@ -370,10 +371,11 @@ def run_gpu(args):
         raise RuntimeError("device status word reports an error after warm-up")
 
     # ---------------------------------------------------- device-timed region
+    # The K timed steps carry no per-kernel events (an event pair around
+    # every launch would add its own gaps to launch-bound steps); the
+    # per-kernel breakdown comes from K more steps with the profiler on.
     clocks = ClockSampler(local)
     clocks.start()
-    api.muon_profiler_reset()
-    api.muon_profiler_enable(True)
     barrier()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     evs[0].record(stream)
@@ -382,10 +384,17 @@ def run_gpu(args):
         evs[k + 1].record(stream)
     e0, e1 = evs[0], evs[-1]
     barrier()
-    api.muon_profiler_enable(False)
     clk = clocks.stop()
     ms_total = max_over_ranks(e0.elapsed_time(e1))
     per_step = sorted(evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps))
+    # ------------------------------------------ per-kernel breakdown (profiled)
+    api.muon_profiler_reset()
+    api.muon_profiler_enable(True)
+    barrier()
+    for k in range(args.steps):
+        step()
+    barrier()
+    api.muon_profiler_enable(False)
 
     def quantile(q):
         x = q * (len(per_step) - 1)
