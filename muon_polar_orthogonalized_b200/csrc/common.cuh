@@ -52,6 +52,9 @@ struct GemmProblem {
   int tiles_m, tiles_n, tiles_per_mat, tile_begin;
   int col_major;            // tile order of a non-symmetric output: tile rows fastest
                             // (else bands of tile columns, tile columns fastest)
+  int chunked;              // tensor-core path: every operand row length is a multiple
+                            // of 64, and the tensor maps are chunked 4-D views (one
+                            // box per operand per pipeline stage)
   // operands (SIMT path reads these directly; the tensor-core path uses tensor maps)
   const void* a; long long a_bs; int a_ld;
   const void* b; long long b_bs; int b_ld;

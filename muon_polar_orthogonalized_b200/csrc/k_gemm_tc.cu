@@ -56,7 +56,10 @@ namespace muon {
 // tile's MMAs.  NSUB = 2: one 512-column accumulator (all of TMEM), 25% fewer
 // operand bytes per FLOP from L2, the epilogue drain no longer overlapped.
 #ifndef MUON_TC_PAIR_STAGES
-#define MUON_TC_PAIR_STAGES 6
+#define MUON_TC_PAIR_STAGES 3
+#endif
+#ifndef MUON_TC_NARROW_BK
+#define MUON_TC_NARROW_BK 128
 #endif
 #ifndef MUON_TC_WIDE_STAGES
 #define MUON_TC_WIDE_STAGES 4
@@ -83,15 +86,26 @@ struct TcCfg {
   static_assert(NSUB == 1 || (PAIR && NSUB == 2), "512-column tiles need CTA pairs");
   static constexpr int BM = PAIR ? 256 : 128;        // tile rows
   static constexpr int BN = 256 * NSUB;              // tile columns
-  static constexpr int BK = 64;
+  // K per pipeline stage: 128 on 256x256 pair tiles (64 KB stages), else 64.
+  // An SM's TMA ingest is set by the number of copies per stage more than by
+  // their bytes (measured: a 32 KB stage moves 44 B/clk as two 16 KB boxes and
+  // 57 B/clk as one 32 KB box; a 64 KB stage 78 B/clk as two 32 KB boxes),
+  // and a 256x256 pair tile consumes 64 B/clk at the full MMA rate.
+  static constexpr int BK = (PAIR && NSUB == 1) ? MUON_TC_NARROW_BK : 64;
+  static constexpr int KCH = BK / 64;                // 64-wide K chunks per stage
+  static constexpr int MN_CHUNK_BYTES = BK * 128;    // MN-major: one 64-wide MN chunk of BK k-rows
   static constexpr int A_ROWS = 128;                 // A rows staged per CTA
   static constexpr int SUB_B_ROWS = PAIR ? 128 : 256;  // B rows staged per CTA per 256-column sub-tile
   static constexpr int B_ROWS = SUB_B_ROWS * NSUB;
+  static constexpr int A_CHUNK_BYTES = A_ROWS * 128;          // K-major: one 64-wide K chunk
+  static constexpr int SUB_B_CHUNK_BYTES = SUB_B_ROWS * 128;
   static constexpr int A_BYTES = A_ROWS * BK * 2;
   static constexpr int SUB_B_BYTES = SUB_B_ROWS * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = NSUB == 2 ? MUON_TC_WIDE_STAGES : PAIR ? MUON_TC_PAIR_STAGES : 4;
+  static_assert(BK == 64 || BK == 128, "K per stage");
+  static_assert(kSymBlock % BK == 0, "a K block lies inside one 256-block of an upper-form operand");
   static constexpr int ACC_BUFS = NSUB == 1 ? 2 : 1;   // TMEM accumulators (512 columns in all)
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;          // barriers, TMEM slot, abort flag
   static constexpr int STAGING_OFF = BAR_OFF + 1024;            // output staging (TC_STAGING_BYTES)
@@ -499,28 +513,34 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
             if (PAIR) sm100::tma_load_3d_pair(dst, m, leader_full, x, y, tc.mat);
             else sm100::tma_load_3d(dst, m, &full_bar[stage], x, y, tc.mat);
           };
+          auto load4 = [&](uint8_t* dst, const CUtensorMap* m, int y, int z) {
+            if (PAIR) sm100::tma_load_4d_pair(dst, m, leader_full, 0, y, z, tc.mat);
+            else sm100::tma_load_4d(dst, m, &full_bar[stage], 0, y, z, tc.mat);
+          };
+          // `rows` operand rows from row0 for this K block.  Shared-memory
+          // layout: K-major [K chunk][row][64 k]; MN-major [MN chunk][BK k][64 mn].
+          // Chunked maps bring it in one box; otherwise one box per 64-wide chunk.
+          auto load_operand = [&](uint8_t* dst, const CUtensorMap* m, bool mn, int row0, int rows) {
+            if (q.chunked) {
+              if (mn) load4(dst, m, k0, row0 / 64);
+              else load4(dst, m, row0, k0 / 64);
+            } else if (mn) {
+              for (int h = 0; h < rows / 64; ++h) load(dst + h * C::MN_CHUNK_BYTES, m, row0 + h * 64, k0);
+            } else {
+#pragma unroll
+              for (int c = 0; c < C::KCH; ++c) load(dst + c * rows * 128, m, k0 + c * 64, row0);
+            }
+          };
           // an upper-form operand's K block left of its rows' diagonal block
           // comes transposed from the block above the diagonal (MN-major)
           const bool a_t = q.a_sym && (k0 / kSymBlock) < (arow / kSymBlock);
-          if (!q.a_mn && !a_t) {
-            load(sa, &p.tmA[tc.prob], k0, arow);
-          } else {
-            const CUtensorMap* ma = a_t ? &p.tmA2[tc.prob] : &p.tmA[tc.prob];
-#pragma unroll
-            for (int h = 0; h < C::A_ROWS / 64; ++h) load(sa + h * 8192, ma, arow + h * 64, k0);
-          }
+          load_operand(sa, a_t ? &p.tmA2[tc.prob] : &p.tmA[tc.prob], q.a_mn || a_t, arow, C::A_ROWS);
 #pragma unroll
           for (int n = 0; n < NSUB; ++n) {
-            uint8_t* sbn = sb + n * C::SUB_B_BYTES;
             const int brow_n = brow + n * TC_BN;
             const bool b_t = q.b_sym && (k0 / kSymBlock) < (brow_n / kSymBlock);
-            if (!q.b_mn && !b_t) {
-              load(sbn, &p.tmB[tc.prob], k0, brow_n);
-            } else {
-              const CUtensorMap* mb = b_t ? &p.tmB2[tc.prob] : &p.tmB[tc.prob];
-#pragma unroll
-              for (int h = 0; h < C::SUB_B_ROWS / 64; ++h) load(sbn + h * 8192, mb, brow_n + h * 64, k0);
-            }
+            load_operand(sb + n * C::SUB_B_BYTES, b_t ? &p.tmB2[tc.prob] : &p.tmB[tc.prob], q.b_mn || b_t,
+                         brow_n, C::SUB_B_ROWS);
           }
           if (++stage == C::STAGES) {
             stage = 0;
@@ -575,24 +595,30 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           const uint32_t sb = sa + C::A_BYTES;
           const int kblk = (kb * C::BK) / kSymBlock;
           const bool a_mn = q.a_mn || (q.a_sym && kblk < ablk);
-          const uint64_t ad0 = a_mn ? sm100::make_sdesc(sa, 8192, 1024) : sm100::make_sdesc(sa, 16, 1024);
-          const uint64_t a_inc = a_mn ? (2048 >> 4) : (32 >> 4);
-          uint64_t bd0[NSUB], b_inc[NSUB];
+          const uint64_t ad0 = a_mn ? sm100::make_sdesc(sa, C::MN_CHUNK_BYTES, 1024) : sm100::make_sdesc(sa, 16, 1024);
+          uint64_t bd0[NSUB];
+          bool bmn[NSUB];
           uint32_t idn[NSUB];
 #pragma unroll
           for (int n = 0; n < NSUB; ++n) {
-            const bool b_mn = q.b_mn || (q.b_sym && kblk < bblk0 + (n * TC_BN) / kSymBlock);
+            bmn[n] = q.b_mn || (q.b_sym && kblk < bblk0 + (n * TC_BN) / kSymBlock);
             const uint32_t sbn = sb + n * C::SUB_B_BYTES;
-            bd0[n] = b_mn ? sm100::make_sdesc(sbn, 8192, 1024) : sm100::make_sdesc(sbn, 16, 1024);
-            b_inc[n] = b_mn ? (2048 >> 4) : (32 >> 4);
-            idn[n] = sm100::make_idesc_bf16(C::BM, TC_BN, a_mn ? 1 : 0, b_mn ? 1 : 0);
+            bd0[n] = bmn[n] ? sm100::make_sdesc(sbn, C::MN_CHUNK_BYTES, 1024) : sm100::make_sdesc(sbn, 16, 1024);
+            idn[n] = sm100::make_idesc_bf16(C::BM, TC_BN, a_mn ? 1 : 0, bmn[n] ? 1 : 0);
           }
+          // start-address step (16-byte units) of K16 step kk: MN-major 2048 B
+          // per step; K-major 32 B per step within a 64-wide chunk, then the
+          // next chunk
+          auto koff = [](bool mn, int kk, int chunk_bytes) -> uint64_t {
+            return mn ? static_cast<uint64_t>(kk * (2048 >> 4))
+                      : static_cast<uint64_t>(((kk >> 2) * chunk_bytes + (kk & 3) * 32) >> 4);
+          };
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
 #pragma unroll
             for (int n = 0; n < NSUB; ++n) {
-              const uint64_t ad = ad0 + static_cast<uint64_t>(kk) * a_inc;
-              const uint64_t bd = bd0[n] + static_cast<uint64_t>(kk) * b_inc[n];
+              const uint64_t ad = ad0 + koff(a_mn, kk, C::A_CHUNK_BYTES);
+              const uint64_t bd = bd0[n] + koff(bmn[n], kk, C::SUB_B_CHUNK_BYTES);
               const uint32_t dn = d_tmem + static_cast<uint32_t>(n * TC_BN);
               if (PAIR) sm100::umma_bf16_pair(dn, ad, bd, idn[n], (kb | kk) ? 1u : 0u);
               else sm100::umma_bf16(dn, ad, bd, idn[n], (kb | kk) ? 1u : 0u);
@@ -776,6 +802,9 @@ cudaError_t launch_selftest_wait(unsigned int* status, unsigned long long limit_
 int tc_tile_m(bool pair) { return pair ? TcCfg<true, 1>::BM : TcCfg<false, 1>::BM; }
 int tc_tile_n(bool wide) { return wide ? TcCfg<true, 2>::BN : TC_BN; }
 int tc_b_box_rows(bool pair) { return pair ? TcCfg<true, 1>::SUB_B_ROWS : TcCfg<false, 1>::SUB_B_ROWS; }
+int tc_bk(bool pair, bool wide) {
+  return wide ? TcCfg<true, 2>::BK : pair ? TcCfg<true, 1>::BK : TcCfg<false, 1>::BK;
+}
 
 template <int EPI, bool PAIR, int NSUB>
 static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_t s) {

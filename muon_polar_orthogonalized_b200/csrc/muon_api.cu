@@ -43,6 +43,7 @@ cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm,
 int tc_tile_m(bool pair);
 int tc_tile_n(bool wide);
 int tc_b_box_rows(bool pair);
+int tc_bk(bool pair, bool wide);
 cudaError_t launch_tc_gemm(const TcGemmParams& p, int epi, bool pair, bool wide, int num_sms, cudaStream_t s);
 cudaError_t launch_selftest_wait(unsigned int* status, unsigned long long limit_ns, cudaStream_t s);
 int simt_tile();
@@ -369,6 +370,31 @@ muon_status make_map(CUtensorMap* map, void* base, int inner, int rows, int batc
   if (r != CUDA_SUCCESS)
     return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %d x %d x %d", static_cast<int>(r),
                 inner, rows, batch);
+  return MUON_OK;
+}
+
+// A chunked 4-D view (64, rows, inner / 64, batch) of the same buffer: the
+// 64-element chunks of a row become a dimension of stride 128 bytes, so one
+// box of box_chunks chunks brings several 64-wide column blocks at once.
+// Used only where inner is a multiple of 64 and the row pitch equals inner
+// (no chunk reaches past a row); chunks beyond the view read as zeros.
+muon_status make_map_chunked(CUtensorMap* map, void* base, int inner, int rows, int batch, size_t row_bytes,
+                             size_t batch_bytes, int box_rows, int box_chunks) {
+  PFN_encodeTiled_t enc = get_encode();
+  if (!enc) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  if (inner % 64 != 0 || row_bytes != static_cast<size_t>(inner) * 2)
+    return fail(MUON_ERR_UNSUPPORTED, "chunked tensor map over a ragged or padded row (%d, %zu)", inner, row_bytes);
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(inner / 64),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(row_bytes), 128, static_cast<cuuint64_t>(batch_bytes)};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_chunks), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for the chunked view of %d x %d x %d",
+                static_cast<int>(r), inner, rows, batch);
   return MUON_OK;
 }
 
@@ -732,11 +758,19 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       const long long add = static_cast<long long>(P.tiles_per_mat) * it.count;
       if (tiles + add > (1ll << 30)) return fail(MUON_ERR_UNSUPPORTED, "too many tiles in one launch");
       if (!f32) {
-        // tensor maps: the natural 3-D view (inner, rows, batch) of each buffer
+        // tensor maps: where every operand row length is a multiple of 64,
+        // chunked 4-D views, so that a K-major operand block (op_rows x BK)
+        // or an MN-major one (BK k-rows x op_rows) is one box per stage; else
+        // the natural 3-D view (inner, rows, batch), one box per 64-wide chunk
+        const int bk = tc_bk(pair, wide);
+        P.chunked = (q.c % 64 == 0 && q.m % 64 == 0) ? 1 : 0;
         auto map_for = [&](CUtensorMap* m, const void* base, int mn, int inner, int rows, int ld,
-                           size_t bstride, int box_rows) {
+                           size_t bstride, int op_rows) {
+          if (P.chunked)
+            return make_map_chunked(m, const_cast<void*>(base), inner, rows, it.count, static_cast<size_t>(ld) * 2,
+                                    bstride, mn ? bk : op_rows, mn ? op_rows / 64 : bk / 64);
           return make_map(m, const_cast<void*>(base), inner, rows, it.count, static_cast<size_t>(ld) * 2,
-                          bstride, 64, mn ? 64 : box_rows);
+                          bstride, 64, mn ? bk : op_rows);
         };
         muon_status st;
         // A boxes: 128 rows per CTA; B boxes: the rows of B this CTA stages
@@ -747,18 +781,18 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
           // A in upper form: K-major boxes, plus MN-major boxes for its transposed K blocks
           st = map_for(&TP.tmA[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, 128);
           if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xoth, 0, q.m, q.m, q.ldm, q.xstride, b_rows);
-          if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
-          if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 64);
+          if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, 128);
+          if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], xoth, 1, q.m, q.m, q.ldm, q.xstride, b_rows);
         } else if (!q.tall) {
           // B' in upper form (A operand here)
           st = map_for(&TP.tmA[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, 128);
           if (st == MUON_OK) st = map_for(&TP.tmB[nprob], xcur, 1, q.c, q.r, q.ldc, q.xstride, b_rows);
-          if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
+          if (st == MUON_OK) st = map_for(&TP.tmA2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 128);
         } else {
           // B' in upper form (B operand here)
           st = map_for(&TP.tmA[nprob], xcur, 0, q.c, q.r, q.ldc, q.xstride, 128);
           if (st == MUON_OK) st = map_for(&TP.tmB[nprob], bbuf, 0, q.m, q.m, q.ldm, q.bstride, b_rows);
-          if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, 64);
+          if (st == MUON_OK) st = map_for(&TP.tmB2[nprob], bbuf, 1, q.m, q.m, q.ldm, q.bstride, b_rows);
         }
         // Gram and B'X output rows are written by TMA stores of 32 x 32 boxes
         // (64-byte swizzle); A*A and the fused update store directly

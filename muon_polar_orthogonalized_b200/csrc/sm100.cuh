@@ -135,6 +135,27 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// 4-D tiled loads, otherwise as above.  The GEMMs use them on a chunked
+// view of a matrix whose rows are split into 64-element chunks (the chunk
+// index a dimension of its own, stride 128 bytes), so that one box brings
+// several 64-wide chunks: fewer, larger copies per pipeline stage.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y,
+                                            int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster_addr,
+                                                 int x, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster_addr)
+      : "memory");
+}
+
 // 3-D tiled store from this CTA's shared memory to global memory, tracked in
 // the issuing thread's bulk async-group; elements outside the tensor are not
 // written.  Callers start it at non-negative coordinates inside the tensor,
@@ -285,8 +306,11 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
 //   [49,52) base offset = 0          [61,64) layout = 2 (SWIZZLE_128B)
 // K-major operand (rows of 64 bf16 = 128 B, 8-row atoms of 1024 B):
 //   SBO = 1024 (next 8-row group), LBO unused (16).
-// MN-major operand (k-rows of 64 MN-contiguous bf16, boxes of 64 k-rows):
-//   LBO = byte distance between 64-wide MN chunks, SBO = 1024 (next 8 k-rows).
+// K-major operand in 64-wide K chunks (rows x 64 each): a K16 step moves the
+//   start address 32 B within a chunk, and to the next chunk every 4 steps.
+// MN-major operand (k-rows of 64 MN-contiguous bf16, one block of BK k-rows
+//   per 64-wide MN chunk): LBO = byte distance between the MN chunks
+//   (BK * 128), SBO = 1024 (next 8 k-rows); a K16 step moves 2048 B.
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
