@@ -117,12 +117,23 @@ constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_RASTER_GN = MUON_TC_RASTER_GN;   // tile-column band width of the non-symmetric raster
 
 struct TileCoord {
-  int prob, mat, tm, tn;
+  int prob, mat, tm;
+  int col0;   // first output column of the tile
 };
 
-// Linear tile index -> (problem, matrix, tile row, tile column).  Symmetric
-// problems enumerate, per tile row I, only the tile columns that reach the
-// upper triangle: J >= I*BM/BN.  A column-major problem walks every tile row
+// A symmetric output's row block I (BM rows) starts its tiles at the
+// 256-block of its rows on the diagonal: the upper form stores nothing left
+// of it, so no tile computes a block that lies wholly below the diagonal.
+template <int BM>
+__host__ __device__ constexpr int sym_col_start(int I) {
+  return kSymBlock * ((I * BM) / kSymBlock);
+}
+
+// Linear tile index -> (problem, matrix, tile row, first column).  Symmetric
+// problems enumerate, per tile row I, the tiles from its diagonal 256-block
+// rightwards (sym_col_start; the last one may reach past N, and its
+// 256-column sub-tiles that lie wholly past N are neither loaded nor
+// multiplied).  A column-major problem walks every tile row
 // of one tile column before the next column (B'X of a wide matrix: the
 // concurrent tiles share few X panels and all of B', which stays in L2, so
 // each operand is read from DRAM about once); the others walk bands of
@@ -139,13 +150,13 @@ __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
   if (q.sym) {
     int I = 0;
     for (;;) {
-      const int cnt = q.tiles_n - (I * BM) / BN;
+      const int c0 = sym_col_start<BM>(I);
+      const int cnt = (q.N - c0 + BN - 1) / BN;
       if (r < cnt) break;
       r -= cnt;
       ++I;
     }
-    tm = I;
-    tn = (I * BM) / BN + r;
+    return {pi, mat, I, sym_col_start<BM>(I) + r * BN};
   } else if (q.col_major) {
     tn = r / q.tiles_m;
     tm = r - tn * q.tiles_m;
@@ -157,7 +168,7 @@ __device__ __forceinline__ TileCoord decode_tile(const TcGemmParams& p, int t) {
     tm = rem / width;
     tn = band * TC_RASTER_GN + (rem - (rem / width) * width);
   }
-  return {pi, mat, tm, tn};
+  return {pi, mat, tm, tn * BN};
 }
 
 __device__ __forceinline__ void record_timeout(unsigned int* status, volatile int* abort_flag) {
@@ -494,7 +505,9 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         const GemmProblem& q = p.prob[tc.prob];
         const int kblocks = (q.K + C::BK - 1) / C::BK;
         const int arow = tc.tm * C::BM + rank * C::A_ROWS;
-        const int brow = tc.tn * C::BN + rank * C::SUB_B_ROWS;   // sub-tile n adds n * TC_BN
+        const int brow = tc.col0 + rank * C::SUB_B_ROWS;   // sub-tile n adds n * TC_BN
+        // 256-column sub-tiles wholly past N are neither loaded nor multiplied
+        const int nact = min(NSUB, (q.N - tc.col0 + TC_BN - 1) / TC_BN);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!sm100::mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) {
             record_timeout(p.status, abort_flag);
@@ -504,7 +517,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           uint8_t* sa = smem + stage * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
           if (!PAIR || rank == 0)
-            sm100::mbar_arrive_expect_tx(&full_bar[stage], (PAIR ? 2 : 1) * C::STAGE_BYTES);
+            sm100::mbar_arrive_expect_tx(&full_bar[stage], (PAIR ? 2 : 1) * (C::A_BYTES + nact * C::SUB_B_BYTES));
           issued_mask |= 1u << stage;
           issued_phase_mask = (issued_phase_mask & ~(1u << stage)) | (phase << stage);
           const int k0 = kb * C::BK;
@@ -537,6 +550,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           load_operand(sa, a_t ? &p.tmA2[tc.prob] : &p.tmA[tc.prob], q.a_mn || a_t, arow, C::A_ROWS);
 #pragma unroll
           for (int n = 0; n < NSUB; ++n) {
+            if (n >= nact) break;
             const int brow_n = brow + n * TC_BN;
             const bool b_t = q.b_sym && (k0 / kSymBlock) < (brow_n / kSymBlock);
             load_operand(sb + n * C::SUB_B_BYTES, b_t ? &p.tmB2[tc.prob] : &p.tmB[tc.prob], q.b_mn || b_t,
@@ -573,7 +587,8 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         const int kblocks = (q.K + C::BK - 1) / C::BK;
         // 256-row blocks of the operand rows (the same for both CTAs of a pair)
         const int ablk = (tc.tm * C::BM) / kSymBlock;
-        const int bblk0 = (tc.tn * C::BN) / kSymBlock;
+        const int bblk0 = tc.col0 / kSymBlock;
+        const int nact = min(NSUB, (q.N - tc.col0 + TC_BN - 1) / TC_BN);   // sub-tiles reaching N
         if (!sm100::mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) {
           record_timeout(p.status, abort_flag);
           break;
@@ -617,6 +632,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
           for (int kk = 0; kk < C::BK / 16; ++kk) {
 #pragma unroll
             for (int n = 0; n < NSUB; ++n) {
+              if (n >= nact) break;
               const uint64_t ad = ad0 + koff(a_mn, kk, C::A_CHUNK_BYTES);
               const uint64_t bd = bd0[n] + koff(bmn[n], kk, C::SUB_B_CHUNK_BYTES);
               const uint32_t dn = d_tmem + static_cast<uint32_t>(n * TC_BN);
@@ -655,7 +671,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       const GemmProblem& q = p.prob[tc.prob];
       const int row0 = tc.tm * C::BM + rank * 128;   // first row this CTA holds
       const int i = row0 + row_in_cta;
-      const int jslice = tc.tn * C::BN + slice * kChunks * 32;
+      const int jslice = tc.col0 + slice * kChunks * 32;
       if (jslice < q.N) epilogue_prefetch<EPI>(p, q, tc.mat, i, jslice, kChunks * 32);
       bool wvec = true;
       if (EPI == EPI_AXPY_UPDATE && i < q.M) {

@@ -748,8 +748,10 @@ muon_status run_gemm(const Ctx& C, const Wave& w, int epi, int k, bool x_in_0) {
       P.tiles_m = (P.M + BM - 1) / BM;
       P.tiles_n = (P.N + BN - 1) / BN;
       if (P.sym) {
+        // per tile row, the tiles from its diagonal 256-block to N (the
+        // kernel's decode_tile enumerates the same)
         int t = 0;
-        for (int I = 0; I < P.tiles_m; ++I) t += P.tiles_n - (I * BM) / BN;
+        for (int I = 0; I < P.tiles_m; ++I) t += (P.N - kSymBlock * ((I * BM) / kSymBlock) + BN - 1) / BN;
         P.tiles_per_mat = t;
       } else {
         P.tiles_per_mat = P.tiles_m * P.tiles_n;
