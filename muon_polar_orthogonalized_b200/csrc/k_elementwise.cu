@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "elt_params.cuh"
+#include "pdl.cuh"
 
 namespace muon {
 
@@ -235,6 +236,8 @@ __device__ __forceinline__ float momentum_chunk(const EltParams& p, const MatRef
 template <bool GBF16>
 __global__ void __launch_bounds__(kEltThreads, kEltMinBlocks)
 momentum_norm_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
     const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
     const long long e0 = static_cast<long long>(blk - r.blk_begin) * kEltChunk;
@@ -335,6 +338,8 @@ __device__ __forceinline__ float rowq_load_regs(const EltParams& p, const MatRef
 template <bool GBF16>
 __global__ void __launch_bounds__(kEltThreads, 3)
 rowq_warp_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int wpb = kEltThreads / 32;
   const bool f32x = p.x_f32 != 0;
@@ -365,6 +370,8 @@ rowq_warp_kernel(const __grid_constant__ EltParams p) {
 template <bool GBF16>
 __global__ void __launch_bounds__(kEltThreads)
 rowq_block_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float row_ss;
   const bool f32x = p.x_f32 != 0;
   for (int row_g = blockIdx.x; row_g < p.total_blocks; row_g += gridDim.x) {
@@ -395,6 +402,8 @@ rowq_block_kernel(const __grid_constant__ EltParams p) {
 template <bool GBF16>
 __global__ void __launch_bounds__(kEltThreads)
 momentum_rowq_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ float4 rowbuf[];  // kRowEqSmemCols / 4 entries at most
   __shared__ float row_ss;
   const bool f32x = p.x_f32 != 0;
@@ -475,6 +484,8 @@ momentum_rowq_kernel(const __grid_constant__ EltParams p) {
 // MuonEq) in fp64 in a fixed order.
 __global__ void __launch_bounds__(kEltThreads)
 norm_finalize_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const MatRef& r = p.mats[blockIdx.x];
   const long long numel = static_cast<long long>(r.rows) * r.cols;
   const int nblk = p.row_eq ? r.rows : static_cast<int>((numel + kEltChunk - 1) / kEltChunk);
@@ -558,6 +569,8 @@ __device__ __forceinline__ void update_chunk(const EltParams& p, const MatRef& r
 template <bool EMIT>
 __global__ void __launch_bounds__(kEltThreads, kEltMinBlocks)
 update_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
     const MatRef& r = p.mats[find_mat(p.mats, p.nmats, blk)];
     update_chunk<EMIT>(p, r, static_cast<long long>(blk - r.blk_begin) * kEltChunk);
@@ -590,6 +603,8 @@ __device__ __forceinline__ void ld_x8(const void* x, long long idx, bool f32, fl
 
 __global__ void __launch_bounds__(kEltThreads)
 normuon_update_kernel(const __grid_constant__ EltParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int wpb = kEltThreads / 32;
   const bool f32x = p.x_f32 != 0;
@@ -742,6 +757,8 @@ __device__ __forceinline__ void sched_scalars(AdamTensor& T, const DevSched* s) 
 template <bool GBF16>
 __global__ void __launch_bounds__(kEltThreads, kAdamMinBlocks)
 adamw_kernel(const __grid_constant__ AdamParams P) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (int blk = blockIdx.x; blk < P.total_blocks; blk += gridDim.x) {
     const int ti = find_tensor(P.t, P.ntensors, blk);
     if (P.sched) {
@@ -762,6 +779,8 @@ adamw_kernel(const __grid_constant__ AdamParams P) {
 // ("Chapter 4: The MuonAdamW Optimizer", trapezoidal schedule).
 __global__ void schedule_advance_kernel(DevSched* s, long long total, double warmup_frac,
                                         double warmdown_frac, double final_frac) {
+  pdl_wait();
+  pdl_launch_dependents();
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   const long long t = s->step + 1;
   const long long step = t - 1;
@@ -784,6 +803,8 @@ constexpr int kReplChunk = kEltThreads * 4 * 4;
 
 __global__ void __launch_bounds__(kEltThreads)
 replicate_kernel(const __grid_constant__ ReplParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
     int mi = 0;
     while (mi + 1 < p.nmats && p.blk_begin[mi + 1] <= blk) ++mi;
@@ -815,6 +836,8 @@ int repl_chunk() { return kReplChunk; }
 template <bool BF16>
 __global__ void __launch_bounds__(kEltThreads)
 reduce_mean_kernel(const __grid_constant__ MeanParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   for (int blk = blockIdx.x; blk < p.total_blocks; blk += gridDim.x) {
     int ti = 0;
     while (ti + 1 < p.ntensors && p.blk_begin[ti + 1] <= blk) ++ti;
@@ -847,21 +870,34 @@ cudaError_t launch_reduce_mean(const MeanParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
   const long long g = static_cast<long long>(sms) * 4;
   const int grid = static_cast<int>(g < p.total_blocks ? g : p.total_blocks);
-  if (p.bf16) reduce_mean_kernel<true><<<grid, kEltThreads, 0, s>>>(p);
-  else reduce_mean_kernel<false><<<grid, kEltThreads, 0, s>>>(p);
+  if (p.bf16) {
+    const cudaError_t le = launch_pdl(reduce_mean_kernel<true>, dim3(grid), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
+  else {
+    const cudaError_t le = launch_pdl(reduce_mean_kernel<false>, dim3(grid), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0 || p.nrep <= 0) return cudaSuccess;
   const long long g = static_cast<long long>(sms) * 4;
-  replicate_kernel<<<static_cast<int>(g < p.total_blocks ? g : p.total_blocks), kEltThreads, 0, s>>>(p);
+  const int rgrid = static_cast<int>(g < p.total_blocks ? g : p.total_blocks);
+  {
+    const cudaError_t le = launch_pdl(replicate_kernel, dim3(rgrid), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
                                     cudaStream_t st) {
-  schedule_advance_kernel<<<1, 32, 0, st>>>(s, total, wu, wd, fin);
+  {
+    const cudaError_t le = launch_pdl(schedule_advance_kernel, dim3(1), dim3(32), 0, st, s, total, wu, wd, fin);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -869,6 +905,8 @@ cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, dou
 // from 1 to final_frac at the last step, total - 1 ("Muon vs AdamW, Lion and
 // Sophia: a fair race", the bake-off's schedule by step).
 __global__ void schedule_cosine_kernel(DevSched* s, long long total, long long warm, double final_frac) {
+  pdl_wait();
+  pdl_launch_dependents();
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   const long long step = s->step;  // 0-based index of the step being taken
   const long long last = total - 1;
@@ -886,7 +924,10 @@ __global__ void schedule_cosine_kernel(DevSched* s, long long total, long long w
 }
 
 cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm, double fin, cudaStream_t st) {
-  schedule_cosine_kernel<<<1, 32, 0, st>>>(s, total, warm, fin);
+  {
+    const cudaError_t le = launch_pdl(schedule_cosine_kernel, dim3(1), dim3(32), 0, st, s, total, warm, fin);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -915,10 +956,16 @@ cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
   if (p.grad_bf16) {
     auto k = momentum_norm_kernel<true>;
-    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   } else {
     auto k = momentum_norm_kernel<false>;
-    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   }
   return cudaGetLastError();
 }
@@ -949,12 +996,18 @@ static cudaError_t launch_rowq(const EltParams& p, int cls, int sms, cudaStream_
   if (cls == 0) {
     auto k = rowq_warp_kernel<GBF16>;
     const int wpb = kEltThreads / 32;
-    k<<<rowq_grid(k, (p.total_blocks + wpb - 1) / wpb, 0, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(rowq_grid(k, (p.total_blocks + wpb - 1) / wpb, 0, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
     return cudaGetLastError();
   }
   if (cls == 1) {
     auto k = rowq_block_kernel<GBF16>;
-    k<<<rowq_grid(k, p.total_blocks, 0, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(rowq_grid(k, p.total_blocks, 0, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
     return cudaGetLastError();
   }
   auto k = momentum_rowq_kernel<GBF16>;
@@ -974,7 +1027,10 @@ static cudaError_t launch_rowq(const EltParams& p, int cls, int sms, cudaStream_
   for (int i = 0; i < p.nmats; ++i)
     if (p.mats[i].vec && p.mats[i].cols <= kRowEqSmemCols && p.mats[i].cols > cols) cols = p.mats[i].cols;
   const size_t smem = static_cast<size_t>((cols + 3) / 4) * sizeof(float4);
-  k<<<rowq_grid(k, p.total_blocks, smem, sms), kEltThreads, smem, s>>>(p);
+  {
+    const cudaError_t le = launch_pdl(k, dim3(rowq_grid(k, p.total_blocks, smem, sms)), dim3(kEltThreads), smem, s, p);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -988,13 +1044,20 @@ cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s) {
   const int wpb = kEltThreads / 32;
   const long long need = (static_cast<long long>(p.total_blocks) + wpb - 1) / wpb;
   const long long cap = static_cast<long long>(sms) * 8;
-  normuon_update_kernel<<<static_cast<int>(need < cap ? need : cap), kEltThreads, 0, s>>>(p);
+  const int ngrid = static_cast<int>(need < cap ? need : cap);
+  {
+    const cudaError_t le = launch_pdl(normuon_update_kernel, dim3(ngrid), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s) {
   if (p.nmats <= 0) return cudaSuccess;
-  norm_finalize_kernel<<<p.nmats, kEltThreads, 0, s>>>(p);
+  {
+    const cudaError_t le = launch_pdl(norm_finalize_kernel, dim3(p.nmats), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   return cudaGetLastError();
 }
 
@@ -1002,10 +1065,16 @@ cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s
   if (p.total_blocks <= 0) return cudaSuccess;
   if (emit) {
     auto k = update_kernel<true>;
-    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   } else {
     auto k = update_kernel<false>;
-    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   }
   return cudaGetLastError();
 }
@@ -1014,10 +1083,16 @@ cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
   if (p.grad_bf16) {
     auto k = adamw_kernel<true>;
-    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   } else {
     auto k = adamw_kernel<false>;
-    k<<<persistent_grid(k, p.total_blocks, sms), kEltThreads, 0, s>>>(p);
+    {
+    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
+    if (le != cudaSuccess) return le;
+  }
   }
   return cudaGetLastError();
 }

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "pdl.cuh"
 
 namespace muon {
 
@@ -31,6 +32,8 @@ __device__ __forceinline__ float cautious_w_f32(float w, float u, float lr, floa
 
 template <int EPI>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const __grid_constant__ SimtGemmParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float As[ST_BK][ST_BM + 1];
   __shared__ float Bs[ST_BK][ST_BN + 1];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -105,10 +108,22 @@ cudaError_t launch_simt_gemm(const SimtGemmParams& p, int epi, int num_sms, cuda
   if (p.total_tiles <= 0) return cudaSuccess;
   const int grid = p.total_tiles < num_sms * 8 ? p.total_tiles : num_sms * 8;
   switch (epi) {
-    case EPI_GRAM: simt_gemm_kernel<EPI_GRAM><<<grid, 256, 0, s>>>(p); break;
-    case EPI_POLY: simt_gemm_kernel<EPI_POLY><<<grid, 256, 0, s>>>(p); break;
-    case EPI_AXPY: simt_gemm_kernel<EPI_AXPY><<<grid, 256, 0, s>>>(p); break;
-    case EPI_AXPY_UPDATE: simt_gemm_kernel<EPI_AXPY_UPDATE><<<grid, 256, 0, s>>>(p); break;
+    case EPI_GRAM: {
+    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_GRAM>, dim3(grid), dim3(256), 0, s, p);
+    if (le != cudaSuccess) return le;
+  } break;
+    case EPI_POLY: {
+    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_POLY>, dim3(grid), dim3(256), 0, s, p);
+    if (le != cudaSuccess) return le;
+  } break;
+    case EPI_AXPY: {
+    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_AXPY>, dim3(grid), dim3(256), 0, s, p);
+    if (le != cudaSuccess) return le;
+  } break;
+    case EPI_AXPY_UPDATE: {
+    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_AXPY_UPDATE>, dim3(grid), dim3(256), 0, s, p);
+    if (le != cudaSuccess) return le;
+  } break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -43,6 +43,7 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "pdl.cuh"
 #include "sm100.cuh"
 
 namespace muon {
@@ -492,6 +493,9 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   if (PAIR) sm100::cluster_sync(); else __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above touched only this CTA's shared memory, TMEM and the
+  // kernel parameters; from here on global memory is read and written
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
@@ -789,6 +793,10 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   __syncwarp();
   if (PAIR) sm100::cluster_sync(); else __syncthreads();
   sm100::tc_fence_after();
+  // every role is done: the next kernel may be scheduled (triggering at the
+  // start would let its blocks sit beside this CTA for the whole kernel,
+  // e.g. AdamW's beside the fused update, and take issue slots from it)
+  pdl_launch_dependents();
   if (warp == 1) {
     __syncwarp();
     if (PAIR) sm100::tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
@@ -830,7 +838,7 @@ static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(TC_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
@@ -853,6 +861,12 @@ static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_
   }
   const int units = p.total_tiles < max_units ? p.total_tiles : max_units;
   cfg.gridDim = dim3((PAIR ? 2 : 1) * units, 1, 1);
+  // programmatic dependent launch (pdl.cuh): the kernel waits for the
+  // previous grid before its first global-memory access
+  attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs += 1;
   e = cudaLaunchKernelEx(&cfg, kern, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
