@@ -3,9 +3,9 @@
 // One quintic iteration ("Chapter 4: The MuonAdamW Optimizer", Polar Express:
 // Newton-Schulz Orthogonalization; "3.9 Optimizers", Muon: Orthogonalizing
 // the Update) is three products:
-//   gram  A = s^2 X X^T          symmetric: only tiles touching the upper
-//                                triangle run, and A is stored in upper form
-//                                (256x256 blocks on and above the diagonal)
+//   gram  A = s^2 X X^T          symmetric: each tile row starts at its
+//                                diagonal 256-block, and A is stored in upper
+//                                form (256x256 blocks on and above the diagonal)
 //   poly  B' = a I + b A + c A A symmetric likewise; A A = A A^T since A is
 //                                symmetric, so both operands are rows of A;
 //                                K blocks left of a row block's diagonal are
@@ -26,14 +26,15 @@
 // only (X0 is stored unscaled; bf16 rounding is scale-free up to exponent).
 //
 // Structure: persistent grouped kernel, one CTA per SM (CTA pairs by
-// default), BK = 64, a TMA -> shared-memory ring, tcgen05.mma kind::f16 (bf16
-// in, fp32 accumulate) issued by one thread into TMEM, and eight epilogue
-// warps that drain TMEM with tcgen05.ld.  Tiles: 256x256 on a CTA pair with
-// two 256-column accumulators (one tile's epilogue overlaps the next tile's
-// MMAs) and a 6-stage ring; the Gram and plain B'X products use 256x512 pair
-// tiles (two N=256 MMAs per K step into one 512-column accumulator, 4-stage
-// ring).
-// Single-CTA mode: 128x256 tiles, 4-stage ring.
+// default), a TMA -> shared-memory ring, tcgen05.mma kind::f16 (bf16 in, fp32
+// accumulate) issued by one thread into TMEM, and eight epilogue warps that
+// drain TMEM with tcgen05.ld.  Tiles: 256x256 on a CTA pair with two
+// 256-column accumulators (one tile's epilogue overlaps the next tile's MMAs)
+// and a 3-stage ring of K = 128; the Gram and plain B'X products use 256x512
+// pair tiles (two N=256 MMAs per K step into one 512-column accumulator,
+// 4-stage ring of K = 64).  Where row lengths allow, each operand block of a
+// stage is one TMA box of a chunked 4-D tensor map.
+// Single-CTA mode: 128x256 tiles, 4-stage ring of K = 64.
 //   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
 //   warps 2-9: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31; two warps
 //              per lane quadrant split the tile's columns)
