@@ -765,6 +765,34 @@ def test_device_timeout_reaches_status_word(dev):
     check_step(hW[0], host64(W[0]), host64(M[0]), rw, rm)
 
 
+def test_dependent_launch_after_and_before_library_kernels(dev):
+    """Every kernel is launched with programmatic dependent launch and waits
+    for the previous grid before touching global memory: gradients produced
+    by a torch kernel right before the step (no synchronisation between) and
+    the parameters read by a torch kernel right after it give the same bits
+    as with a device synchronisation on both sides."""
+    shapes = [(384, 1536), (1536, 384), (100, 300)]
+    res = []
+    for sync in (True, False):
+        groups, W, G, M, _, _ = make_state(dev, shapes, "bf16", 31)
+        ws = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+        torch.cuda.synchronize()
+        for k in range(3):
+            for g in G:          # a library kernel writes every gradient just before the step
+                g.mul_(1.0 + 0.25 * k)
+            if sync:
+                torch.cuda.synchronize()
+            api.muon_step(W, G, M, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws)
+            if sync:
+                torch.cuda.synchronize()
+            snap = [w.clone() for w in W]   # and reads every parameter just after it
+        torch.cuda.synchronize()
+        assert api.muon_query_status(ws) == N.MUON_OK
+        res.append([host64(w) for w in snap] + [host64(m) for m in M])
+    for a, b in zip(*res):
+        assert np.array_equal(a, b)
+
+
 def test_cuda_graph_replay_matches_eager(dev):
     """muon_step launches only stream-ordered work with by-value descriptors, so
     a captured step replays bit-identically to eager calls (fresh gradients
