@@ -63,9 +63,6 @@ namespace muon {
 #ifndef MUON_TC_NARROW_BK
 #define MUON_TC_NARROW_BK 128
 #endif
-#ifndef MUON_TC_WIDE_BK
-#define MUON_TC_WIDE_BK 64
-#endif
 #ifndef MUON_TC_WIDE_STAGES
 #define MUON_TC_WIDE_STAGES 4
 #endif
@@ -96,7 +93,7 @@ struct TcCfg {
   // their bytes (measured: a 32 KB stage moves 44 B/clk as two 16 KB boxes and
   // 57 B/clk as one 32 KB box; a 64 KB stage 78 B/clk as two 32 KB boxes),
   // and a 256x256 pair tile consumes 64 B/clk at the full MMA rate.
-  static constexpr int BK = (PAIR && NSUB == 1) ? MUON_TC_NARROW_BK : NSUB == 2 ? MUON_TC_WIDE_BK : 64;
+  static constexpr int BK = (PAIR && NSUB == 1) ? MUON_TC_NARROW_BK : 64;
   static constexpr int KCH = BK / 64;                // 64-wide K chunks per stage
   static constexpr int MN_CHUNK_BYTES = BK * 128;    // MN-major: one 64-wide MN chunk of BK k-rows
   static constexpr int A_ROWS = 128;                 // A rows staged per CTA
