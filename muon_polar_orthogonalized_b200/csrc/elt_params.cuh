@@ -16,6 +16,7 @@ struct MatRef {
   int rows, cols, ldx;
   int vec;           // 1: 4-wide vector path is legal for this matrix
   int blk_begin;     // first block of this matrix in the launch
+  int item_begin;    // momentum_bulk: first stage item (two chunks) of this matrix
   int sidx;          // index of this matrix's scale in the wave's scale array
   float lr;          // lr * lr_scale (update kernel)
   int pbase;         // MuonEq momentum: index of the first row's partial in `partials`
@@ -25,6 +26,7 @@ struct EltParams {
   MatRef mats[kMaxMatsPerLaunch];
   int nmats;
   int total_blocks;  // work chunks (one partial sum each); blocks loop over them
+  int total_items;   // momentum_bulk: stage items (up to two chunks of one matrix)
   int grid;          // launched blocks (persistent, <= total_blocks)
   int grad_bf16;     // grads of every matrix in this launch are bf16
   int x_f32;         // workspace X is fp32 (debug mode)
@@ -37,6 +39,7 @@ struct EltParams {
   float* partials;   // momentum kernel: one partial sum of squares per block (or row)
   float* scales;     // per-matrix 1/(||m~||+eps)
   const DevSched* sched;  // nullptr, or the device schedule (lr multiplier)
+  unsigned int* status;   // momentum_bulk: status word (a bounded wait ran out)
 };
 
 // ---------------------------------------------------------------- AdamW

@@ -28,6 +28,8 @@ namespace muon {
 int elt_chunk();
 int adam_chunk();
 cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s);
+cudaError_t launch_momentum_bulk(const EltParams& p, int sms, cudaStream_t s);
+int bulk_chunks();
 cudaError_t launch_momentum_rowq(const EltParams& p, int cls, int sms, cudaStream_t s);
 int rowq_class(int cols, bool vec);
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
@@ -505,6 +507,10 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
   std::memset(&P, 0, sizeof(P));
   long long launch_blk0 = 0;  // wave-relative first block of the pending launch
   int pending_dtype = -1;
+  // momentum: the bulk-copy kernel when every matrix of the launch allows it
+  // (momentum present, bf16 X0 of pitch cols, 16-byte aligned G, m and X0,
+  // numel a multiple of 8); it gives the same bits as momentum_norm_kernel
+  bool bulk_ok = true;
   auto flush = [&]() -> muon_status {
     if (P.nmats == 0) return MUON_OK;
     P.beta = a.beta;
@@ -520,7 +526,10 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
     if (kind == 0) {
       P.partials = partials + launch_blk0;
       P.grad_bf16 = pending_dtype == MUON_BF16;
-      e = timed_launch(K_MOMENTUM, a.stream, [&] { return launch_momentum_norm(P, C.dev.sms, a.stream); });
+      P.status = reinterpret_cast<unsigned int*>(a.ws);
+      e = timed_launch(K_MOMENTUM, a.stream, [&] {
+        return bulk_ok ? launch_momentum_bulk(P, C.dev.sms, a.stream) : launch_momentum_norm(P, C.dev.sms, a.stream);
+      });
     } else if (kind == 1) {
       P.partials = partials;
       e = timed_launch(K_NORM, a.stream, [&] { return launch_norm_finalize(P, a.stream); });
@@ -534,6 +543,7 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
     if (e != cudaSuccess) return cuda_fail(e, "elementwise launch");
     launch_blk0 += P.total_blocks;
     std::memset(&P, 0, sizeof(P));
+    bulk_ok = true;
     return MUON_OK;
   };
   long long wave_blk = 0;
@@ -568,6 +578,11 @@ muon_status run_elementwise(const Ctx& C, const Wave& w, int kind) {
         r.vec = c4 && aligned(r.g, ga) && (!r.m || aligned(r.m, 16));
         r.blk_begin = P.total_blocks;
         P.total_blocks += static_cast<int>(q.nblk);
+        const long long numel = static_cast<long long>(q.r) * q.c;
+        bulk_ok = bulk_ok && r.m && !f32 && q.ldc == q.c && numel % 8 == 0 && aligned(r.g, 16) &&
+                  aligned(r.m, 16) && aligned(r.x, 16);
+        r.item_begin = P.total_items;
+        P.total_items += static_cast<int>((q.nblk + bulk_chunks() - 1) / bulk_chunks());
       } else if (kind == 1) {
         r.blk_begin = static_cast<int>(wave_blk);
       } else if (kind == 2) {

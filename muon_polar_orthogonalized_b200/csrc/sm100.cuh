@@ -165,6 +165,21 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
                ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
                : "memory");
 }
+// 1-D bulk copies (no tensor map), for streaming kernels: global -> this
+// CTA's shared memory with completion on an mbarrier as transaction bytes,
+// and shared -> global in the issuing thread's bulk async-group.  Both
+// addresses 16-byte aligned, sizes multiples of 16 bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
 // 32-byte global accesses (one whole sector per lane; the address must be
 // 32-byte aligned).  A warp whose lanes each own one row reads or writes 32
 // rows per instruction, so two 16-byte accesses to the same sector would

@@ -765,6 +765,33 @@ def test_device_timeout_reaches_status_word(dev):
     check_step(hW[0], host64(W[0]), host64(M[0]), rw, rm)
 
 
+def test_bulk_momentum_matches_register_path(dev):
+    """The momentum kernel that streams m and G through shared memory with
+    bulk copies (taken when every matrix of the launch has a multiple of 8
+    elements and X0 rows of pitch cols) and the one that loads them into
+    registers (taken for the whole launch here by adding a 7 x 9 matrix)
+    give the same bits over three steps for the matrices both runs share:
+    momentum, parameters, status.  Shapes cover several matrices per group,
+    an odd number of 2048-element chunks and a ragged last chunk (100 x 328:
+    17 chunks, the last of 32 elements)."""
+    shapes = [(384, 1536), (1536, 384), (256, 1000), (100, 328)]
+    counts = [2, 1, 3, 2]
+    shared = sum(counts)
+    res = []
+    for extra in (False, True):
+        sh = shapes + ([(7, 9)] if extra else [])
+        cn = counts + ([1] if extra else [])
+        groups, W, G, M, _, _ = make_state(dev, sh, "bf16", 41, counts=cn)
+        ws = workspace(api.muon_workspace_size(groups, STEP_FLAGS), dev)
+        for k in range(3):
+            api.muon_step(W, G, M, groups, 0.02, 0.95, 0.01, 5, FIXED, STEP_FLAGS, ws)
+        torch.cuda.synchronize()
+        assert api.muon_query_status(ws) == N.MUON_OK
+        res.append([host64(w) for w in W[:shared]] + [host64(m) for m in M[:shared]])
+    for a, b in zip(*res):
+        assert np.array_equal(a, b)
+
+
 def test_dependent_launch_after_and_before_library_kernels(dev):
     """Every kernel is launched with programmatic dependent launch and waits
     for the previous grid before touching global memory: gradients produced
