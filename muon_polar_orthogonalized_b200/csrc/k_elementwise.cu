@@ -253,7 +253,9 @@ momentum_norm_kernel(const __grid_constant__ EltParams p) {
 // The same update as momentum_norm_kernel, streamed through shared memory by
 // the bulk-copy engine: per stage one thread loads two chunks (4096
 // elements) of m and G into a 3-stage ring and stores the new m and X0 back
-// from it, while all threads compute in shared memory.  With the copies off
+// from it, while all threads compute in shared memory; three blocks per SM
+// (measured in the power-capped step of 32 layers: 15.4-17.3 ms against
+// 19.1-22.8 ms with two blocks of three or four stages or four of two).  With the copies off
 // the load/store units the stream keeps its HBM rate when the SM clock drops
 // under the board's power cap (measured on 16 x 4096^2 bf16 gradients:
 // 6.25-6.30 TB/s at 1275-1374 MHz, against 5.44-5.58 TB/s for
@@ -265,7 +267,14 @@ momentum_norm_kernel(const __grid_constant__ EltParams p) {
 // multiple of 8 elements.
 constexpr int kBulkChunks = 2;                        // chunks per stage
 constexpr int kBulkElems = kBulkChunks * kEltChunk;   // 4096
-constexpr int kBulkStages = 3;
+#ifndef MUON_BULK_STAGES
+#define MUON_BULK_STAGES 3
+#endif
+#ifndef MUON_BULK_BLOCKS
+#define MUON_BULK_BLOCKS 3
+#endif
+constexpr int kBulkStages = MUON_BULK_STAGES;
+constexpr int kBulkBlocks = MUON_BULK_BLOCKS;         // resident blocks per SM
 template <bool GBF16>
 struct BulkCfg {
   static constexpr int GSZ = GBF16 ? 2 : 4;
@@ -275,7 +284,7 @@ struct BulkCfg {
 };
 
 template <bool GBF16>
-__global__ void __launch_bounds__(kEltThreads, 2)
+__global__ void __launch_bounds__(kEltThreads, kBulkBlocks)
 momentum_bulk_kernel(const __grid_constant__ EltParams p) {
   using B = BulkCfg<GBF16>;
   extern __shared__ __align__(128) uint8_t bulk_smem[];
@@ -1146,7 +1155,17 @@ static cudaError_t launch_momentum_bulk_t(const EltParams& p, int sms, cudaStrea
   auto k = momentum_bulk_kernel<GBF16>;
   const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BulkCfg<GBF16>::SMEM);
   if (e != cudaSuccess) return e;
-  const int grid = p.total_items < 2 * sms ? p.total_items : 2 * sms;   // two blocks per SM
+  // as many blocks as are resident at once (three per SM with bf16 grads,
+  // two with the larger fp32 stages): every block stays until the end
+  static int per_sm = 0;   // per instantiation; the same for every device of a node
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kEltThreads, BulkCfg<GBF16>::SMEM) != cudaSuccess || n < 1)
+      n = 1;
+    per_sm = n;
+  }
+  const int cap = per_sm * sms;
+  const int grid = p.total_items < cap ? p.total_items : cap;
   return launch_pdl(k, dim3(grid), dim3(kEltThreads), BulkCfg<GBF16>::SMEM, s, p);
 }
 
