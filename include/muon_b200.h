@@ -313,6 +313,18 @@ muon_status adamw_step_scheduled(const adamw_group* groups, int n_groups,
                                  const muon_schedule_state* state, muon_stream_t stream);
 
 /*
+ * AdamW's failure channel (it takes no caller workspace).  Synchronises
+ * `stream` and returns MUON_ERR_TIMEOUT if, since the previous call, a
+ * bounded device wait inside an adamw_step / adamw_step_scheduled kernel on
+ * the current device ran out (the kernel then stopped without updating the
+ * chunks it had not reached), else MUON_OK; the record is cleared.  The
+ * waits are those of the kernel that streams g, p, m and v through shared
+ * memory with bulk copies, used when every tensor of a launch has a multiple
+ * of 8 elements.
+ */
+muon_status adamw_query_status(muon_stream_t stream);
+
+/*
  * Synchronises `stream`, reads the workspace status word written by the
  * device during the last muon_step / muon_orthogonalize on it, and returns
  * MUON_OK or the recorded error (MUON_ERR_TIMEOUT).

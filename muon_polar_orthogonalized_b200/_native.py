@@ -77,6 +77,7 @@ SIGNATURES = {
                                     c_void_p]),
     "adamw_step_scheduled": (c_int, [POINTER(AdamWGroup), c_int, c_void_p, c_void_p]),
     "muon_query_status": (c_int, [c_void_p, c_void_p]),
+    "adamw_query_status": (c_int, [c_void_p]),
     "muon_selftest_wait_timeout": (c_int, [c_void_p, ctypes.c_uint64, c_void_p]),
     "muon_status_string": (c_char_p, [c_int]),
     "muon_last_error": (c_char_p, []),

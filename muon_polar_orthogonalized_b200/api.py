@@ -300,6 +300,12 @@ def muon_query_status(workspace, stream=None) -> int:
     return int(N.lib().muon_query_status(c_void_p(ws), c_void_p(_stream_handle(stream))))
 
 
+def adamw_query_status(stream=None) -> int:
+    """MUON_ERR_TIMEOUT if a bounded wait in an AdamW kernel on this device ran
+    out since the last call (the record is then cleared), else MUON_OK."""
+    return int(N.lib().adamw_query_status(c_void_p(_stream_handle(stream))))
+
+
 # --------------------------------------------------------------- profiler
 def muon_profiler_enable(on: bool) -> bool:
     return bool(N.lib().muon_profiler_enable(1 if on else 0))

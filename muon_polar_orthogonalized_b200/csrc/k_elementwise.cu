@@ -970,6 +970,143 @@ adamw_kernel(const __grid_constant__ AdamParams P) {
   }
 }
 
+// ------------------------------------------------------------- adamw_bulk
+// The same update as adamw_kernel, streamed through shared memory by the
+// bulk-copy engine like momentum_bulk_kernel: per stage one thread loads a
+// 2048-element chunk of g, p, m and v into a ring and stores p, m and v back
+// from it; every thread updates its elements in place in shared memory with
+// adam_elem, so the results are bitwise those of adamw_kernel.  Used where
+// every tensor of the launch has a multiple of 8 elements.
+#ifndef MUON_ADAM_BULK_STAGES
+#define MUON_ADAM_BULK_STAGES 3
+#endif
+constexpr int kAdamBulkStages = MUON_ADAM_BULK_STAGES;
+template <bool GBF16>
+struct AdamBulkCfg {
+  static constexpr int GSZ = GBF16 ? 2 : 4;
+  static constexpr int P_OFF = 0, M_OFF = kAdamChunk * 4, V_OFF = 2 * kAdamChunk * 4, G_OFF = 3 * kAdamChunk * 4;
+  static constexpr int STAGE = 3 * kAdamChunk * 4 + kAdamChunk * GSZ;
+  static constexpr int SMEM = kAdamBulkStages * STAGE + 64;   // + the stages' mbarriers
+};
+
+// Per device: set when a bounded wait in adamw_bulk_kernel ran out (read and
+// cleared by adamw_query_status; AdamW has no caller workspace).
+__device__ unsigned int g_adamw_status;
+
+template <bool GBF16>
+__global__ void __launch_bounds__(kEltThreads)
+adamw_bulk_kernel(const __grid_constant__ AdamParams P) {
+  using B = AdamBulkCfg<GBF16>;
+  extern __shared__ __align__(128) uint8_t adam_smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(adam_smem + kAdamBulkStages * B::STAGE);
+  __shared__ int abort_flag;
+  struct Item { int ti, ne; long long e0; };
+  __shared__ Item stage_item[kAdamBulkStages];
+  __shared__ int blk_begin[kMaxAdamTensors];   // the tensors' first chunks, searched per chunk
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i < P.ntensors; i += blockDim.x) blk_begin[i] = P.t[i].blk_begin;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < kAdamBulkStages; ++s) sm100::mbar_init(&full[s], 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  const int mine = static_cast<int>(blockIdx.x) < P.total_blocks
+                       ? (P.total_blocks - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x : 0;
+  auto issue = [&](int k) {   // the loading thread only
+    const int blk = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+    int lo = 0, hi = P.ntensors - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (blk_begin[mid] <= blk) lo = mid; else hi = mid - 1;
+    }
+    const AdamTensor& T = P.t[lo];
+    Item t;
+    t.ti = lo;
+    t.e0 = static_cast<long long>(blk - blk_begin[lo]) * kAdamChunk;
+    t.ne = static_cast<int>(T.numel - t.e0 < kAdamChunk ? T.numel - t.e0 : kAdamChunk);
+    const int s = k % kAdamBulkStages;
+    uint8_t* st = adam_smem + s * B::STAGE;
+    stage_item[s] = t;   // published to the other threads by the barrier's arrival
+    const uint32_t ne = static_cast<uint32_t>(t.ne);
+    sm100::mbar_arrive_expect_tx(&full[s], ne * (12 + B::GSZ));
+    sm100::bulk_load(st + B::P_OFF, T.p + t.e0, ne * 4, &full[s]);
+    sm100::bulk_load(st + B::M_OFF, T.m + t.e0, ne * 4, &full[s]);
+    sm100::bulk_load(st + B::V_OFF, T.v + t.e0, ne * 4, &full[s]);
+    sm100::bulk_load(st + B::G_OFF, static_cast<const uint8_t*>(T.g) + t.e0 * B::GSZ, ne * B::GSZ, &full[s]);
+  };
+  if (threadIdx.x == 0)
+    for (int k = 0; k < mine && k < kAdamBulkStages - 1; ++k) issue(k);
+  int next = mine < kAdamBulkStages - 1 ? mine : kAdamBulkStages - 1;   // next chunk to load (every thread tracks it)
+  int k = 0;
+  for (; k < mine; ++k) {
+    const int s = k % kAdamBulkStages;
+    uint8_t* st = adam_smem + s * B::STAGE;
+    const bool got = sm100::mbar_wait(&full[s], static_cast<uint32_t>((k / kAdamBulkStages) & 1), &abort_flag);
+    if (!__syncthreads_and(got)) {   // the same decision in every thread; nothing more is stored
+      if (threadIdx.x == 0) atomicOr(&g_adamw_status, kDevTimeout);
+      break;
+    }
+    const Item t = stage_item[s];
+    AdamTensor T = P.t[t.ti];
+    if (P.sched) sched_scalars(T, P.sched);
+    float* sp = reinterpret_cast<float*>(st + B::P_OFF);
+    float* smv = reinterpret_cast<float*>(st + B::M_OFF);
+    float* svv = reinterpret_cast<float*>(st + B::V_OFF);
+#pragma unroll
+    for (int u = 0; u < kAdamUnroll; ++u) {
+      const int e = (u * kEltThreads + static_cast<int>(threadIdx.x)) * 4;
+      if (e < t.ne) {
+        float4 g;
+        if constexpr (GBF16) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(st + B::G_OFF + e * 2);
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+          const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+          g = make_float4(a.x, a.y, b.x, b.y);
+        } else {
+          g = *reinterpret_cast<const float4*>(st + B::G_OFF + e * 4);
+        }
+        float4 pv = *reinterpret_cast<const float4*>(sp + e);
+        float4 mv = *reinterpret_cast<const float4*>(smv + e);
+        float4 vv = *reinterpret_cast<const float4*>(svv + e);
+        adam_elem(T, g.x, pv.x, mv.x, vv.x);
+        adam_elem(T, g.y, pv.y, mv.y, vv.y);
+        adam_elem(T, g.z, pv.z, mv.z, vv.z);
+        adam_elem(T, g.w, pv.w, mv.w, vv.w);
+        *reinterpret_cast<float4*>(sp + e) = pv;
+        *reinterpret_cast<float4*>(smv + e) = mv;
+        *reinterpret_cast<float4*>(svv + e) = vv;
+      }
+    }
+    sm100::fence_proxy_async_smem();   // the generic-proxy writes above, for the bulk stores
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t ne = static_cast<uint32_t>(t.ne);
+      sm100::bulk_store(T.p + t.e0, sp, ne * 4);
+      sm100::bulk_store(T.m + t.e0, smv, ne * 4);
+      sm100::bulk_store(T.v + t.e0, svv, ne * 4);
+      sm100::bulk_commit_group();
+      if (next < mine) {
+        sm100::bulk_wait_group_read<1>();   // the stage stored one chunk ago may be refilled
+        issue(next);
+      }
+    }
+    if (next < mine) ++next;
+  }
+  if (threadIdx.x == 0) {
+    sm100::bulk_wait_group<0>();   // every store written
+    // after a timeout: loads issued but not consumed land before the block
+    // exits (each wait bounded)
+    for (int j = k; j < next; ++j) {
+      const uint64_t t0 = sm100::globaltimer();
+      while (!sm100::mbar_try_wait(&full[j % kAdamBulkStages], static_cast<uint32_t>((j / kAdamBulkStages) & 1)) &&
+             sm100::globaltimer() - t0 < 100000000ull) {
+      }
+    }
+  }
+}
+
 // ----------------------------------------------------------- schedule
 // step <- step + 1; lr_mult <- trapezoid(step - 1): linear warmup from 0 over
 // int(total*warmup_frac) steps, 1 on the flat part, linear warmdown to
@@ -1301,6 +1438,33 @@ cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s
   }
   }
   return cudaGetLastError();
+}
+
+template <bool GBF16>
+static cudaError_t launch_adamw_bulk_t(const AdamParams& p, int sms, cudaStream_t s) {
+  auto k = adamw_bulk_kernel<GBF16>;
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AdamBulkCfg<GBF16>::SMEM);
+  if (e != cudaSuccess) return e;
+  static int per_sm = 0;   // resident blocks per SM, per instantiation
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kEltThreads, AdamBulkCfg<GBF16>::SMEM) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    per_sm = n;
+  }
+  const int cap = per_sm * sms;
+  const int grid = p.total_blocks < cap ? p.total_blocks : cap;
+  return launch_pdl(k, dim3(grid), dim3(kEltThreads), AdamBulkCfg<GBF16>::SMEM, s, p);
+}
+
+cudaError_t adamw_status_address(unsigned int** addr) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(addr), g_adamw_status);
+}
+
+cudaError_t launch_adamw_bulk(const AdamParams& p, int sms, cudaStream_t s) {
+  if (p.total_blocks <= 0) return cudaSuccess;
+  return p.grad_bf16 ? launch_adamw_bulk_t<true>(p, sms, s) : launch_adamw_bulk_t<false>(p, sms, s);
 }
 
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s) {

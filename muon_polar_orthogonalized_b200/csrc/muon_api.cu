@@ -36,6 +36,8 @@ cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s);
 cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s);
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s);
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s);
+cudaError_t launch_adamw_bulk(const AdamParams& p, int sms, cudaStream_t s);
+cudaError_t adamw_status_address(unsigned int** addr);
 cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s);
 cudaError_t launch_reduce_mean(const MeanParams& p, int sms, cudaStream_t s);
 int repl_chunk();
@@ -1126,13 +1128,20 @@ static muon_status adamw_impl(const adamw_group* groups, int n_groups, int64_t s
     std::memset(&P, 0, sizeof(P));
     P.grad_bf16 = dt;
     P.sched = sched;
+    // the bulk-copy kernel where every tensor of the launch has a multiple of
+    // 8 elements (its chunks' byte counts are then multiples of 16); it gives
+    // the same bits as adamw_kernel
+    bool bulk_ok = true;
     auto flush = [&]() -> muon_status {
       if (P.ntensors == 0) return MUON_OK;
-      cudaError_t e = timed_launch(K_ADAMW, s, [&] { return launch_adamw(P, dev.sms, s); });
+      cudaError_t e = timed_launch(K_ADAMW, s, [&] {
+        return bulk_ok ? launch_adamw_bulk(P, dev.sms, s) : launch_adamw(P, dev.sms, s);
+      });
       if (e != cudaSuccess) return cuda_fail(e, "adamw launch");
       P.ntensors = 0;
       P.total_blocks = 0;
       P.sched = sched;
+      bulk_ok = true;
       return MUON_OK;
     };
     for (int gi = 0; gi < n_groups; ++gi) {
@@ -1156,6 +1165,7 @@ static muon_status adamw_impl(const adamw_group* groups, int n_groups, int64_t s
         T.numel = n;
         T.blk_begin = P.total_blocks;
         T.vec = (n % 4) == 0;
+        bulk_ok = bulk_ok && (n % 8) == 0;
         T.decay = static_cast<float>(1.0 - static_cast<double>(g.lr) * g.wd);
         T.b1 = g.beta1;
         T.omb1 = static_cast<float>(1.0 - b1);
@@ -1232,6 +1242,24 @@ muon_status muon_query_status(const void* workspace, muon_stream_t stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (word & kDevTimeout) return fail(MUON_ERR_TIMEOUT, "a device-side wait ran out of time");
+  return MUON_OK;
+}
+
+muon_status adamw_query_status(muon_stream_t stream) {
+  g_err[0] = '\0';
+  unsigned int* addr = nullptr;
+  cudaError_t e = adamw_status_address(&addr);   // looked up per call: the module may be reloaded
+  if (e != cudaSuccess) return cuda_fail(e, "adamw status address");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int word = 0;
+  e = cudaMemcpyAsync(&word, addr, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && word != 0) {
+    e = cudaMemsetAsync(addr, 0, 4, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "adamw status read");
+  if (word & kDevTimeout) return fail(MUON_ERR_TIMEOUT, "a device-side wait in an AdamW step ran out of time");
   return MUON_OK;
 }
 
