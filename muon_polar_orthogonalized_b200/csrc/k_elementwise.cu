@@ -1205,35 +1205,20 @@ cudaError_t launch_reduce_mean(const MeanParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
   const long long g = static_cast<long long>(sms) * 4;
   const int grid = static_cast<int>(g < p.total_blocks ? g : p.total_blocks);
-  if (p.bf16) {
-    const cudaError_t le = launch_pdl(reduce_mean_kernel<true>, dim3(grid), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  else {
-    const cudaError_t le = launch_pdl(reduce_mean_kernel<false>, dim3(grid), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  const auto k = p.bf16 ? reduce_mean_kernel<true> : reduce_mean_kernel<false>;
+  return launch_pdl(k, dim3(grid), dim3(kEltThreads), 0, s, p);
 }
 
 cudaError_t launch_replicate(const ReplParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0 || p.nrep <= 0) return cudaSuccess;
   const long long g = static_cast<long long>(sms) * 4;
   const int rgrid = static_cast<int>(g < p.total_blocks ? g : p.total_blocks);
-  {
-    const cudaError_t le = launch_pdl(replicate_kernel, dim3(rgrid), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  return launch_pdl(replicate_kernel, dim3(rgrid), dim3(kEltThreads), 0, s, p);
 }
 
 cudaError_t launch_schedule_advance(DevSched* s, long long total, double wu, double wd, double fin,
                                     cudaStream_t st) {
-  {
-    const cudaError_t le = launch_pdl(schedule_advance_kernel, dim3(1), dim3(32), 0, st, s, total, wu, wd, fin);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  return launch_pdl(schedule_advance_kernel, dim3(1), dim3(32), 0, st, s, total, wu, wd, fin);
 }
 
 // step <- step + 1; lr_mult <- linear climb over `warm` steps, then a cosine
@@ -1259,11 +1244,7 @@ __global__ void schedule_cosine_kernel(DevSched* s, long long total, long long w
 }
 
 cudaError_t launch_schedule_cosine(DevSched* s, long long total, long long warm, double fin, cudaStream_t st) {
-  {
-    const cudaError_t le = launch_pdl(schedule_cosine_kernel, dim3(1), dim3(32), 0, st, s, total, warm, fin);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  return launch_pdl(schedule_cosine_kernel, dim3(1), dim3(32), 0, st, s, total, warm, fin);
 }
 
 // ------------------------------------------------------------- launchers
@@ -1315,20 +1296,8 @@ int bulk_chunks() { return kBulkChunks; }
 
 cudaError_t launch_momentum_norm(const EltParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (p.grad_bf16) {
-    auto k = momentum_norm_kernel<true>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  } else {
-    auto k = momentum_norm_kernel<false>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  }
-  return cudaGetLastError();
+  const auto k = p.grad_bf16 ? momentum_norm_kernel<true> : momentum_norm_kernel<false>;
+  return launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
 }
 
 int rowq_class(int cols, bool vec) {
@@ -1357,19 +1326,11 @@ static cudaError_t launch_rowq(const EltParams& p, int cls, int sms, cudaStream_
   if (cls == 0) {
     auto k = rowq_warp_kernel<GBF16>;
     const int wpb = kEltThreads / 32;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(rowq_grid(k, (p.total_blocks + wpb - 1) / wpb, 0, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(rowq_grid(k, (p.total_blocks + wpb - 1) / wpb, 0, sms)), dim3(kEltThreads), 0, s, p);
   }
   if (cls == 1) {
     auto k = rowq_block_kernel<GBF16>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(rowq_grid(k, p.total_blocks, 0, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(rowq_grid(k, p.total_blocks, 0, sms)), dim3(kEltThreads), 0, s, p);
   }
   auto k = momentum_rowq_kernel<GBF16>;
   // the attribute is set once per device; concurrent callers may both set it
@@ -1388,11 +1349,7 @@ static cudaError_t launch_rowq(const EltParams& p, int cls, int sms, cudaStream_
   for (int i = 0; i < p.nmats; ++i)
     if (p.mats[i].vec && p.mats[i].cols <= kRowEqSmemCols && p.mats[i].cols > cols) cols = p.mats[i].cols;
   const size_t smem = static_cast<size_t>((cols + 3) / 4) * sizeof(float4);
-  {
-    const cudaError_t le = launch_pdl(k, dim3(rowq_grid(k, p.total_blocks, smem, sms)), dim3(kEltThreads), smem, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(rowq_grid(k, p.total_blocks, smem, sms)), dim3(kEltThreads), smem, s, p);
 }
 
 cudaError_t launch_momentum_rowq(const EltParams& p, int cls, int sms, cudaStream_t s) {
@@ -1406,38 +1363,18 @@ cudaError_t launch_normuon_update(const EltParams& p, int sms, cudaStream_t s) {
   const long long need = (static_cast<long long>(p.total_blocks) + wpb - 1) / wpb;
   const long long cap = static_cast<long long>(sms) * 8;
   const int ngrid = static_cast<int>(need < cap ? need : cap);
-  {
-    const cudaError_t le = launch_pdl(normuon_update_kernel, dim3(ngrid), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  return launch_pdl(normuon_update_kernel, dim3(ngrid), dim3(kEltThreads), 0, s, p);
 }
 
 cudaError_t launch_norm_finalize(const EltParams& p, cudaStream_t s) {
   if (p.nmats <= 0) return cudaSuccess;
-  {
-    const cudaError_t le = launch_pdl(norm_finalize_kernel, dim3(p.nmats), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  return cudaGetLastError();
+  return launch_pdl(norm_finalize_kernel, dim3(p.nmats), dim3(kEltThreads), 0, s, p);
 }
 
 cudaError_t launch_update(const EltParams& p, bool emit, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (emit) {
-    auto k = update_kernel<true>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  } else {
-    auto k = update_kernel<false>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  }
-  return cudaGetLastError();
+  const auto k = emit ? update_kernel<true> : update_kernel<false>;
+  return launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
 }
 
 template <bool GBF16>
@@ -1469,20 +1406,8 @@ cudaError_t launch_adamw_bulk(const AdamParams& p, int sms, cudaStream_t s) {
 
 cudaError_t launch_adamw(const AdamParams& p, int sms, cudaStream_t s) {
   if (p.total_blocks <= 0) return cudaSuccess;
-  if (p.grad_bf16) {
-    auto k = adamw_kernel<true>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  } else {
-    auto k = adamw_kernel<false>;
-    {
-    const cudaError_t le = launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
-    if (le != cudaSuccess) return le;
-  }
-  }
-  return cudaGetLastError();
+  const auto k = p.grad_bf16 ? adamw_kernel<true> : adamw_kernel<false>;
+  return launch_pdl(k, dim3(persistent_grid(k, p.total_blocks, sms)), dim3(kEltThreads), 0, s, p);
 }
 
 }  // namespace muon

@@ -108,25 +108,12 @@ cudaError_t launch_simt_gemm(const SimtGemmParams& p, int epi, int num_sms, cuda
   if (p.total_tiles <= 0) return cudaSuccess;
   const int grid = p.total_tiles < num_sms * 8 ? p.total_tiles : num_sms * 8;
   switch (epi) {
-    case EPI_GRAM: {
-    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_GRAM>, dim3(grid), dim3(256), 0, s, p);
-    if (le != cudaSuccess) return le;
-  } break;
-    case EPI_POLY: {
-    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_POLY>, dim3(grid), dim3(256), 0, s, p);
-    if (le != cudaSuccess) return le;
-  } break;
-    case EPI_AXPY: {
-    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_AXPY>, dim3(grid), dim3(256), 0, s, p);
-    if (le != cudaSuccess) return le;
-  } break;
-    case EPI_AXPY_UPDATE: {
-    const cudaError_t le = launch_pdl(simt_gemm_kernel<EPI_AXPY_UPDATE>, dim3(grid), dim3(256), 0, s, p);
-    if (le != cudaSuccess) return le;
-  } break;
+    case EPI_GRAM: return launch_pdl(simt_gemm_kernel<EPI_GRAM>, dim3(grid), dim3(256), 0, s, p);
+    case EPI_POLY: return launch_pdl(simt_gemm_kernel<EPI_POLY>, dim3(grid), dim3(256), 0, s, p);
+    case EPI_AXPY: return launch_pdl(simt_gemm_kernel<EPI_AXPY>, dim3(grid), dim3(256), 0, s, p);
+    case EPI_AXPY_UPDATE: return launch_pdl(simt_gemm_kernel<EPI_AXPY_UPDATE>, dim3(grid), dim3(256), 0, s, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace muon
