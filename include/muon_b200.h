@@ -52,7 +52,7 @@ typedef struct CUstream_st* muon_stream_t;
 typedef enum {
   MUON_OK = 0,
   MUON_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, bad scalar, misaligned pointer */
-  MUON_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run (no sm_100 device, ...) */
+  MUON_ERR_UNSUPPORTED = 2,  /* valid request this library cannot run (no sm_100 device, ...) */
   MUON_ERR_WORKSPACE = 3,    /* workspace null, misaligned or smaller than muon_workspace_min_size */
   MUON_ERR_CUDA = 4,         /* a CUDA runtime/driver call or kernel launch failed */
   MUON_ERR_TIMEOUT = 5       /* a device-side bounded wait ran out (status word) */

@@ -353,7 +353,7 @@ def update_pin_failures(upd):
     w = rng.standard_normal((6, 7))
     u = rng.standard_normal((6, 7))
     lr, wd = 0.02, 0.1
-    # no decay: W -= lr * update  (the spec form)
+    # no decay: W -= lr * update  (the plain update form)
     if _rel(upd(w, u, lr, 0.0, True), w - lr * u) > 1e-15:
         fails.append("no_decay")
     # plain decoupled decay as "Chapter 4 / The Full Muon Step" sequences it:
