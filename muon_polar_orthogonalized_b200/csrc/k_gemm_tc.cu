@@ -27,17 +27,19 @@
 //
 // Structure: persistent grouped kernel, one CTA per SM (CTA pairs by
 // default), a TMA -> shared-memory ring, tcgen05.mma kind::f16 (bf16 in, fp32
-// accumulate) issued by one thread into TMEM, and eight epilogue warps that
-// drain TMEM with tcgen05.ld.  Tiles: 256x256 on a CTA pair with two
-// 256-column accumulators (one tile's epilogue overlaps the next tile's MMAs)
-// and a 3-stage ring of K = 128; the Gram and plain B'X products use 256x512
+// accumulate) issued by one thread into TMEM, and eight (fused update:
+// twelve) epilogue warps that drain TMEM with tcgen05.ld.  Tiles: 256x256 on
+// a CTA pair with two 256-column accumulators (one tile's epilogue overlaps
+// the next tile's MMAs) and a 3-stage ring of K = 128; the Gram and plain B'X
+// products use 256x512
 // pair tiles (two N=256 MMAs per K step into one 512-column accumulator,
 // 4-stage ring of K = 64).  Where row lengths allow, each operand block of a
 // stage is one TMA box of a chunked 4-D tensor map.
 // Single-CTA mode: 128x256 tiles, 4-stage ring of K = 64.
 //   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
 //   warps 2-9: epilogue (warp w reads TMEM lanes 32*(w%4) .. +31; two warps
-//              per lane quadrant split the tile's columns)
+//              per lane quadrant split the tile's columns); the fused
+//              update has warps 2-13, three per quadrant
 // No TMA or bulk load uses multicast; the only multicast is the
 // tcgen05.commit that signals an mbarrier in both CTAs of a pair.
 #include <cuda_bf16.h>
@@ -73,16 +75,35 @@ namespace muon {
 #ifndef MUON_TC_EPI_WARPS
 #define MUON_TC_EPI_WARPS 8
 #endif
-// Epilogue warps: a multiple of 4, since warp w may only read TMEM lanes
-// 32*(w%4) .. +31; with 8, two warps share each lane quadrant and split the
-// tile's 256 columns between them.
-constexpr int TC_EPI_WARPS = MUON_TC_EPI_WARPS;
-constexpr int TC_EPI_SPLIT = TC_EPI_WARPS / 4;          // column slices per lane quadrant
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;       // producer + MMA + epilogue warps
+#ifndef MUON_TC_UPD_EPI_WARPS
+#define MUON_TC_UPD_EPI_WARPS 12
+#endif
+#ifndef MUON_TC_POLY_EPI_WARPS
+#define MUON_TC_POLY_EPI_WARPS 8
+#endif
 // Output staging for the TMA row stores: per epilogue warp two 2 KB buffers of
 // 32 rows x 32 bf16 (64-byte swizzle), used alternately.
 constexpr int TC_STAGE_TILE_BYTES = 32 * 32 * 2;
-constexpr int TC_STAGING_BYTES = TC_EPI_WARPS * 2 * TC_STAGE_TILE_BYTES;
+// Epilogue warps: a multiple of 4, since warp w may only read TMEM lanes
+// 32*(w%4) .. +31; the warps of a lane quadrant split the tile's 32-column
+// chunks between them.  Eight by default (two per quadrant).  The fused
+// update's epilogue (W read, masked, written per element) is the longer one:
+// where K is short it outlasts the next tile's MMAs, so it gets twelve (three
+// per quadrant), which its registers and shared memory allow (it stores from
+// registers and needs no staging).
+template <int EPI, int NSUB>
+struct EpiCfg {
+  static constexpr int WARPS = (EPI == EPI_AXPY_UPDATE && NSUB == 1) ? MUON_TC_UPD_EPI_WARPS
+                               : (EPI == EPI_POLY && NSUB == 1)      ? MUON_TC_POLY_EPI_WARPS
+                                                                     : MUON_TC_EPI_WARPS;
+  static constexpr int SPLIT = WARPS / 4;                    // warps per lane quadrant
+  static constexpr int THREADS = 64 + 32 * WARPS;            // producer + MMA + epilogue warps
+  static constexpr bool STAGED = (EPI == EPI_GRAM || EPI == EPI_AXPY);   // rows leave by TMA stores
+  static constexpr int STAGING_BYTES = STAGED ? WARPS * 2 * TC_STAGE_TILE_BYTES : 0;
+  static constexpr int NCH = 256 * NSUB / 32;                // 32-column chunks per tile row
+  static constexpr int MAX_CH = (NCH + SPLIT - 1) / SPLIT;   // most chunks one warp takes
+  static_assert(WARPS % 4 == 0 && WARPS >= 4 && WARPS <= 16, "epilogue warps");
+};
 template <bool PAIR, int NSUB>
 struct TcCfg {
   static_assert(NSUB == 1 || (PAIR && NSUB == 2), "512-column tiles need CTA pairs");
@@ -110,9 +131,9 @@ struct TcCfg {
   static_assert(kSymBlock % BK == 0, "a K block lies inside one 256-block of an upper-form operand");
   static constexpr int ACC_BUFS = NSUB == 1 ? 2 : 1;   // TMEM accumulators (512 columns in all)
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;          // barriers, TMEM slot, abort flag
-  static constexpr int STAGING_OFF = BAR_OFF + 1024;            // output staging (TC_STAGING_BYTES)
-  static constexpr int SMEM_BYTES = STAGING_OFF + TC_STAGING_BYTES + 1024 /*align slack*/;
-  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+  static constexpr int STAGING_OFF = BAR_OFF + 1024;            // output staging (EpiCfg::STAGING_BYTES)
+  template <int EPI>
+  static constexpr int smem_bytes() { return STAGING_OFF + EpiCfg<EPI, NSUB>::STAGING_BYTES + 1024 /*align slack*/; }
 };
 constexpr int TC_BN = 256;   // columns of one MMA (N) and of a narrow tile
 constexpr int TC_TMEM_COLS = 512;
@@ -445,9 +466,11 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
 }
 
 template <int EPI, bool PAIR, int NSUB>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(EpiCfg<EPI, NSUB>::THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   using C = TcCfg<PAIR, NSUB>;
+  using E = EpiCfg<EPI, NSUB>;
+  static_assert(C::template smem_bytes<EPI>() <= 232448, "shared memory per block");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -471,7 +494,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     }
     for (int b = 0; b < 2; ++b) {
       sm100::mbar_init(&tfull_bar[b], 1);
-      sm100::mbar_init(&tempty_bar[b], (PAIR ? 2 : 1) * TC_EPI_WARPS);   // one arrival per epilogue warp
+      sm100::mbar_init(&tempty_bar[b], (PAIR ? 2 : 1) * E::WARPS);   // one arrival per epilogue warp
     }
     *abort_flag = 0;
     sm100::fence_mbar_init();
@@ -665,9 +688,11 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
     // ----------------------------------------------------------- epilogue
     const int quad = warp & 3;                          // TMEM lane quadrant this warp may read
     const int slice = (warp - 2) / 4;                   // which column slice of the tile
-    constexpr int kChunks = C::BN / 32 / TC_EPI_SPLIT;  // 32-column chunks per warp
+    constexpr int kChunks = E::MAX_CH;                  // 32-column chunks per warp, at most
+    const int ch0 = slice * E::NCH / E::SPLIT;          // this warp's chunks: [ch0, ch0 + nch)
+    const int nch = (slice + 1) * E::NCH / E::SPLIT - ch0;
     const int row_in_cta = quad * 32 + lane;
-    uint8_t* my_staging = staging + (warp - 2) * 2 * TC_STAGE_TILE_BYTES;
+    uint8_t* my_staging = staging + (warp - 2) * 2 * TC_STAGE_TILE_BYTES;   // used when E::STAGED
     int stage_ctr = 0;   // staging buffer in use: stage_ctr & 1
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -676,8 +701,8 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       const GemmProblem& q = p.prob[tc.prob];
       const int row0 = tc.tm * C::BM + rank * 128;   // first row this CTA holds
       const int i = row0 + row_in_cta;
-      const int jslice = tc.col0 + slice * kChunks * 32;
-      if (jslice < q.N) epilogue_prefetch<EPI>(p, q, tc.mat, i, jslice, kChunks * 32);
+      const int jslice = tc.col0 + ch0 * 32;
+      if (jslice < q.N) epilogue_prefetch<EPI>(p, q, tc.mat, i, jslice, nch * 32);
       bool wvec = true;
       if (EPI == EPI_AXPY_UPDATE && i < q.M) {
         const int wi = q.w_first + tc.mat;
@@ -694,7 +719,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       // symmetric output in upper form: chunks left of the rows' 256-block are not stored
       const int rblk = row0 / kSymBlock;
       int c_hi = 0;
-      if (jslice < q.N) c_hi = min(kChunks, (q.N - jslice + 31) / 32);
+      if (jslice < q.N) c_hi = min(nch, (q.N - jslice + 31) / 32);
       int c_lo = 0;
       if (q.sym) c_lo = max(0, (kSymBlock * rblk - jslice) / 32);
       auto chunk_j0 = [&](int cc) { return jslice + cc * 32; };
@@ -742,7 +767,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * C::BN);
       auto tmem_req = [&](int cc, uint32_t (&r)[32]) {
-        sm100::tmem_ld32_async(t_row + static_cast<uint32_t>((slice * kChunks + cc) * 32), r);
+        sm100::tmem_ld32_async(t_row + static_cast<uint32_t>((ch0 + cc) * 32), r);
       };
       auto process = [&](int cc, const EpiIn& in) {
         const int j0 = chunk_j0(cc);
@@ -834,14 +859,15 @@ int tc_bk(bool pair, bool wide) {
 template <int EPI, bool PAIR, int NSUB>
 static cudaError_t launch_tc_epi(const TcGemmParams& p, int num_sms, cudaStream_t s) {
   using C = TcCfg<PAIR, NSUB>;
+  constexpr int kSmem = C::template smem_bytes<EPI>();
   auto kern = tc_gemm_kernel<EPI, PAIR, NSUB>;
   static thread_local int max_units = 0;   // co-resident tile units (CTAs or CTA pairs)
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
-  cfg.blockDim = dim3(TC_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.blockDim = dim3(EpiCfg<EPI, NSUB>::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   if (PAIR) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
