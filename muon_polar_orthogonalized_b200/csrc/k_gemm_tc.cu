@@ -144,6 +144,16 @@ struct TileCoord {
   int col0;   // first output column of the tile
 };
 
+// Columns one MMA of a tile computes: 256, or 128 for a 256-column tile
+// (one sub-tile) of which at most 128 columns lie inside N (the ragged last
+// tile column of a width that is an odd multiple of 128, e.g. 1664).  Such a
+// tile runs N = 128 MMAs, half the work; with CTA pairs each CTA then stages
+// 64 rows of B, so the second CTA's B rows start 64 (not 128) past col0.
+template <int NSUB>
+__device__ __forceinline__ int mma_cols(const GemmProblem& q, const TileCoord& tc) {
+  return (NSUB == 1 && q.N - tc.col0 <= TC_BN / 2) ? TC_BN / 2 : TC_BN;
+}
+
 // A symmetric output's row block I (BM rows) starts its tiles at the
 // 256-block of its rows on the diagonal: the upper form stores nothing left
 // of it, so no tile computes a block that lies wholly below the diagonal.
@@ -533,7 +543,9 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
         const GemmProblem& q = p.prob[tc.prob];
         const int kblocks = (q.K + C::BK - 1) / C::BK;
         const int arow = tc.tm * C::BM + rank * C::A_ROWS;
-        const int brow = tc.col0 + rank * C::SUB_B_ROWS;   // sub-tile n adds n * TC_BN
+        // B rows this CTA stages (sub-tile n adds n * TC_BN): half of the
+        // MMA's columns per CTA of a pair
+        const int brow = tc.col0 + rank * (C::SUB_B_ROWS * mma_cols<NSUB>(q, tc) / TC_BN);
         // 256-column sub-tiles wholly past N are neither loaded nor multiplied
         const int nact = min(NSUB, (q.N - tc.col0 + TC_BN - 1) / TC_BN);
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -647,7 +659,7 @@ tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
             bmn[n] = q.b_mn || (q.b_sym && kblk < bblk0 + (n * TC_BN) / kSymBlock);
             const uint32_t sbn = sb + n * C::SUB_B_BYTES;
             bd0[n] = bmn[n] ? sm100::make_sdesc(sbn, C::MN_CHUNK_BYTES, 1024) : sm100::make_sdesc(sbn, 16, 1024);
-            idn[n] = sm100::make_idesc_bf16(C::BM, TC_BN, a_mn ? 1 : 0, bmn[n] ? 1 : 0);
+            idn[n] = sm100::make_idesc_bf16(C::BM, mma_cols<NSUB>(q, tc), a_mn ? 1 : 0, bmn[n] ? 1 : 0);
           }
           // start-address step (16-byte units) of K16 step kk: MN-major 2048 B
           // per step; K-major 32 B per step within a 64-wide chunk, then the
