@@ -265,6 +265,27 @@ __device__ __forceinline__ void stage_row_store(const CUtensorMap* tmap, uint8_t
   }
 }
 
+// The same update for two neighbouring elements, with packed fp32 arithmetic
+// (fma.rn.f32x2: per lane the same rounding as fmaf, so the same bits).  The
+// mask drops cautious_w's w == 0 test: where w = +-0, wd*w + u is u for any
+// u != 0, and u == 0 keeps the mask on anyway, so the result is unchanged.
+// u0, u1: bf16(v0), bf16(v1) from one packed conversion.
+__device__ __forceinline__ float2 cautious_w2(float2 w, float v0, float v1, float lr, float wd, bool cautious) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v0, v1);
+  const uint32_t bits = *reinterpret_cast<const uint32_t*>(&b);
+  const float2 u = make_float2(__uint_as_float(bits << 16), __uint_as_float(bits & 0xffff0000u));
+  const float2 t = __ffma2_rn(make_float2(wd, wd), w, u);   // decayed
+  float2 tm = t;
+  if (cautious) {
+    // decay off where the signs differ and u != 0
+    const bool off0 = ((__float_as_int(u.x) ^ __float_as_int(w.x)) < 0) && (u.x != 0.f);
+    const bool off1 = ((__float_as_int(u.y) ^ __float_as_int(w.y)) < 0) && (u.y != 0.f);
+    tm.x = off0 ? u.x : t.x;
+    tm.y = off1 ? u.y : t.y;
+  }
+  return __ffma2_rn(make_float2(-lr, -lr), tm, w);
+}
+
 __device__ __forceinline__ float cautious_w(float w, float u, float lr, float wd, bool cautious) {
   bool mask = true;
   if (cautious) {
@@ -415,8 +436,13 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
     }
   } else {
     // Gram: s^2 on the first iteration; axpy: s on the first iteration
+    // (packed: the same product per element)
 #pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] *= f;
+    for (int c = 0; c < 32; c += 2) {
+      const float2 r = __fmul2_rn(make_float2(v[c], v[c + 1]), make_float2(f, f));
+      v[c] = r.x;
+      v[c + 1] = r.y;
+    }
   }
 
   if constexpr (EPI == EPI_AXPY_UPDATE) {
@@ -431,12 +457,10 @@ __device__ __forceinline__ void epilogue_store(const TcGemmParams& p, const Gemm
       float4 nw[8];
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
-        float4 ww = win.w[c4];
-        ww.x = cautious_w(ww.x, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 0])), lr, p.wd, cautious);
-        ww.y = cautious_w(ww.y, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 1])), lr, p.wd, cautious);
-        ww.z = cautious_w(ww.z, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 2])), lr, p.wd, cautious);
-        ww.w = cautious_w(ww.w, __bfloat162float(__float2bfloat16_rn(v[c4 * 4 + 3])), lr, p.wd, cautious);
-        nw[c4] = ww;
+        const float4 ww = win.w[c4];
+        const float2 lo = cautious_w2(make_float2(ww.x, ww.y), v[c4 * 4 + 0], v[c4 * 4 + 1], lr, p.wd, cautious);
+        const float2 hi = cautious_w2(make_float2(ww.z, ww.w), v[c4 * 4 + 2], v[c4 * 4 + 3], lr, p.wd, cautious);
+        nw[c4] = make_float4(lo.x, lo.y, hi.x, hi.y);
       }
       // W and each copy: 32-byte stores where the row segment is 32-byte aligned
       auto store_row = [&](float* dst) {
