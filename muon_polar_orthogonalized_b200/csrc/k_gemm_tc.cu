@@ -31,9 +31,8 @@
 // twelve) epilogue warps that drain TMEM with tcgen05.ld.  Tiles: 256x256 on
 // a CTA pair with two 256-column accumulators (one tile's epilogue overlaps
 // the next tile's MMAs) and a 3-stage ring of K = 128; the Gram and plain B'X
-// products use 256x512
-// pair tiles (two N=256 MMAs per K step into one 512-column accumulator,
-// 4-stage ring of K = 64).  Where row lengths allow, each operand block of a
+// products use 256x512 pair tiles (two N=256 MMAs per K step into one
+// 512-column accumulator, 4-stage ring of K = 64).  Where row lengths allow, each operand block of a
 // stage is one TMA box of a chunked 4-D tensor map.
 // Single-CTA mode: 128x256 tiles, 4-stage ring of K = 64.
 //   warp 0: TMA producer        warp 1: MMA issuer (+ TMEM owner)
