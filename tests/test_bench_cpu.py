@@ -136,3 +136,24 @@ def test_cpu_baseline_median_and_spread():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1
     assert cb["spread_ms"][0] <= cb["value"] <= cb["spread_ms"][1]
     assert cb["extrapolated"] is False   # one matrix and one AdamW tensor: the sample is the step
+
+
+def test_profile_summary_quotes_the_captured_traffic():
+    """The committed ncu summary the bench's DRAM-traffic figure comes from
+    names the same source fingerprint and per-layer bytes (the sum of its
+    B'X launches' DRAM reads and writes) as bench.TRAFFIC_CAPTURES."""
+    import re
+    cap = bench.TRAFFIC_CAPTURES["ns_axpy"]
+    text = open(os.path.join(bench.ROOT, "profiles", "tc_gemm_pair_llama_8b_1layer.md")).read()
+    assert f"`{cap['sha']}`" in text.split("Command")[0]
+    per_layer = cap["bytes_per_pass"]["llama_8b_1layer"]
+    assert f"{per_layer:,}" in text
+    rows = [ln for ln in text.splitlines() if ln.startswith("| ns_axpy")]
+    assert len(rows) == 2
+    moved = 0
+    for ln in rows:
+        cells = [c.strip() for c in ln.strip("|").split("|")]
+        for c in cells[4:6]:
+            m = re.match(r"([0-9][0-9,]*)", c)
+            moved += int(m.group(1).replace(",", ""))
+    assert moved == per_layer
